@@ -1,0 +1,119 @@
+"""fp64 CPU oracle of the LSE-weighted merge -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+arm of ``bench.py`` may import this package.  The product path
+(``lse_weighted_merge_b200``) never imports it and shares no code with it.
+
+The arithmetic lives in ``lse_merge_oracle.c`` (plain C, fp64), which states
+the merge of the page "[flashinfer] FlashInfer의 Context-Parallel Decode
+최적화: Fused A2A + LSE Reduce", sections "들어가며" and "코드 분석 / 1. Fused
+Kernel 구현".  This module only compiles that file with gcc and marshals numpy
+arrays into it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "lse_merge_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+# Element types, numbered like the public C-ABI (defined again here on purpose).
+F32, F16, BF16 = 0, 1, 2
+
+
+def build(out_path: str = LIB, mutant: int = 0) -> str:
+    """Compile the oracle with gcc (optionally with one planted mistake)."""
+    cmd = ["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-fno-fast-math",
+           SRC, "-o", out_path, "-lm"]
+    if mutant:
+        cmd.insert(1, f"-DORACLE_MUTANT={int(mutant)}")
+    subprocess.run(cmd, check=True)
+    return out_path
+
+
+def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.oracle_widen.restype = ctypes.c_double
+    lib.oracle_widen.argtypes = [ctypes.c_uint32, ctypes.c_int]
+    lib.oracle_lse_merge.restype = ctypes.c_int
+    lib.oracle_lse_merge.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, i64p, i64p, ctypes.c_int, dp, dp]
+    lib.oracle_attention_shard.restype = None
+    lib.oracle_attention_shard.argtypes = [
+        dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+        ctypes.c_int, dp, dp]
+    lib.oracle_mutant.restype = ctypes.c_int
+    return lib
+
+
+_cached: dict[str, ctypes.CDLL] = {}
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the oracle library, building it first if it is missing or stale."""
+    path = path or LIB
+    if path in _cached:
+        return _cached[path]
+    if path == LIB and (not os.path.exists(LIB)
+                        or os.path.getmtime(LIB) < os.path.getmtime(SRC)):
+        build(LIB)
+    lib = _bind(ctypes.CDLL(path))
+    _cached[path] = lib
+    return lib
+
+
+def widen(bits: int, dtype: int, lib: ctypes.CDLL | None = None) -> float:
+    return (lib or load()).oracle_widen(int(bits), int(dtype))
+
+
+def merge(partial_o: np.ndarray, partial_lse: np.ndarray, R: int, B: int, H: int,
+          D: int, o_strides, lse_strides, in_dtype: int,
+          lib: ctypes.CDLL | None = None):
+    """Run the fp64 merge.
+
+    partial_o: a flat numpy buffer holding the raw elements (uint16 bit
+    patterns for F16/BF16, float32 for F32); partial_lse: flat float32.
+    Strides are (r, b, h) in elements; the d stride is 1.
+    Returns (out [B, H, D] float64, out_lse [B, H] float64).
+    """
+    lib = lib or load()
+    po = np.ascontiguousarray(partial_o)
+    pl = np.ascontiguousarray(partial_lse, dtype=np.float32)
+    want = np.float32 if in_dtype == F32 else np.uint16
+    if po.dtype != want:
+        raise TypeError(f"partial_o must be {np.dtype(want).name} for dtype {in_dtype}")
+    os_ = (ctypes.c_int64 * 3)(*[int(s) for s in o_strides])
+    ls_ = (ctypes.c_int64 * 3)(*[int(s) for s in lse_strides])
+    out = np.empty((B, H, D), dtype=np.float64)
+    out_lse = np.empty((B, H), dtype=np.float64)
+    rc = lib.oracle_lse_merge(
+        po.ctypes.data, pl.ctypes.data, R, B, H, D, os_, ls_, in_dtype,
+        out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+        out_lse.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    if rc != 0:
+        raise ValueError(f"oracle_lse_merge returned {rc}")
+    return out, out_lse
+
+
+def attention_shard(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                    begin: int, end: int, lib: ctypes.CDLL | None = None):
+    """Softmax attention of q [D] over keys [begin, end) of k, v [L, D] (fp64)."""
+    lib = lib or load()
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    L, D = k.shape
+    o = np.empty(D, dtype=np.float64)
+    lse = np.empty(1, dtype=np.float64)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.oracle_attention_shard(q.ctypes.data_as(dp), k.ctypes.data_as(dp),
+                               v.ctypes.data_as(dp), L, D, float(scale), begin, end,
+                               o.ctypes.data_as(dp), lse.ctypes.data_as(dp))
+    return o, float(lse[0])
