@@ -1,0 +1,150 @@
+/*
+ * lse_merge.h -- C ABI of the B200 (sm_100a) LSE-weighted merge.
+ *
+ * The operation.  Under context-parallel decode the KV cache is split along
+ * the sequence into R shards; attention over shard r yields a partial output
+ * o_r[D] and lse_r, the natural-log log-sum-exp of that shard's scores (page
+ * "[flashinfer] FlashInfer의 Context-Parallel Decode 최적화: Fused A2A + LSE
+ * Reduce", section "들어가며").  The merge combines the R partials of every
+ * (b, h) row into the output of attention over the whole sequence: weights
+ * from the lse values, fp32 accumulation over the partial axis, division by
+ * the sum of the weights, conversion to the output type (same page, section
+ * "코드 분석 / 1. Fused Kernel 구현", its Before/After snippet and the fused
+ * kernel's steps 2 and 3).  Per row:
+ *
+ *     m       = max_r lse_r
+ *     e_r     = exp(lse_r - m)          (0 when lse_r = -inf: an empty shard)
+ *     out[d]  = sum_r e_r * o_r[d] / sum_r e_r
+ *     out_lse = m + log(sum_r e_r)
+ *
+ * and out = 0, out_lse = -inf for a row whose shards are all empty.  The
+ * partial rows of an empty shard do not reach the result (NaN there does not
+ * leak).  lse = +inf or NaN is outside the domain; NaN then propagates.
+ *
+ * Everything runs on the GPU inside one kernel launch per call; the library
+ * allocates nothing, keeps no pointer after returning, never synchronises
+ * the host, and only enqueues work on `stream`, so a call can be captured in
+ * a CUDA graph.
+ */
+#ifndef LSE_MERGE_H
+#define LSE_MERGE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types of partial_o and out_o.  lse values are always fp32. */
+typedef enum {
+    LSE_MERGE_F32 = 0,
+    LSE_MERGE_F16 = 1,   /* IEEE binary16 */
+    LSE_MERGE_BF16 = 2   /* bfloat16 */
+} lse_merge_dtype;
+
+/* The same type as cudaStream_t; declared here so that this header needs no
+ * CUDA header.  NULL is the legacy default stream. */
+typedef struct CUstream_st* lse_merge_stream_t;
+
+/* Element (not byte) strides of the two inputs along r, b and h.  The d
+ * stride of partial_o is 1.  All strides must be >= 0.  Examples with dense
+ * storage:
+ *   partial_o [B,H,R,D], partial_lse [B,H,R]:  o = {D, H*R*D, R*D},  lse = {1, H*R, R}
+ *   partial_o [R,B,H,D], partial_lse [R,B,H]:  o = {B*H*D, H*D, D},  lse = {B*H, H, 1}  */
+typedef struct {
+    int64_t o_r, o_b, o_h;
+    int64_t lse_r, lse_b, lse_h;
+} lse_merge_strides;
+
+/* Return codes.  No error is ever reported by a device trap or by an
+ * exception crossing the ABI. */
+#define LSE_MERGE_OK 0
+#define LSE_MERGE_EDTYPE (-1)   /* in_dtype / out_dtype not one of lse_merge_dtype */
+#define LSE_MERGE_EDIMS (-2)    /* R, B, H or D < 1, or the extents overflow */
+#define LSE_MERGE_ENULL (-3)    /* a required pointer is NULL */
+#define LSE_MERGE_ESTRIDE (-4)  /* a negative stride */
+#define LSE_MERGE_EALIAS (-5)   /* an output overlaps an input or the other output */
+#define LSE_MERGE_ELAUNCH (-6)  /* the CUDA launch failed (see lse_merge_last_cuda_error) */
+#define LSE_MERGE_EALIGN (-7)   /* a pointer not aligned to its element size */
+#define LSE_MERGE_EPATH (-8)    /* the requested path cannot take these arguments */
+
+/* Kernel paths.  AUTO picks one from the sizes, dtypes and alignment. */
+#define LSE_MERGE_PATH_AUTO 0
+#define LSE_MERGE_PATH_VECTOR 1   /* 16-byte vector loads, many CTAs (throughput) */
+#define LSE_MERGE_PATH_LATENCY 2  /* the vector kernel as one small CTA (tiny B*H) */
+#define LSE_MERGE_PATH_SCALAR 3   /* element loads, any alignment of strides and D */
+
+/*
+ * Merge R partials of B*H rows.
+ *
+ *   partial_o    device pointer, element (r,b,h,d) at
+ *                r*o_r + b*o_b + h*o_h + d (elements of in_dtype)
+ *   partial_lse  device pointer, element (r,b,h) at r*lse_r + b*lse_b + h*lse_h
+ *   R, B, H, D   partials per row, batch, heads, head dimension; all >= 1
+ *   strides      as above; NULL means dense [B,H,R,D] / [B,H,R]
+ *   in_dtype     element type of partial_o (lse_merge_dtype)
+ *   out_dtype    element type of out_o (lse_merge_dtype)
+ *   out_o        device pointer, dense [B,H,D] of out_dtype, written
+ *   out_lse      device pointer, dense [B,H] fp32, written
+ *   stream       CUDA stream the kernel is enqueued on
+ *
+ * The caller owns every buffer.  Pointers must be aligned to their element
+ * size; the fast path additionally wants 16-byte aligned partial_o rows and
+ * falls back to the scalar kernel otherwise.  Outputs must not overlap the
+ * inputs or each other.  Returns LSE_MERGE_OK, or a negative code with
+ * nothing enqueued (argument errors) or after a failed launch (ELAUNCH).
+ */
+int lse_merge(const void* partial_o, const float* partial_lse,
+              int R, int B, int H, int D,
+              const lse_merge_strides* strides,
+              int in_dtype, int out_dtype,
+              void* out_o, float* out_lse,
+              lse_merge_stream_t stream);
+
+/* lse_merge with an explicit kernel path (one of LSE_MERGE_PATH_*).  Returns
+ * LSE_MERGE_EPATH when that path cannot take the arguments (for example the
+ * vector path with a misaligned stride).  Meant for tests and benchmarks. */
+int lse_merge_with_path(const void* partial_o, const float* partial_lse,
+                        int R, int B, int H, int D,
+                        const lse_merge_strides* strides,
+                        int in_dtype, int out_dtype,
+                        void* out_o, float* out_lse,
+                        lse_merge_stream_t stream, int path);
+
+/* The launch plan lse_merge_with_path would use.  Host-only: validates the
+ * arguments exactly as lse_merge does (pointers are only inspected, never
+ * dereferenced) and fills *plan without touching the GPU. */
+typedef struct {
+    int path;            /* LSE_MERGE_PATH_VECTOR / _LATENCY / _SCALAR */
+    int vec;             /* elements per lane per partial load (16 B / elem size; 1 for scalar) */
+    int lanes;           /* lanes that share one row slice (power of two, <= 32) */
+    int rc;              /* partial rows whose loads are in flight together per lane */
+    int slices_per_row;  /* row slices (lane groups) that cover one row of D */
+    int block;           /* threads per CTA */
+    int64_t grid;        /* CTAs */
+    int64_t groups;      /* row slices in total: B*H*slices_per_row */
+} lse_merge_plan;
+
+int lse_merge_plan_query(const void* partial_o, const float* partial_lse,
+                         int R, int B, int H, int D,
+                         const lse_merge_strides* strides,
+                         int in_dtype, int out_dtype,
+                         const void* out_o, const float* out_lse,
+                         int path, lse_merge_plan* plan);
+
+/* A static, human-readable description of a return code. */
+const char* lse_merge_strerror(int code);
+
+/* The cudaError_t of the last failed launch on this host thread (0 if none). */
+int lse_merge_last_cuda_error(void);
+
+/* ABI version of this header; bumped on any incompatible change. */
+int lse_merge_version(void);
+
+#define LSE_MERGE_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSE_MERGE_H */

@@ -1,0 +1,27 @@
+"""B200 (sm_100a) LSE-weighted merge of context-parallel decode partials.
+
+    out, out_lse = merge(partial_o, partial_lse)
+
+combines R partial attention outputs o_r (one per KV shard) and their
+log-sum-exp values lse_r into the output of attention over the whole KV
+sequence (page "[flashinfer] FlashInfer의 Context-Parallel Decode 최적화:
+Fused A2A + LSE Reduce", sections "들어가며" and "코드 분석 / 1. Fused Kernel
+구현").  PyTorch only supplies device memory and the current stream; the
+merge itself is one launch of the library's CUDA kernel through its C ABI.
+"""
+from __future__ import annotations
+
+# The binding is loaded on first use, so that the input generators (synth)
+# and the build script import without the compiled library.  Using any of
+# these names without liblse_merge.so raises ImportError: there is no
+# fallback.
+_API = ("merge", "merge_raw", "plan_query", "strerror", "LseMergeError", "dtype_code",
+        "F32", "F16", "BF16", "PATH_AUTO", "PATH_VECTOR", "PATH_LATENCY", "PATH_SCALAR")
+__all__ = list(_API)
+
+
+def __getattr__(name):
+    if name in _API:
+        from . import api
+        return getattr(api, name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")

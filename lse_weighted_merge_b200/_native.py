@@ -1,0 +1,112 @@
+"""ctypes binding of liblse_merge.so (argument marshalling only).
+
+Every step of the merge runs in the library's CUDA kernels.  There is no
+Python or CPU fallback: if the library is missing, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "liblse_merge.so")
+
+F32, F16, BF16 = 0, 1, 2
+PATH_AUTO, PATH_VECTOR, PATH_LATENCY, PATH_SCALAR = 0, 1, 2, 3
+PATH_NAMES = {PATH_VECTOR: "vector", PATH_LATENCY: "latency", PATH_SCALAR: "scalar"}
+
+OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH = 0, -1, -2, -3, -4, -5, -6, -7, -8
+
+# Every symbol include/lse_merge.h declares.
+EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merge_strerror",
+           "lse_merge_last_cuda_error", "lse_merge_version")
+ABI_VERSION = 1
+
+
+class Strides(ctypes.Structure):
+    _fields_ = [("o_r", ctypes.c_int64), ("o_b", ctypes.c_int64), ("o_h", ctypes.c_int64),
+                ("lse_r", ctypes.c_int64), ("lse_b", ctypes.c_int64), ("lse_h", ctypes.c_int64)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("vec", ctypes.c_int), ("lanes", ctypes.c_int),
+                ("rc", ctypes.c_int), ("slices_per_row", ctypes.c_int), ("block", ctypes.c_int),
+                ("grid", ctypes.c_int64), ("groups", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        d = {f: getattr(self, f) for f, _ in self._fields_}
+        d["path_name"] = PATH_NAMES.get(self.path, "?")
+        return d
+
+
+class LseMergeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"lse_merge failed ({code}): {what}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m lse_weighted_merge_b200.build` "
+            "(nvcc, sm_100a). The merge has no CPU fallback.")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    common = [vp, vp, i, i, i, i, ctypes.POINTER(Strides), i, i, vp, vp, vp]
+    lib.lse_merge.argtypes = common
+    lib.lse_merge.restype = i
+    lib.lse_merge_with_path.argtypes = common + [i]
+    lib.lse_merge_with_path.restype = i
+    lib.lse_merge_plan_query.argtypes = [vp, vp, i, i, i, i, ctypes.POINTER(Strides), i, i, vp, vp,
+                                         i, ctypes.POINTER(Plan)]
+    lib.lse_merge_plan_query.restype = i
+    lib.lse_merge_strerror.argtypes = [i]
+    lib.lse_merge_strerror.restype = ctypes.c_char_p
+    lib.lse_merge_last_cuda_error.argtypes = []
+    lib.lse_merge_last_cuda_error.restype = i
+    lib.lse_merge_version.argtypes = []
+    lib.lse_merge_version.restype = i
+    if lib.lse_merge_version() != ABI_VERSION:
+        raise ImportError(f"{LIB_PATH}: ABI version {lib.lse_merge_version()} != {ABI_VERSION}")
+    return lib
+
+
+lib = _load()
+
+
+def strerror(code: int) -> str:
+    return lib.lse_merge_strerror(int(code)).decode()
+
+
+def _strides(s) -> ctypes.POINTER(Strides) | None:
+    if s is None:
+        return None
+    if isinstance(s, Strides):
+        return ctypes.pointer(s)
+    o, l = s
+    return ctypes.pointer(Strides(*[int(x) for x in o], *[int(x) for x in l]))
+
+
+def merge_raw(o_ptr: int, lse_ptr: int, R: int, B: int, H: int, D: int, strides,
+              in_dtype: int, out_dtype: int, out_ptr: int, out_lse_ptr: int, stream: int = 0,
+              path: int = PATH_AUTO, check: bool = True) -> int:
+    """Call lse_merge_with_path on raw device pointers; raises on error if ``check``."""
+    rc = lib.lse_merge_with_path(o_ptr, lse_ptr, R, B, H, D, _strides(strides), in_dtype,
+                                 out_dtype, out_ptr, out_lse_ptr, stream or None, path)
+    if check and rc != OK:
+        extra = ""
+        if rc == ELAUNCH:
+            extra = f" (cudaError {lib.lse_merge_last_cuda_error()})"
+        raise LseMergeError(rc, strerror(rc) + extra)
+    return rc
+
+
+def plan_query(o_ptr: int, lse_ptr: int, R: int, B: int, H: int, D: int, strides,
+               in_dtype: int, out_dtype: int, out_ptr: int, out_lse_ptr: int,
+               path: int = PATH_AUTO) -> tuple[int, dict | None]:
+    """Host-only: the launch plan (or the error code) for these arguments."""
+    plan = Plan()
+    rc = lib.lse_merge_plan_query(o_ptr, lse_ptr, R, B, H, D, _strides(strides), in_dtype,
+                                  out_dtype, out_ptr, out_lse_ptr, path, ctypes.byref(plan))
+    return rc, (plan.as_dict() if rc == OK else None)

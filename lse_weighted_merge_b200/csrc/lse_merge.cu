@@ -1,0 +1,429 @@
+// lse_merge.cu -- sm_100a kernels and the C entry points of the LSE-weighted merge.
+//
+// The operation (page "[flashinfer] FlashInfer의 Context-Parallel Decode 최적화:
+// Fused A2A + LSE Reduce", section "코드 분석 / 1. Fused Kernel 구현": weights
+// from the lse values, fp32 accumulation over the partial axis, division by
+// the sum of the weights, conversion to FP16/BF16; the KV-shard partials
+// o_r, lse_r are introduced in section "들어가며"):
+//     m = max_r lse_r,  e_r = exp(lse_r - m),  out = sum_r e_r o_r / sum_r e_r,
+//     out_lse = m + log(sum_r e_r);   all shards empty -> out = 0, out_lse = -inf.
+//
+// The merge moves R*D input elements per (b,h) row for 2 flops each, so it is
+// bound by HBM bandwidth and uses no tensor cores.  Design:
+//   * a row (or a slice of a long row) belongs to a group of `lanes`
+//     consecutive lanes of one warp; each lane owns 16 contiguous bytes of
+//     every partial row (8 bf16/fp16 or 4 fp32 elements);
+//   * each lane issues the 16-byte loads of RC partial rows before it needs
+//     any weight, so RC * 16 bytes per lane are in flight while the lse
+//     values are still being reduced;
+//   * lane j of a group holds lse_j; max and sum are group shuffles, and
+//     the weight of partial i is broadcast from lane i by a shuffle;
+//   * accumulation in fp32 registers, one reciprocal of the weight sum,
+//     round-to-nearest-even conversion, 16-byte stores;
+//   * a partial with weight 0 is skipped by a select, so NaN stored in an
+//     empty shard cannot reach the output.
+// The partial rows are streamed once: loads bypass L1 and ask L2 for 256-byte
+// prefetch (the neighbouring lanes' sectors of the same row).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "lse_merge.h"
+#include "plan.h"
+
+namespace lsem {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+struct KParams {
+    const char* o;      // partial_o
+    const float* lse;   // partial_lse
+    char* out;          // out_o, dense [B,H,D]
+    float* out_lse;     // dense [B,H]
+    int64_t o_r, o_b, o_h;  // partial_o strides in BYTES
+    int64_t l_r, l_b, l_h;  // partial_lse strides in elements
+    int R, H, D;
+    int dv;             // 16-byte vectors per row (vector kernels)
+    int lanes, lg;      // lanes per group, log2(lanes)
+    int spr;            // groups (slices) per row
+    int64_t groups;     // total groups
+};
+
+// ---------------------------------------------------------------- loads / stores
+
+// 16-byte streaming load: read-only path, no L1 allocation, 256-byte L2 prefetch.
+__device__ __forceinline__ uint4 ld_stream16(const char* p) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+    static constexpr int kVec = 4;  // elements per 16 bytes
+    __device__ static void unpack(const uint4& v, float* f) {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+    __device__ static float load1(const char* p) { return __ldg(reinterpret_cast<const float*>(p)); }
+    __device__ static void store1(char* p, float x) { *reinterpret_cast<float*>(p) = x; }
+};
+
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float* f) {
+    f[0] = __uint_as_float(w << 16);          // element at the lower address
+    f[1] = __uint_as_float(w & 0xffff0000u);
+}
+
+__device__ __forceinline__ void unpack_f16x2(uint32_t w, float* f) {
+    __half2 h;
+    memcpy(&h, &w, 4);
+    const float2 x = __half22float2(h);
+    f[0] = x.x;
+    f[1] = x.y;
+}
+
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    __device__ static void unpack(const uint4& v, float* f) {
+        unpack_bf16x2(v.x, f + 0);
+        unpack_bf16x2(v.y, f + 2);
+        unpack_bf16x2(v.z, f + 4);
+        unpack_bf16x2(v.w, f + 6);
+    }
+    __device__ static float load1(const char* p) {
+        const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
+        return __uint_as_float((uint32_t)u << 16);
+    }
+    __device__ static void store1(char* p, float x) {
+        *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x);
+    }
+    __device__ static uint32_t pack2(float a, float b) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        uint32_t w;
+        memcpy(&w, &h, 4);
+        return w;
+    }
+};
+
+template <>
+struct Elem<__half> {
+    static constexpr int kVec = 8;
+    __device__ static void unpack(const uint4& v, float* f) {
+        unpack_f16x2(v.x, f + 0);
+        unpack_f16x2(v.y, f + 2);
+        unpack_f16x2(v.z, f + 4);
+        unpack_f16x2(v.w, f + 6);
+    }
+    __device__ static float load1(const char* p) {
+        const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
+        __half h;
+        memcpy(&h, &u, 2);
+        return __half2float(h);
+    }
+    __device__ static void store1(char* p, float x) {
+        *reinterpret_cast<__half*>(p) = __float2half_rn(x);
+    }
+    __device__ static uint32_t pack2(float a, float b) {
+        const __half2 h = __floats2half2_rn(a, b);
+        uint32_t w;
+        memcpy(&w, &h, 4);
+        return w;
+    }
+};
+
+// Store N fp32 values as N elements of TOut at p (aligned to min(16, N*sizeof(TOut))).
+template <typename TOut, int N>
+__device__ __forceinline__ void store_vec(char* p, const float* f) {
+    if constexpr (sizeof(TOut) == 4) {
+#pragma unroll
+        for (int k = 0; k < N; k += 4)
+            *reinterpret_cast<float4*>(p + k * 4) = make_float4(f[k], f[k + 1], f[k + 2], f[k + 3]);
+    } else if constexpr (N == 8) {
+        uint4 w;
+        w.x = Elem<TOut>::pack2(f[0], f[1]);
+        w.y = Elem<TOut>::pack2(f[2], f[3]);
+        w.z = Elem<TOut>::pack2(f[4], f[5]);
+        w.w = Elem<TOut>::pack2(f[6], f[7]);
+        *reinterpret_cast<uint4*>(p) = w;
+    } else {
+        uint2 w;
+        w.x = Elem<TOut>::pack2(f[0], f[1]);
+        w.y = Elem<TOut>::pack2(f[2], f[3]);
+        *reinterpret_cast<uint2*>(p) = w;
+    }
+}
+
+// --------------------------------------------------------------- group reductions
+
+// Groups are `lanes` consecutive lanes starting at a multiple of `lanes`, so an
+// xor offset below `lanes` stays inside the group.
+__device__ __forceinline__ float group_max(float v, int lanes) {
+    for (int off = lanes >> 1; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, off));
+    return v;
+}
+
+__device__ __forceinline__ float group_sum(float v, int lanes) {
+    for (int off = lanes >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+    return v;
+}
+
+// ------------------------------------------------------------------ vector kernel
+
+// One group of p.lanes lanes merges one slice of one (b,h) row.  Lane j owns
+// the 16-byte column v = slice*lanes + j of every partial row.  Control flow
+// that reaches a shuffle depends only on R, lanes and RC, which are the same
+// for every thread of the grid, so every shuffle sees all 32 lanes.
+template <typename TIn, typename TOut, int RC>
+__global__ void __launch_bounds__(kBlock) merge_vec_kernel(const KParams p) {
+    constexpr int N = Elem<TIn>::kVec;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t grp = t >> p.lg;
+    const int j = (int)(t & (p.lanes - 1));
+    const bool live = grp < p.groups;
+    int64_t row = 0;
+    int slice = 0;
+    if (live) {
+        row = grp / p.spr;
+        slice = (int)(grp - row * p.spr);
+    }
+    const int64_t b = row / p.H, h = row - b * p.H;
+    const int v = slice * p.lanes + j;
+    const bool vlive = live && v < p.dv;
+    const char* orow = p.o + b * p.o_b + h * p.o_h + (int64_t)v * 16;
+    const float* lrow = p.lse + b * p.l_b + h * p.l_h;
+
+    // Partial rows 0..RC-1 go in flight first; nothing here waits on lse.
+    uint4 x[RC];
+#pragma unroll
+    for (int i = 0; i < RC; ++i) {
+        x[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (vlive && i < p.R) x[i] = ld_stream16(orow + (int64_t)i * p.o_r);
+    }
+
+    // m = max_r lse_r over the group (lane j reads lse_j, lse_{j+lanes}, ...).
+    float l0 = -INFINITY;
+    if (live && j < p.R) l0 = __ldg(lrow + (int64_t)j * p.l_r);
+    float m = l0;
+    for (int c = p.lanes; c < p.R; c += p.lanes)
+        if (live && c + j < p.R) m = fmaxf(m, __ldg(lrow + (int64_t)(c + j) * p.l_r));
+    m = group_max(m, p.lanes);
+    // An all-empty row has m = -inf; subtracting 0 instead keeps every weight
+    // exp(-inf) = 0 rather than exp(-inf + inf) = NaN.
+    const float mref = (m == -INFINITY) ? 0.f : m;
+
+    float acc[N];
+#pragma unroll
+    for (int k = 0; k < N; ++k) acc[k] = 0.f;
+    float esum = 0.f;
+
+    for (int c = 0; c < p.R; c += p.lanes) {
+        float l = l0;
+        if (c > 0) {
+            l = -INFINITY;
+            if (live && c + j < p.R) l = __ldg(lrow + (int64_t)(c + j) * p.l_r);
+        }
+        const float e = expf(l - mref);  // weight of partial c+j; 0 for an empty shard
+        esum += e;
+        const int cn = min(p.R - c, p.lanes);
+        for (int s0 = 0; s0 < cn; s0 += RC) {
+            if (c > 0 || s0 > 0) {
+#pragma unroll
+                for (int i = 0; i < RC; ++i)
+                    if (vlive && s0 + i < cn) x[i] = ld_stream16(orow + (int64_t)(c + s0 + i) * p.o_r);
+            }
+#pragma unroll
+            for (int i = 0; i < RC; ++i) {
+                const float w = __shfl_sync(kFull, e, s0 + i, p.lanes);
+                if (s0 + i < cn && w != 0.f) {
+                    float f[N];
+                    Elem<TIn>::unpack(x[i], f);
+#pragma unroll
+                    for (int k = 0; k < N; ++k) acc[k] = fmaf(w, f[k], acc[k]);
+                }
+            }
+        }
+    }
+    esum = group_sum(esum, p.lanes);
+
+    // esum >= 1 for a row with a finite max (its own weight is exp(0)).
+    const float inv = esum > 0.f ? 1.f / esum : 0.f;
+    if (vlive) {
+#pragma unroll
+        for (int k = 0; k < N; ++k) acc[k] *= inv;
+        store_vec<TOut, N>(p.out + (row * p.D + (int64_t)v * N) * (int64_t)sizeof(TOut), acc);
+    }
+    if (live && slice == 0 && j == 0) p.out_lse[row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+}
+
+// ------------------------------------------------------------------ scalar kernel
+
+// Any alignment of strides and D: one warp per row, lane j handles the
+// elements d = j, j+32, ...; element loads.
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kBlock) merge_scalar_kernel(const KParams p) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = t >> 5;
+    const int j = (int)(t & 31);
+    const bool live = row < p.groups;
+    const int64_t b = live ? row / p.H : 0, h = live ? row - b * p.H : 0;
+    const char* orow = p.o + b * p.o_b + h * p.o_h;
+    const float* lrow = p.lse + b * p.l_b + h * p.l_h;
+
+    float m = -INFINITY;
+    for (int c = 0; c < p.R; c += 32)
+        if (live && c + j < p.R) m = fmaxf(m, __ldg(lrow + (int64_t)(c + j) * p.l_r));
+    m = group_max(m, 32);
+    const float mref = (m == -INFINITY) ? 0.f : m;
+
+    float e0 = 0.f;
+    if (live && j < p.R) e0 = expf(__ldg(lrow + (int64_t)j * p.l_r) - mref);
+    float esum = e0;
+    for (int c = 32; c < p.R; c += 32)
+        if (live && c + j < p.R) esum += expf(__ldg(lrow + (int64_t)(c + j) * p.l_r) - mref);
+    esum = group_sum(esum, 32);
+    const float inv = esum > 0.f ? 1.f / esum : 0.f;
+
+    for (int d0 = 0; d0 < p.D; d0 += 32) {
+        const int d = d0 + j;
+        const bool dlive = live && d < p.D;
+        float acc = 0.f;
+        for (int c = 0; c < p.R; c += 32) {
+            float e = e0;
+            if (c > 0) {
+                e = 0.f;
+                if (live && c + j < p.R) e = expf(__ldg(lrow + (int64_t)(c + j) * p.l_r) - mref);
+            }
+            const int cn = min(p.R - c, 32);
+            for (int i = 0; i < cn; ++i) {
+                const float w = __shfl_sync(kFull, e, i);
+                if (dlive && w != 0.f)
+                    acc = fmaf(w, Elem<TIn>::load1(orow + (int64_t)(c + i) * p.o_r +
+                                                   (int64_t)d * (int64_t)sizeof(TIn)),
+                               acc);
+            }
+        }
+        if (dlive) Elem<TOut>::store1(p.out + (row * p.D + d) * (int64_t)sizeof(TOut), acc * inv);
+    }
+    if (live && j == 0) p.out_lse[row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+}
+
+// ------------------------------------------------------------------------ dispatch
+
+using KernelFn = void (*)(KParams);
+
+template <typename TIn, typename TOut>
+KernelFn pick_kernel(const lse_merge_plan& pl) {
+    if (pl.path == LSE_MERGE_PATH_SCALAR) return merge_scalar_kernel<TIn, TOut>;
+    switch (pl.rc) {
+        case 4: return merge_vec_kernel<TIn, TOut, 4>;
+        case 8: return merge_vec_kernel<TIn, TOut, 8>;
+        default: return merge_vec_kernel<TIn, TOut, 16>;
+    }
+}
+
+template <typename TIn>
+KernelFn pick_out(const lse_merge_plan& pl, int out_dtype) {
+    switch (out_dtype) {
+        case LSE_MERGE_F32: return pick_kernel<TIn, float>(pl);
+        case LSE_MERGE_F16: return pick_kernel<TIn, __half>(pl);
+        default: return pick_kernel<TIn, __nv_bfloat16>(pl);
+    }
+}
+
+KernelFn pick(const lse_merge_plan& pl, int in_dtype, int out_dtype) {
+    switch (in_dtype) {
+        case LSE_MERGE_F32: return pick_out<float>(pl, out_dtype);
+        case LSE_MERGE_F16: return pick_out<__half>(pl, out_dtype);
+        default: return pick_out<__nv_bfloat16>(pl, out_dtype);
+    }
+}
+
+thread_local int g_last_cuda_error = 0;
+
+int log2i(int x) {
+    int l = 0;
+    while ((1 << l) < x) ++l;
+    return l;
+}
+
+int run(const void* partial_o, const float* partial_lse, int R, int B, int H, int D,
+        const lse_merge_strides* strides, int in_dtype, int out_dtype, void* out_o,
+        float* out_lse, cudaStream_t stream, int path) {
+    if (R < 1 || B < 1 || H < 1 || D < 1) return LSE_MERGE_EDIMS;
+    const lse_merge_strides st = strides ? *strides : default_strides(R, B, H, D);
+    lse_merge_plan pl;
+    const int rc = make_plan(partial_o, partial_lse, R, B, H, D, st, in_dtype, out_dtype, out_o,
+                             out_lse, path, &pl);
+    if (rc != LSE_MERGE_OK) return rc;
+
+    const int ib = elem_bytes(in_dtype);
+    KParams kp;
+    kp.o = static_cast<const char*>(partial_o);
+    kp.lse = partial_lse;
+    kp.out = static_cast<char*>(out_o);
+    kp.out_lse = out_lse;
+    kp.o_r = st.o_r * ib;
+    kp.o_b = st.o_b * ib;
+    kp.o_h = st.o_h * ib;
+    kp.l_r = st.lse_r;
+    kp.l_b = st.lse_b;
+    kp.l_h = st.lse_h;
+    kp.R = R;
+    kp.H = H;
+    kp.D = D;
+    kp.dv = pl.path == LSE_MERGE_PATH_SCALAR ? D : D / pl.vec;
+    kp.lanes = pl.lanes;
+    kp.lg = log2i(pl.lanes);
+    kp.spr = pl.slices_per_row;
+    kp.groups = pl.groups;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.grid);
+    cfg.blockDim = dim3((unsigned)pl.block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, pick(pl, in_dtype, out_dtype), kp);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = (int)e;
+        (void)cudaGetLastError();  // the failure belongs to this call; do not leave it pending
+        return LSE_MERGE_ELAUNCH;
+    }
+    return LSE_MERGE_OK;
+}
+
+}  // namespace
+}  // namespace lsem
+
+extern "C" {
+
+int lse_merge(const void* partial_o, const float* partial_lse, int R, int B, int H, int D,
+              const lse_merge_strides* strides, int in_dtype, int out_dtype, void* out_o,
+              float* out_lse, lse_merge_stream_t stream) {
+    return lsem::run(partial_o, partial_lse, R, B, H, D, strides, in_dtype, out_dtype, out_o,
+                     out_lse, reinterpret_cast<cudaStream_t>(stream), LSE_MERGE_PATH_AUTO);
+}
+
+int lse_merge_with_path(const void* partial_o, const float* partial_lse, int R, int B, int H,
+                        int D, const lse_merge_strides* strides, int in_dtype, int out_dtype,
+                        void* out_o, float* out_lse, lse_merge_stream_t stream, int path) {
+    return lsem::run(partial_o, partial_lse, R, B, H, D, strides, in_dtype, out_dtype, out_o,
+                     out_lse, reinterpret_cast<cudaStream_t>(stream), path);
+}
+
+int lse_merge_last_cuda_error(void) { return lsem::g_last_cuda_error; }
+
+}  // extern "C"

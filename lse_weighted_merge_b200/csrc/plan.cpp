@@ -1,0 +1,175 @@
+// plan.cpp -- validation and launch geometry of the LSE-weighted merge.
+//
+// Geometry of the vector kernels (the merge of one (b,h) row is spread over
+// a group of `lanes` consecutive lanes of one warp):
+//   * vec     = 16 bytes / element size: one 16-byte load per lane per partial;
+//   * lanes   = the power of two >= D/vec (at most 32), and at least rc so the
+//               lanes of a group can hold one lse value each for a batch;
+//   * slices  = ceil((D/vec) / lanes) groups per row when D/vec > 32;
+//   * rc      = 4, 8 or 16 partial rows loaded before the first FMA, so up to
+//               rc * 16 bytes per lane are in flight.
+// The latency path is the same kernel launched as one CTA of exactly the
+// threads needed, for problems of at most kLatencyMaxThreads threads.
+#include "plan.h"
+
+#include <cstdint>
+
+namespace lsem {
+
+int elem_bytes(int dtype) {
+    switch (dtype) {
+        case LSE_MERGE_F32: return 4;
+        case LSE_MERGE_F16: return 2;
+        case LSE_MERGE_BF16: return 2;
+        default: return 0;
+    }
+}
+
+lse_merge_strides default_strides(int R, int B, int H, int D) {
+    (void)B;
+    lse_merge_strides s;
+    s.o_r = D;
+    s.o_b = (int64_t)H * R * D;
+    s.o_h = (int64_t)R * D;
+    s.lse_r = 1;
+    s.lse_b = (int64_t)H * R;
+    s.lse_h = R;
+    return s;
+}
+
+namespace {
+
+using i128 = __int128;
+
+// Byte interval [lo, hi) of a buffer.
+struct Span {
+    uintptr_t lo;
+    i128 hi;
+};
+
+bool overlap(const Span& a, const Span& b) {
+    return (i128)a.lo < b.hi && (i128)b.lo < a.hi;
+}
+
+int next_pow2(int x) {
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+bool aligned(const void* p, int a) { return ((uintptr_t)p % (uintptr_t)a) == 0; }
+
+}  // namespace
+
+int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
+              const lse_merge_strides& st, int in_dtype, int out_dtype, const void* out_o,
+              const float* out_lse, int path, lse_merge_plan* plan) {
+    const int ib = elem_bytes(in_dtype), ob = elem_bytes(out_dtype);
+    if (ib == 0 || ob == 0) return LSE_MERGE_EDTYPE;
+    if (R < 1 || B < 1 || H < 1 || D < 1) return LSE_MERGE_EDIMS;
+    if (!o || !lse || !out_o || !out_lse || !plan) return LSE_MERGE_ENULL;
+    if (st.o_r < 0 || st.o_b < 0 || st.o_h < 0 || st.lse_r < 0 || st.lse_b < 0 || st.lse_h < 0)
+        return LSE_MERGE_ESTRIDE;
+    if (path < LSE_MERGE_PATH_AUTO || path > LSE_MERGE_PATH_SCALAR) return LSE_MERGE_EPATH;
+    if (!aligned(o, ib) || !aligned(out_o, ob) || !aligned(lse, 4) || !aligned(out_lse, 4))
+        return LSE_MERGE_EALIGN;
+
+    // Extents in bytes, in 128-bit arithmetic so that no product can wrap.
+    const i128 o_last = (i128)(R - 1) * st.o_r + (i128)(B - 1) * st.o_b + (i128)(H - 1) * st.o_h + D;
+    const i128 l_last = (i128)(R - 1) * st.lse_r + (i128)(B - 1) * st.lse_b + (i128)(H - 1) * st.lse_h + 1;
+    const i128 rows = (i128)B * H;
+    const i128 lim = (i128)1 << 62;
+    const i128 o_bytes = o_last * ib, l_bytes = l_last * 4, out_bytes = rows * D * ob, ol_bytes = rows * 4;
+    if (o_bytes > lim || l_bytes > lim || out_bytes > lim || ol_bytes > lim) return LSE_MERGE_EDIMS;
+
+    const Span so{(uintptr_t)o, (i128)(uintptr_t)o + o_bytes};
+    const Span sl{(uintptr_t)lse, (i128)(uintptr_t)lse + l_bytes};
+    const Span su{(uintptr_t)out_o, (i128)(uintptr_t)out_o + out_bytes};
+    const Span sv{(uintptr_t)out_lse, (i128)(uintptr_t)out_lse + ol_bytes};
+    if (overlap(su, so) || overlap(su, sl) || overlap(sv, so) || overlap(sv, sl) || overlap(su, sv))
+        return LSE_MERGE_EALIAS;
+
+    // Can the 16-byte vector kernels take these arguments?
+    const int vec = 16 / ib;
+    const int out_align = (vec * ob) < 16 ? vec * ob : 16;
+    const bool vec_ok = (D % vec) == 0 && aligned(o, 16) && ((st.o_r * ib) % 16) == 0 &&
+                        ((st.o_b * ib) % 16) == 0 && ((st.o_h * ib) % 16) == 0 &&
+                        aligned(out_o, out_align);
+
+    lse_merge_plan p{};
+    if (vec_ok && path != LSE_MERGE_PATH_SCALAR) {
+        const int dv = D / vec;
+        const int rc = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
+        int lanes = next_pow2(dv < 32 ? dv : 32);
+        if (lanes < rc) lanes = rc;
+        const int slices = (dv + lanes - 1) / lanes;
+        const i128 groups = rows * slices;
+        const i128 threads = groups * lanes;
+        const bool small = threads <= kLatencyMaxThreads;
+        int chosen = path;
+        if (chosen == LSE_MERGE_PATH_AUTO) chosen = small ? LSE_MERGE_PATH_LATENCY : LSE_MERGE_PATH_VECTOR;
+        if (chosen == LSE_MERGE_PATH_LATENCY && !small) return LSE_MERGE_EPATH;
+        p.path = chosen;
+        p.vec = vec;
+        p.lanes = lanes;
+        p.rc = rc;
+        p.slices_per_row = slices;
+        p.groups = (int64_t)groups;
+        if (chosen == LSE_MERGE_PATH_LATENCY) {
+            p.block = (int)((threads + 31) / 32 * 32);
+            p.grid = 1;
+        } else {
+            p.block = kBlock;
+            const i128 grid = (threads + kBlock - 1) / kBlock;
+            if (grid > 0x7fffffff) return LSE_MERGE_EDIMS;
+            p.grid = (int64_t)grid;
+        }
+    } else {
+        if (path == LSE_MERGE_PATH_VECTOR || path == LSE_MERGE_PATH_LATENCY) return LSE_MERGE_EPATH;
+        p.path = LSE_MERGE_PATH_SCALAR;
+        p.vec = 1;
+        p.lanes = 32;
+        p.rc = 0;
+        p.slices_per_row = 1;
+        p.groups = (int64_t)rows;
+        p.block = kBlock;
+        const i128 grid = (rows * 32 + kBlock - 1) / kBlock;
+        if (grid > 0x7fffffff) return LSE_MERGE_EDIMS;
+        p.grid = (int64_t)grid;
+    }
+    *plan = p;
+    return LSE_MERGE_OK;
+}
+
+}  // namespace lsem
+
+extern "C" {
+
+int lse_merge_plan_query(const void* partial_o, const float* partial_lse, int R, int B, int H,
+                         int D, const lse_merge_strides* strides, int in_dtype, int out_dtype,
+                         const void* out_o, const float* out_lse, int path,
+                         lse_merge_plan* plan) {
+    if (R < 1 || B < 1 || H < 1 || D < 1) return LSE_MERGE_EDIMS;
+    const lse_merge_strides st = strides ? *strides : lsem::default_strides(R, B, H, D);
+    return lsem::make_plan(partial_o, partial_lse, R, B, H, D, st, in_dtype, out_dtype, out_o,
+                           out_lse, path, plan);
+}
+
+const char* lse_merge_strerror(int code) {
+    switch (code) {
+        case LSE_MERGE_OK: return "ok";
+        case LSE_MERGE_EDTYPE: return "unknown element type (in_dtype/out_dtype)";
+        case LSE_MERGE_EDIMS: return "R, B, H and D must be >= 1 and the extents must fit";
+        case LSE_MERGE_ENULL: return "a required pointer is NULL";
+        case LSE_MERGE_ESTRIDE: return "strides must be >= 0";
+        case LSE_MERGE_EALIAS: return "an output overlaps an input or the other output";
+        case LSE_MERGE_ELAUNCH: return "CUDA kernel launch failed";
+        case LSE_MERGE_EALIGN: return "a pointer is not aligned to its element size";
+        case LSE_MERGE_EPATH: return "the requested kernel path cannot take these arguments";
+        default: return "unknown lse_merge error code";
+    }
+}
+
+int lse_merge_version(void) { return LSE_MERGE_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,134 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol, and
+its argument validation and launch planning behave as documented.  Nothing
+here launches a kernel; rejected calls return before any CUDA call, and the
+planner only inspects pointer values, never dereferences them."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from lse_weighted_merge_b200 import _native as nat
+from lse_weighted_merge_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lse_merge.h")
+
+# Fake, suitably aligned device addresses far apart (never dereferenced).
+PO, PL, OUT, OUTL = 0x7f0000000000, 0x7f1000000000, 0x7f2000000000, 0x7f3000000000
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(lse_merge\w*)\s*\(", text, re.M)))
+
+
+def test_header_and_binding_agree():
+    assert sorted(nat.EXPORTS) == declared_functions()
+
+
+def test_every_declared_symbol_is_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", nat.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(nat.lib, name)
+
+
+def test_version_and_strerror():
+    assert nat.lib.lse_merge_version() == nat.ABI_VERSION == 1
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+        assert nat.strerror(code) and "unknown lse_merge error" not in nat.strerror(code)
+    assert "unknown lse_merge error" in nat.strerror(-99)
+
+
+def q(R=2, B=1, H=2, D=64, strides=None, i=nat.BF16, o=nat.BF16, po=PO, pl=PL, out=OUT,
+      outl=OUTL, path=nat.PATH_AUTO):
+    return nat.plan_query(po, pl, R, B, H, D, strides, i, o, out, outl, path)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(i=3), nat.EDTYPE), (dict(o=-1), nat.EDTYPE),
+    (dict(R=0), nat.EDIMS), (dict(B=0), nat.EDIMS), (dict(H=-1), nat.EDIMS), (dict(D=0), nat.EDIMS),
+    (dict(po=0), nat.ENULL), (dict(pl=0), nat.ENULL), (dict(out=0), nat.ENULL), (dict(outl=0), nat.ENULL),
+    (dict(strides=((-64, 128, 64), (1, 2, 1))), nat.ESTRIDE),
+    (dict(strides=((64, 128, 64), (1, -2, 1))), nat.ESTRIDE),
+    (dict(po=PO + 1), nat.EALIGN), (dict(pl=PL + 2), nat.EALIGN), (dict(outl=OUTL + 1), nat.EALIGN),
+    (dict(i=nat.F32, po=PO + 2), nat.EALIGN), (dict(out=OUT + 1), nat.EALIGN),
+    (dict(out=PO + 64), nat.EALIAS), (dict(outl=PL), nat.EALIAS), (dict(outl=OUT + 8), nat.EALIAS),
+    (dict(out=PL), nat.EALIAS),
+    (dict(path=7), nat.EPATH),
+    (dict(B=64, H=64, path=nat.PATH_LATENCY), nat.EPATH),
+    (dict(D=60, path=nat.PATH_VECTOR), nat.EPATH),
+    (dict(po=PO + 2, path=nat.PATH_VECTOR), nat.EPATH),
+    (dict(R=2 ** 30, B=2 ** 30, H=2 ** 30, D=2 ** 30), nat.EDIMS),
+])
+def test_validation(kw, code):
+    rc, plan = q(**kw)
+    assert rc == code, (kw, rc, nat.strerror(rc))
+    assert plan is None
+
+
+def test_rejected_calls_return_before_any_cuda_call():
+    # Argument errors come back from lse_merge itself, with nothing enqueued.
+    assert nat.merge_raw(0, PL, 2, 1, 2, 64, None, nat.BF16, nat.BF16, OUT, OUTL, check=False) == nat.ENULL
+    assert nat.merge_raw(PO, PL, 0, 1, 2, 64, None, nat.BF16, nat.BF16, OUT, OUTL, check=False) == nat.EDIMS
+    assert nat.merge_raw(PO, PL, 2, 1, 2, 64, None, 9, nat.BF16, OUT, OUTL, check=False) == nat.EDTYPE
+    assert nat.merge_raw(PO, PL, 2, 1, 2, 64, None, nat.BF16, nat.BF16, PO, OUTL, check=False) == nat.EALIAS
+    with pytest.raises(nat.LseMergeError) as ei:
+        nat.merge_raw(PO, PL, 2, 1, 2, 64, None, nat.BF16, nat.BF16, PO, OUTL)
+    assert ei.value.code == nat.EALIAS
+    assert nat.lib.lse_merge(None, None, 1, 1, 1, 1, None, 0, 0, None, None, None) == nat.ENULL
+
+
+def test_plans_of_the_five_workloads():
+    expect = {  # name -> (path, lanes, rc, slices, block, grid)
+        "r2_b1_h2_d64": (nat.PATH_LATENCY, 8, 4, 1, 32, 1),
+        "r8_b1_h8_d128": (nat.PATH_LATENCY, 16, 8, 1, 128, 1),
+        "r4_b64_h32_d128_masked": (nat.PATH_VECTOR, 16, 4, 1, 256, 64 * 32 * 16 // 256),
+        "r8_b256_h64_d128_rankmajor": (nat.PATH_VECTOR, 16, 8, 1, 256, 256 * 64 * 16 // 256),
+        "r16_b512_h16_d512": (nat.PATH_VECTOR, 32, 16, 2, 256, 512 * 16 * 2 * 32 // 256),
+    }
+    for name, w in synth.WORKLOADS.items():
+        st = synth.strides(w.layout, w.R, w.B, w.H, w.D)
+        rc, plan = nat.plan_query(PO, PL, w.R, w.B, w.H, w.D, st, synth.DTYPES[w.in_dtype],
+                                  synth.DTYPES[w.out_dtype], OUT, OUTL)
+        assert rc == 0, name
+        got = (plan["path"], plan["lanes"], plan["rc"], plan["slices_per_row"], plan["block"],
+               plan["grid"])
+        assert got == expect[name], (name, got)
+        assert plan["vec"] == 8
+        assert plan["groups"] == w.B * w.H * plan["slices_per_row"]
+
+
+def test_fallback_to_scalar_and_forced_paths():
+    # D not a multiple of 8 bf16 elements -> scalar; misaligned stride -> scalar
+    assert q(D=60)[1]["path"] == nat.PATH_SCALAR
+    assert q(strides=((65, 130, 65), (1, 2, 1)), D=64)[1]["path"] == nat.PATH_SCALAR
+    assert q(po=PO + 2)[1]["path"] == nat.PATH_SCALAR
+    # f32 output of a bf16 row needs 16-byte alignment of out (8 elements = 32 B)
+    assert q(o=nat.F32, out=OUT + 8)[1]["path"] == nat.PATH_SCALAR
+    # f32 input: 4 elements per vector; bf16 out then needs 8-byte alignment
+    assert q(i=nat.F32, D=12)[1]["vec"] == 4
+    assert q(i=nat.F32, o=nat.BF16, out=OUT + 8)[1]["path"] == nat.PATH_LATENCY
+    for path in (nat.PATH_VECTOR, nat.PATH_LATENCY, nat.PATH_SCALAR):
+        rc, plan = q(path=path)
+        assert rc == 0 and plan["path"] == path
+    rc, plan = q(B=64, H=64, path=nat.PATH_SCALAR)
+    assert plan["grid"] == 64 * 64 * 32 // 256 and plan["lanes"] == 32
+
+
+@pytest.mark.parametrize("R,want_rc,want_lanes", [(1, 4, 8), (3, 4, 8), (5, 8, 8), (9, 16, 16),
+                                                   (16, 16, 16), (33, 16, 16)])
+def test_rc_and_lanes_follow_R(R, want_rc, want_lanes):
+    rc, plan = q(R=R, D=64)      # 8 vectors per row
+    assert rc == 0 and plan["rc"] == want_rc and plan["lanes"] == want_lanes
+
+
+@pytest.mark.parametrize("D,lanes,slices", [(8, 4, 1), (24, 4, 1), (128, 16, 1), (256, 32, 1),
+                                             (264, 32, 2), (1024, 32, 4)])
+def test_lanes_and_slices_follow_D(D, lanes, slices):
+    rc, plan = q(R=2, D=D, B=8, H=64)
+    assert rc == 0 and plan["lanes"] == lanes and plan["slices_per_row"] == slices
