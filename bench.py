@@ -262,32 +262,27 @@ def n_sets(bytes_per_set: int, l2_bytes: int) -> int:
     return int(min(256, max(2, math.ceil(2 * l2_bytes / max(bytes_per_set, 1)) + 1)))
 
 
-def time_eager(sets: DeviceSets, steps: int, warmup: int, device, per_launch: bool = True):
-    """Run `warmup` then `steps` launches; returns (region_ms, mean_launch_ms, t0, t1)."""
+def time_eager(sets: DeviceSets, steps: int, warmup: int, device):
+    """Run `warmup` then `steps` back-to-back launches on the current stream;
+    returns (region_ms, t0, t1).  One kernel launch per step, so region/steps
+    is the kernel's average launch duration; no event sits between launches
+    (an event record between two launches would serialise them)."""
     import torch
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
     for i in range(warmup):
         sets.launch(i, sh)
     torch.cuda.synchronize(device)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)] if per_launch else None
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)] if per_launch else None
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     t0 = time.perf_counter()
     e0.record(stream)
     for i in range(steps):
-        if per_launch:
-            starts[i].record(stream)
         sets.launch(warmup + i, sh)
-        if per_launch:
-            ends[i].record(stream)
     e1.record(stream)
     torch.cuda.synchronize(device)
     t1 = time.perf_counter()
-    region = e0.elapsed_time(e1)
-    mean_launch = (sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / steps) if per_launch else region / steps
-    return region, mean_launch, t0, t1
+    return e0.elapsed_time(e1), t0, t1
 
 
 def time_graph(sets: DeviceSets, calls: int, replays: int, device) -> float:
@@ -482,18 +477,18 @@ def run_ours(args):
     for attempt in range(2):
         barrier(dist, device)
         torch.cuda.synchronize(device)
-        region_ms, launch_ms, t0, t1 = time_eager(sets, args.steps, args.warmup, device)
+        region_ms, t0, t1 = time_eager(sets, args.steps, args.warmup, device)
         barrier(dist, device)
         region_ms = max_over_ranks(region_ms, dist, device)
-        launch_ms = max_over_ranks(launch_ms, dist, device)
         clk = clock.summary(t0, t1)
-        attempts.append((region_ms, launch_ms, clk))
+        attempts.append((region_ms, clk))
         bad = [r for r in clk.get("reasons", []) if r in BAD_REASONS]
         bad_flag = max_over_ranks(1.0 if bad else 0.0, dist, device)
         if bad_flag == 0.0:
             break
         log(f"clock reasons {bad} during the timed region: measuring once more")
-    region_ms, launch_ms, clk = attempts[-1]
+    region_ms, clk = attempts[-1]
+    launch_ms = region_ms / args.steps
     if len(attempts) > 1:
         clk["remeasured"] = True
 
@@ -565,7 +560,7 @@ def extra_workloads(device, l2: int, dist) -> dict:
         tiny = w.bytes_total() < 1 << 20
         nset = 4 if tiny else n_sets(w.bytes_total(), l2)
         sets = DeviceSets(inp, nset, device)
-        region, launch, _, _ = time_eager(sets, 400 if tiny else 200, 20, device, per_launch=False)
+        region, _, _ = time_eager(sets, 400 if tiny else 200, 20, device)
         eager_us = region * 1e3 / (400 if tiny else 200)
         row = {"eager_us_per_call": eager_us, "gbs": w.bytes_total() / (eager_us * 1e-6) / 1e9,
                "l2": "resident (latency shape)" if tiny else f"rotating {nset} sets"}

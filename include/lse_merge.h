@@ -73,6 +73,8 @@ typedef struct {
 #define LSE_MERGE_PATH_VECTOR 1   /* 16-byte vector loads, many CTAs (throughput) */
 #define LSE_MERGE_PATH_LATENCY 2  /* the vector kernel as one small CTA (tiny B*H) */
 #define LSE_MERGE_PATH_SCALAR 3   /* element loads, any alignment of strides and D */
+#define LSE_MERGE_PATH_STREAM 4   /* persistent vector kernel, loads of the next row slice
+                                     issued as the current one is consumed (R <= 16) */
 
 /*
  * Merge R partials of B*H rows.
@@ -115,13 +117,14 @@ int lse_merge_with_path(const void* partial_o, const float* partial_lse,
  * arguments exactly as lse_merge does (pointers are only inspected, never
  * dereferenced) and fills *plan without touching the GPU. */
 typedef struct {
-    int path;            /* LSE_MERGE_PATH_VECTOR / _LATENCY / _SCALAR */
+    int path;            /* LSE_MERGE_PATH_VECTOR / _LATENCY / _SCALAR / _STREAM */
     int vec;             /* elements per lane per partial load (16 B / elem size; 1 for scalar) */
     int lanes;           /* lanes that share one row slice (power of two, <= 32) */
     int rc;              /* partial rows whose loads are in flight together per lane */
     int slices_per_row;  /* row slices (lane groups) that cover one row of D */
     int block;           /* threads per CTA */
-    int64_t grid;        /* CTAs */
+    int64_t grid;        /* CTAs; 0 for STREAM, whose persistent grid is sized at
+                            launch to the CTAs that fit on the device at once */
     int64_t groups;      /* row slices in total: B*H*slices_per_row */
 } lse_merge_plan;
 

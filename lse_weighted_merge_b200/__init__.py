@@ -16,7 +16,8 @@ from __future__ import annotations
 # these names without liblse_merge.so raises ImportError: there is no
 # fallback.
 _API = ("merge", "merge_raw", "plan_query", "strerror", "LseMergeError", "dtype_code",
-        "F32", "F16", "BF16", "PATH_AUTO", "PATH_VECTOR", "PATH_LATENCY", "PATH_SCALAR")
+        "F32", "F16", "BF16", "PATH_AUTO", "PATH_VECTOR", "PATH_LATENCY", "PATH_SCALAR",
+        "PATH_STREAM")
 __all__ = list(_API)
 
 

@@ -1,7 +1,8 @@
 """The torch-facing call: tensors in, one C-ABI launch, tensors out."""
 from __future__ import annotations
 
-from ._native import (BF16, F16, F32, PATH_AUTO, PATH_LATENCY, PATH_SCALAR, PATH_VECTOR,
+from ._native import (BF16, F16, F32, PATH_AUTO, PATH_LATENCY, PATH_SCALAR, PATH_STREAM,
+                      PATH_VECTOR,
                       LseMergeError, merge_raw, plan_query, strerror)
 
 

@@ -30,6 +30,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "lse_merge.h"
 #include "plan.h"
@@ -51,7 +52,45 @@ struct KParams {
     int lanes, lg;      // lanes per group, log2(lanes)
     int spr;            // groups (slices) per row
     int64_t groups;     // total groups
+    // n / spr and n / H for 32-bit n by one high multiply (d == 1: n itself);
+    // used when every group and row index fits in 32 bits (idx32).
+    uint64_t c_spr, c_H;
+    int idx32;
 };
+
+// Division by a run-time constant d >= 2 of any 32-bit n as the high 64 bits
+// of c * n with c = ceil(2^64 / d) (Lemire, Kaser and Kurz, "Faster remainder
+// by direct computation", 2019, for N = 32 and F = 64 bits).
+__host__ __device__ __forceinline__ uint64_t fastdiv_c(uint32_t d) {
+    return d <= 1 ? 0 : ~0ull / d + 1;
+}
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, uint64_t c, uint32_t d) {
+    return d == 1 ? n : (uint32_t)__umul64hi(c, (uint64_t)n);
+}
+
+// Row, slice, batch and head of group `grp` (valid when grp < groups).
+struct RowIdx {
+    int64_t row, b, h;
+    int slice;
+};
+__device__ __forceinline__ RowIdx row_of(const KParams& p, int64_t grp) {
+    RowIdx r;
+    if (p.idx32) {
+        const uint32_t g = (uint32_t)grp;
+        const uint32_t q = fastdiv(g, p.c_spr, (uint32_t)p.spr);
+        const uint32_t bb = fastdiv(q, p.c_H, (uint32_t)p.H);
+        r.row = q;
+        r.slice = (int)(g - q * (uint32_t)p.spr);
+        r.b = bb;
+        r.h = q - bb * (uint32_t)p.H;
+    } else {
+        r.row = grp / p.spr;
+        r.slice = (int)(grp - r.row * p.spr);
+        r.b = r.row / p.H;
+        r.h = r.row - r.b * p.H;
+    }
+    return r;
+}
 
 // ---------------------------------------------------------------- loads / stores
 
@@ -62,6 +101,24 @@ __device__ __forceinline__ uint4 ld_stream16(const char* p) {
         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
         : "l"(p));
     return v;
+}
+
+// Two fp32 values in one 64-bit register pair, for the packed sm_100 FMA:
+// fma.rn.f32x2 performs two independent IEEE fp32 fused multiply-adds, so
+// every lane of the pair rounds exactly like fmaf.
+__device__ __forceinline__ uint64_t pack2u(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t pack2f(float lo, float hi) {
+    return pack2u(__float_as_uint(lo), __float_as_uint(hi));
+}
+__device__ __forceinline__ void unpack2f(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ void fma2(uint64_t& acc, uint64_t x, uint64_t w) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(x), "l"(w));
 }
 
 template <typename T>
@@ -75,6 +132,11 @@ struct Elem<float> {
         f[1] = __uint_as_float(v.y);
         f[2] = __uint_as_float(v.z);
         f[3] = __uint_as_float(v.w);
+    }
+    // 16 bytes as fp32 pairs (element 2k in the low half of pair k)
+    __device__ static void unpack2(const uint4& v, uint64_t* x) {
+        x[0] = pack2u(v.x, v.y);
+        x[1] = pack2u(v.z, v.w);
     }
     __device__ static float load1(const char* p) { return __ldg(reinterpret_cast<const float*>(p)); }
     __device__ static void store1(char* p, float x) { *reinterpret_cast<float*>(p) = x; }
@@ -102,6 +164,12 @@ struct Elem<__nv_bfloat16> {
         unpack_bf16x2(v.z, f + 4);
         unpack_bf16x2(v.w, f + 6);
     }
+    __device__ static void unpack2(const uint4& v, uint64_t* x) {
+        x[0] = pack2u(v.x << 16, v.x & 0xffff0000u);
+        x[1] = pack2u(v.y << 16, v.y & 0xffff0000u);
+        x[2] = pack2u(v.z << 16, v.z & 0xffff0000u);
+        x[3] = pack2u(v.w << 16, v.w & 0xffff0000u);
+    }
     __device__ static float load1(const char* p) {
         const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
         return __uint_as_float((uint32_t)u << 16);
@@ -125,6 +193,12 @@ struct Elem<__half> {
         unpack_f16x2(v.y, f + 2);
         unpack_f16x2(v.z, f + 4);
         unpack_f16x2(v.w, f + 6);
+    }
+    __device__ static void unpack2(const uint4& v, uint64_t* x) {
+        float f[8];
+        unpack(v, f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = pack2f(f[2 * k], f[2 * k + 1]);
     }
     __device__ static float load1(const char* p) {
         const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
@@ -185,24 +259,28 @@ __device__ __forceinline__ float group_sum(float v, int lanes) {
 // the 16-byte column v = slice*lanes + j of every partial row.  Control flow
 // that reaches a shuffle depends only on R, lanes and RC, which are the same
 // for every thread of the grid, so every shuffle sees all 32 lanes.
+// Programmatic dependent launch: wait for the previous grid in the stream
+// (and its memory) before the first global access, and let the next grid be
+// scheduled as soon as every CTA of this one is running.  Both are no-ops
+// for a launch without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 template <typename TIn, typename TOut, int RC>
-__global__ void __launch_bounds__(kBlock) merge_vec_kernel(const KParams p) {
+__global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KParams p) {
     constexpr int N = Elem<TIn>::kVec;
+    constexpr int N2 = N / 2;
+    pdl_wait();
+    pdl_release();
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t grp = t >> p.lg;
     const int j = (int)(t & (p.lanes - 1));
     const bool live = grp < p.groups;
-    int64_t row = 0;
-    int slice = 0;
-    if (live) {
-        row = grp / p.spr;
-        slice = (int)(grp - row * p.spr);
-    }
-    const int64_t b = row / p.H, h = row - b * p.H;
-    const int v = slice * p.lanes + j;
+    const RowIdx ri = row_of(p, live ? grp : 0);
+    const int v = ri.slice * p.lanes + j;
     const bool vlive = live && v < p.dv;
-    const char* orow = p.o + b * p.o_b + h * p.o_h + (int64_t)v * 16;
-    const float* lrow = p.lse + b * p.l_b + h * p.l_h;
+    const char* orow = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)v * 16;
+    const float* lrow = p.lse + ri.b * p.l_b + ri.h * p.l_h;
 
     // Partial rows 0..RC-1 go in flight first; nothing here waits on lse.
     uint4 x[RC];
@@ -223,9 +301,9 @@ __global__ void __launch_bounds__(kBlock) merge_vec_kernel(const KParams p) {
     // exp(-inf) = 0 rather than exp(-inf + inf) = NaN.
     const float mref = (m == -INFINITY) ? 0.f : m;
 
-    float acc[N];
+    uint64_t acc[N2];
 #pragma unroll
-    for (int k = 0; k < N; ++k) acc[k] = 0.f;
+    for (int k = 0; k < N2; ++k) acc[k] = 0ull;
     float esum = 0.f;
 
     for (int c = 0; c < p.R; c += p.lanes) {
@@ -237,6 +315,10 @@ __global__ void __launch_bounds__(kBlock) merge_vec_kernel(const KParams p) {
         const float e = expf(l - mref);  // weight of partial c+j; 0 for an empty shard
         esum += e;
         const int cn = min(p.R - c, p.lanes);
+        // Warp-uniform: does any group of this warp have a zero weight in this
+        // chunk?  Only then is the per-partial test needed (a partial of weight
+        // 0 may hold NaN and must not reach the sum).
+        const bool any_zero = __any_sync(kFull, j < cn && e == 0.f);
         for (int s0 = 0; s0 < cn; s0 += RC) {
             if (c > 0 || s0 > 0) {
 #pragma unroll
@@ -246,11 +328,12 @@ __global__ void __launch_bounds__(kBlock) merge_vec_kernel(const KParams p) {
 #pragma unroll
             for (int i = 0; i < RC; ++i) {
                 const float w = __shfl_sync(kFull, e, s0 + i, p.lanes);
-                if (s0 + i < cn && w != 0.f) {
-                    float f[N];
-                    Elem<TIn>::unpack(x[i], f);
+                if (s0 + i < cn && (!any_zero || w != 0.f)) {
+                    uint64_t xx[N2];
+                    Elem<TIn>::unpack2(x[i], xx);
+                    const uint64_t ww = pack2f(w, w);
 #pragma unroll
-                    for (int k = 0; k < N; ++k) acc[k] = fmaf(w, f[k], acc[k]);
+                    for (int k = 0; k < N2; ++k) fma2(acc[k], xx[k], ww);
                 }
             }
         }
@@ -260,11 +343,113 @@ __global__ void __launch_bounds__(kBlock) merge_vec_kernel(const KParams p) {
     // esum >= 1 for a row with a finite max (its own weight is exp(0)).
     const float inv = esum > 0.f ? 1.f / esum : 0.f;
     if (vlive) {
+        float f[N];
 #pragma unroll
-        for (int k = 0; k < N; ++k) acc[k] *= inv;
-        store_vec<TOut, N>(p.out + (row * p.D + (int64_t)v * N) * (int64_t)sizeof(TOut), acc);
+        for (int k = 0; k < N2; ++k) {
+            unpack2f(acc[k], f[2 * k], f[2 * k + 1]);
+            f[2 * k] *= inv;
+            f[2 * k + 1] *= inv;
+        }
+        store_vec<TOut, N>(p.out + (ri.row * p.D + (int64_t)v * N) * (int64_t)sizeof(TOut), f);
     }
-    if (live && slice == 0 && j == 0) p.out_lse[row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+    if (live && ri.slice == 0 && j == 0) p.out_lse[ri.row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+}
+
+
+// ------------------------------------------------------------------ stream kernel
+
+// Persistent form of the vector kernel for R <= RC: each lane group walks
+// the row slices grp, grp + G, grp + 2G, ... (G groups in the grid).  As soon
+// as partial i of the current slice has been folded into the accumulator,
+// its register is refilled with partial i of the next slice, so every lane
+// keeps up to R 16-byte loads in flight across slice boundaries and no warp
+// ever waits for a CTA to retire or launch.
+template <typename TIn, typename TOut, int RC>
+__global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const KParams p, const int64_t G) {
+    constexpr int N = Elem<TIn>::kVec;
+    constexpr int N2 = N / 2;
+    pdl_wait();
+    pdl_release();
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int j = (int)(t & (p.lanes - 1));
+    // The first group of a warp has the most slices: a warp-uniform trip count
+    // keeps every shuffle convergent; groups past their last slice idle.
+    const int64_t grp0 = t >> p.lg;
+    const int64_t grp_w = (t & ~(int64_t)31) >> p.lg;
+    const int64_t trips = grp_w < p.groups ? (p.groups - grp_w + G - 1) / G : 0;
+
+    struct Slice {
+        const char* o;
+        const float* l;
+        int64_t row;
+        int v, slice;
+        bool live, vlive;
+    };
+    auto locate = [&](int64_t g) {
+        Slice s;
+        s.live = g < p.groups;
+        const RowIdx ri = row_of(p, s.live ? g : 0);
+        s.row = ri.row;
+        s.slice = ri.slice;
+        s.v = ri.slice * p.lanes + j;
+        s.vlive = s.live && s.v < p.dv;
+        s.o = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)s.v * 16;
+        s.l = p.lse + ri.b * p.l_b + ri.h * p.l_h;
+        return s;
+    };
+
+    Slice cur = locate(grp0);
+    uint4 x[RC];
+#pragma unroll
+    for (int i = 0; i < RC; ++i) {
+        x[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (cur.vlive && i < p.R) x[i] = ld_stream16(cur.o + (int64_t)i * p.o_r);
+    }
+    float l = (cur.live && j < p.R) ? __ldg(cur.l + (int64_t)j * p.l_r) : -INFINITY;
+
+    for (int64_t k = 0; k < trips; ++k) {
+        const Slice nxt = locate(grp0 + (k + 1) * G);
+        const float ln = (nxt.live && j < p.R) ? __ldg(nxt.l + (int64_t)j * p.l_r) : -INFINITY;
+
+        const float m = group_max(l, p.lanes);
+        const float mref = (m == -INFINITY) ? 0.f : m;
+        const float e = expf(l - mref);
+        const float esum = group_sum(e, p.lanes);
+        const bool any_zero = __any_sync(kFull, j < p.R && e == 0.f);
+
+        uint64_t acc[N2];
+#pragma unroll
+        for (int q = 0; q < N2; ++q) acc[q] = 0ull;
+#pragma unroll
+        for (int i = 0; i < RC; ++i) {
+            const float w = __shfl_sync(kFull, e, i, p.lanes);
+            if (i < p.R) {
+                if (!any_zero || w != 0.f) {
+                    uint64_t xx[N2];
+                    Elem<TIn>::unpack2(x[i], xx);
+                    const uint64_t ww = pack2f(w, w);
+#pragma unroll
+                    for (int q = 0; q < N2; ++q) fma2(acc[q], xx[q], ww);
+                }
+                if (nxt.vlive) x[i] = ld_stream16(nxt.o + (int64_t)i * p.o_r);
+            }
+        }
+        const float inv = esum > 0.f ? 1.f / esum : 0.f;
+        if (cur.vlive) {
+            float f[N];
+#pragma unroll
+            for (int q = 0; q < N2; ++q) {
+                unpack2f(acc[q], f[2 * q], f[2 * q + 1]);
+                f[2 * q] *= inv;
+                f[2 * q + 1] *= inv;
+            }
+            store_vec<TOut, N>(p.out + (cur.row * p.D + (int64_t)cur.v * N) * (int64_t)sizeof(TOut), f);
+        }
+        if (cur.live && cur.slice == 0 && j == 0)
+            p.out_lse[cur.row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+        cur = nxt;
+        l = ln;
+    }
 }
 
 // ------------------------------------------------------------------ scalar kernel
@@ -273,6 +458,8 @@ __global__ void __launch_bounds__(kBlock) merge_vec_kernel(const KParams p) {
 // elements d = j, j+32, ...; element loads.
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kBlock) merge_scalar_kernel(const KParams p) {
+    pdl_wait();
+    pdl_release();
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t row = t >> 5;
     const int j = (int)(t & 31);
@@ -322,6 +509,70 @@ __global__ void __launch_bounds__(kBlock) merge_scalar_kernel(const KParams p) {
 // ------------------------------------------------------------------------ dispatch
 
 using KernelFn = void (*)(KParams);
+using StreamFn = void (*)(KParams, int64_t);
+
+template <typename TIn, typename TOut>
+StreamFn pick_stream_kernel(int rc) {
+    switch (rc) {
+        case 4: return merge_stream_kernel<TIn, TOut, 4>;
+        case 8: return merge_stream_kernel<TIn, TOut, 8>;
+        default: return merge_stream_kernel<TIn, TOut, 16>;
+    }
+}
+template <typename TIn>
+StreamFn pick_stream_out(int rc, int out_dtype) {
+    switch (out_dtype) {
+        case LSE_MERGE_F32: return pick_stream_kernel<TIn, float>(rc);
+        case LSE_MERGE_F16: return pick_stream_kernel<TIn, __half>(rc);
+        default: return pick_stream_kernel<TIn, __nv_bfloat16>(rc);
+    }
+}
+StreamFn pick_stream(int rc, int in_dtype, int out_dtype) {
+    switch (in_dtype) {
+        case LSE_MERGE_F32: return pick_stream_out<float>(rc, out_dtype);
+        case LSE_MERGE_F16: return pick_stream_out<__half>(rc, out_dtype);
+        default: return pick_stream_out<__nv_bfloat16>(rc, out_dtype);
+    }
+}
+
+// CTAs of `fn` that fit on one SM of the current device, and its SM count;
+// queried once per (device, kernel) and cached.
+struct OccEntry {
+    const void* fn;
+    int dev, ctas, sms;
+};
+constexpr int kOccSlots = 512;
+OccEntry g_occ[kOccSlots];
+int g_occ_n = 0;
+std::mutex g_occ_mu;
+
+int persistent_grid(const void* fn, int block, int64_t want_ctas, int* grid_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return (int)e;
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mu);
+        for (int i = 0; i < g_occ_n; ++i)
+            if (g_occ[i].fn == fn && g_occ[i].dev == dev) {
+                const int64_t g = (int64_t)g_occ[i].ctas * g_occ[i].sms;
+                *grid_out = (int)(want_ctas < g ? want_ctas : g);
+                return 0;
+            }
+    }
+    int ctas = 0, sms = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas, fn, block, 0);
+    if (e != cudaSuccess) return (int)e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return (int)e;
+    if (ctas < 1) ctas = 1;
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mu);
+        if (g_occ_n < kOccSlots) g_occ[g_occ_n++] = OccEntry{fn, dev, ctas, sms};
+    }
+    const int64_t g = (int64_t)ctas * sms;
+    *grid_out = (int)(want_ctas < g ? want_ctas : g);
+    return 0;
+}
 
 template <typename TIn, typename TOut>
 KernelFn pick_kernel(const lse_merge_plan& pl) {
@@ -388,15 +639,38 @@ int run(const void* partial_o, const float* partial_lse, int R, int B, int H, in
     kp.lg = log2i(pl.lanes);
     kp.spr = pl.slices_per_row;
     kp.groups = pl.groups;
+    kp.idx32 = (pl.groups < ((int64_t)1 << 32)) ? 1 : 0;
+    kp.c_spr = fastdiv_c((uint32_t)pl.slices_per_row);
+    kp.c_H = fastdiv_c((uint32_t)H);
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)pl.grid);
     cfg.blockDim = dim3((unsigned)pl.block);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, pick(pl, in_dtype, out_dtype), kp);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    const bool pdl = kPdl != 0;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e;
+    if (pl.path == LSE_MERGE_PATH_STREAM) {
+        const StreamFn fn = pick_stream(pl.rc, in_dtype, out_dtype);
+        const int64_t want = (pl.groups * pl.lanes + pl.block - 1) / pl.block;
+        int grid = 0;
+        const int qe = persistent_grid((const void*)fn, pl.block, want, &grid);
+        if (qe != 0) {
+            g_last_cuda_error = qe;
+            (void)cudaGetLastError();
+            return LSE_MERGE_ELAUNCH;
+        }
+        cfg.gridDim = dim3((unsigned)grid);
+        const int64_t G = (int64_t)grid * pl.block / pl.lanes;
+        e = cudaLaunchKernelEx(&cfg, fn, kp, G);
+    } else {
+        e = cudaLaunchKernelEx(&cfg, pick(pl, in_dtype, out_dtype), kp);
+    }
     if (e != cudaSuccess) {
         g_last_cuda_error = (int)e;
         (void)cudaGetLastError();  // the failure belongs to this call; do not leave it pending

@@ -70,7 +70,7 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
     if (!o || !lse || !out_o || !out_lse || !plan) return LSE_MERGE_ENULL;
     if (st.o_r < 0 || st.o_b < 0 || st.o_h < 0 || st.lse_r < 0 || st.lse_b < 0 || st.lse_h < 0)
         return LSE_MERGE_ESTRIDE;
-    if (path < LSE_MERGE_PATH_AUTO || path > LSE_MERGE_PATH_SCALAR) return LSE_MERGE_EPATH;
+    if (path < LSE_MERGE_PATH_AUTO || path > LSE_MERGE_PATH_STREAM) return LSE_MERGE_EPATH;
     if (!aligned(o, ib) || !aligned(out_o, ob) || !aligned(lse, 4) || !aligned(out_lse, 4))
         return LSE_MERGE_EALIGN;
 
@@ -106,9 +106,13 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
         const i128 groups = rows * slices;
         const i128 threads = groups * lanes;
         const bool small = threads <= kLatencyMaxThreads;
+        const bool stream_ok = R <= rc;   // every partial of a row slice in one batch
         int chosen = path;
-        if (chosen == LSE_MERGE_PATH_AUTO) chosen = small ? LSE_MERGE_PATH_LATENCY : LSE_MERGE_PATH_VECTOR;
+        if (chosen == LSE_MERGE_PATH_AUTO)
+            chosen = small ? LSE_MERGE_PATH_LATENCY
+                           : (kAutoStream && stream_ok ? LSE_MERGE_PATH_STREAM : LSE_MERGE_PATH_VECTOR);
         if (chosen == LSE_MERGE_PATH_LATENCY && !small) return LSE_MERGE_EPATH;
+        if (chosen == LSE_MERGE_PATH_STREAM && !stream_ok) return LSE_MERGE_EPATH;
         p.path = chosen;
         p.vec = vec;
         p.lanes = lanes;
@@ -118,6 +122,9 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
         if (chosen == LSE_MERGE_PATH_LATENCY) {
             p.block = (int)((threads + 31) / 32 * 32);
             p.grid = 1;
+        } else if (chosen == LSE_MERGE_PATH_STREAM) {
+            p.block = kBlock;
+            p.grid = 0;   // persistent: sized at launch from the device's occupancy
         } else {
             p.block = kBlock;
             const i128 grid = (threads + kBlock - 1) / kBlock;
@@ -125,7 +132,9 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
             p.grid = (int64_t)grid;
         }
     } else {
-        if (path == LSE_MERGE_PATH_VECTOR || path == LSE_MERGE_PATH_LATENCY) return LSE_MERGE_EPATH;
+        if (path == LSE_MERGE_PATH_VECTOR || path == LSE_MERGE_PATH_LATENCY ||
+            path == LSE_MERGE_PATH_STREAM)
+            return LSE_MERGE_EPATH;
         p.path = LSE_MERGE_PATH_SCALAR;
         p.vec = 1;
         p.lanes = 32;

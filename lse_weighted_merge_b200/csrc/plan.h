@@ -7,8 +7,32 @@
 
 namespace lsem {
 
-// Threads per CTA of the throughput (vector) and scalar kernels.
-constexpr int kBlock = 256;
+// Threads per CTA of the throughput (vector) and scalar kernels.  Small CTAs
+// retire warp by warp: a finished 2-warp CTA frees its registers at once,
+// where an 8-warp CTA holds them until its slowest warp ends (measured on
+// B200: 64 threads 0.79, 128 threads 0.75, 256 threads 0.71 of the HBM copy
+// peak on the R=16 B=512 H=16 D=512 merge, before launch overlap).
+#ifndef LSEM_BLOCK
+#define LSEM_BLOCK 64
+#endif
+constexpr int kBlock = LSEM_BLOCK;
+// Lower bound on resident CTAs per SM given to __launch_bounds__ (caps registers).
+#ifndef LSEM_MINB
+#define LSEM_MINB 1
+#endif
+constexpr int kMinBlocks = LSEM_MINB;
+// Launch with programmatic stream serialization (the next kernel in the
+// stream may be scheduled while this one drains; it waits before touching
+// memory).  Hides the launch gap between back-to-back merges.
+#ifndef LSEM_PDL
+#define LSEM_PDL 1
+#endif
+constexpr int kPdl = LSEM_PDL;
+// Let AUTO pick the persistent STREAM kernel for problems beyond one CTA.
+#ifndef LSEM_AUTO_STREAM
+#define LSEM_AUTO_STREAM 0
+#endif
+constexpr int kAutoStream = LSEM_AUTO_STREAM;
 // Largest launch the latency path runs as a single CTA (the kernels are
 // compiled with __launch_bounds__(kBlock), so one CTA holds at most kBlock).
 constexpr int kLatencyMaxThreads = kBlock;

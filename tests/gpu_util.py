@@ -7,7 +7,10 @@ Tolerance (written here once, used by every GPU test):
     (bf16) or 2^-12 |x| (fp16);
   * fp32 output: |gpu - oracle| <= 1e-5 * (1 + |oracle|); fp32 accumulation
     of R products adds about R * 2^-24 * max|o| at worst;
-  * merged lse: |gpu - oracle| <= 1e-5 absolute;
+  * merged lse: |gpu - oracle| <= max(1e-5, 2^-22 |oracle|): 1e-5 absolute
+    wherever fp32 can hold it (|lse| < 41.9, which covers every workload);
+    beyond that two fp32 ulps, since the fp32 output itself cannot be closer
+    than half an ulp (3e-5 at |lse| = 1000);
   * a row whose shards are all empty: out exactly 0 and lse exactly -inf;
   * no NaN anywhere unless an input lse is NaN or +inf.
 """
@@ -71,12 +74,13 @@ def check(got, got_lse, want, want_lse, out_dtype: str, what: str = "") -> dict:
     empty = want_lse == -np.inf
     assert np.array_equal(got_lse == -np.inf, empty), f"{what}: -inf rows differ"
     assert np.all(got[empty] == 0.0), f"{what}: an all-empty row is not 0"
-    lerr = np.abs(got_lse[~empty] - want_lse[~empty])
+    wl = want_lse[~empty]
+    lerr = np.abs(got_lse[~empty] - wl) / np.maximum(LSE_TOL, 2.0 ** -22 * np.abs(wl))
     lworst = float(lerr.max()) if lerr.size else 0.0
-    assert lworst <= LSE_TOL, f"{what}: max |lse err| = {lworst:.3e} > {LSE_TOL:g}"
+    assert lworst <= 1.0, f"{what}: lse error {lworst:.3f} x its bound"
     big = np.abs(want) > 1e-2
     rel = float((np.abs(got - want)[big] / np.abs(want[big])).max()) if big.any() else 0.0
-    return {"max_scaled_err": worst, "max_lse_err": lworst, "max_rel_err": rel,
+    return {"max_scaled_err": worst, "lse_err_over_bound": lworst, "max_rel_err": rel,
             "empty_rows": int(empty.sum())}
 
 

@@ -60,7 +60,10 @@ def q(R=2, B=1, H=2, D=64, strides=None, i=nat.BF16, o=nat.BF16, po=PO, pl=PL, o
     (dict(out=PO + 64), nat.EALIAS), (dict(outl=PL), nat.EALIAS), (dict(outl=OUT + 8), nat.EALIAS),
     (dict(out=PL), nat.EALIAS),
     (dict(path=7), nat.EPATH),
+    (dict(R=17, B=64, H=64, path=nat.PATH_STREAM), nat.EPATH),
+    (dict(D=60, path=nat.PATH_STREAM), nat.EPATH),
     (dict(B=64, H=64, path=nat.PATH_LATENCY), nat.EPATH),
+    (dict(B=1, H=16, path=nat.PATH_LATENCY), nat.EPATH),     # 128 threads > one 64-thread CTA
     (dict(D=60, path=nat.PATH_VECTOR), nat.EPATH),
     (dict(po=PO + 2, path=nat.PATH_VECTOR), nat.EPATH),
     (dict(R=2 ** 30, B=2 ** 30, H=2 ** 30, D=2 ** 30), nat.EDIMS),
@@ -84,12 +87,13 @@ def test_rejected_calls_return_before_any_cuda_call():
 
 
 def test_plans_of_the_five_workloads():
+    blk = 64
     expect = {  # name -> (path, lanes, rc, slices, block, grid)
         "r2_b1_h2_d64": (nat.PATH_LATENCY, 8, 4, 1, 32, 1),
-        "r8_b1_h8_d128": (nat.PATH_LATENCY, 16, 8, 1, 128, 1),
-        "r4_b64_h32_d128_masked": (nat.PATH_VECTOR, 16, 4, 1, 256, 64 * 32 * 16 // 256),
-        "r8_b256_h64_d128_rankmajor": (nat.PATH_VECTOR, 16, 8, 1, 256, 256 * 64 * 16 // 256),
-        "r16_b512_h16_d512": (nat.PATH_VECTOR, 32, 16, 2, 256, 512 * 16 * 2 * 32 // 256),
+        "r8_b1_h8_d128": (nat.PATH_VECTOR, 16, 8, 1, blk, 8 * 16 // blk),
+        "r4_b64_h32_d128_masked": (nat.PATH_VECTOR, 16, 4, 1, blk, 64 * 32 * 16 // blk),
+        "r8_b256_h64_d128_rankmajor": (nat.PATH_VECTOR, 16, 8, 1, blk, 256 * 64 * 16 // blk),
+        "r16_b512_h16_d512": (nat.PATH_VECTOR, 32, 16, 2, blk, 512 * 16 * 2 * 32 // blk),
     }
     for name, w in synth.WORKLOADS.items():
         st = synth.strides(w.layout, w.R, w.B, w.H, w.D)
@@ -113,11 +117,13 @@ def test_fallback_to_scalar_and_forced_paths():
     # f32 input: 4 elements per vector; bf16 out then needs 8-byte alignment
     assert q(i=nat.F32, D=12)[1]["vec"] == 4
     assert q(i=nat.F32, o=nat.BF16, out=OUT + 8)[1]["path"] == nat.PATH_LATENCY
-    for path in (nat.PATH_VECTOR, nat.PATH_LATENCY, nat.PATH_SCALAR):
+    for path in (nat.PATH_VECTOR, nat.PATH_LATENCY, nat.PATH_SCALAR, nat.PATH_STREAM):
         rc, plan = q(path=path)
         assert rc == 0 and plan["path"] == path
+    rc, plan = q(B=64, H=64, R=16, path=nat.PATH_STREAM)
+    assert rc == 0 and plan["grid"] == 0 and plan["rc"] == 16
     rc, plan = q(B=64, H=64, path=nat.PATH_SCALAR)
-    assert plan["grid"] == 64 * 64 * 32 // 256 and plan["lanes"] == 32
+    assert plan["grid"] == 64 * 64 * 32 // plan["block"] and plan["lanes"] == 32
 
 
 @pytest.mark.parametrize("R,want_rc,want_lanes", [(1, 4, 8), (3, 4, 8), (5, 8, 8), (9, 16, 16),

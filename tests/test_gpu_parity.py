@@ -33,21 +33,23 @@ def test_workload_full_size(name):
 
 
 @pytest.mark.parametrize("name", list(W))
-@pytest.mark.parametrize("path", [nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_LATENCY])
+@pytest.mark.parametrize("path", [nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_LATENCY,
+                                  nat.PATH_STREAM])
 def test_workload_every_path(name, path):
     w = W[name]
-    # a reduced batch keeps the scalar path and the one-CTA latency path quick
+    # a reduced batch keeps the scalar path quick; the latency path is one CTA
     B = 1 if path == nat.PATH_LATENCY else min(w.B, 8)
-    H = min(w.H, 4) if path == nat.PATH_LATENCY else w.H
+    H = 1 if path == nat.PATH_LATENCY else w.H
     inp = synth.make_inputs(w, B=B, H=H, seed=w.seed + 17)
     parity(inp, path=path, what=f"{name}/{path}")
 
 
 def test_empty_shards_poisoned_with_nan():
     w = W["r4_b64_h32_d128_masked"]
-    for path in (nat.PATH_AUTO, nat.PATH_SCALAR):
+    for path in (nat.PATH_AUTO, nat.PATH_SCALAR, nat.PATH_VECTOR, nat.PATH_STREAM):
         inp = synth.make_inputs(w, poison_empty=True)
-        assert (inp["o"] == 0x7fc0).any()          # bf16 NaN bit pattern is present
+        o = inp["o"]
+        assert (((o & 0x7f80) == 0x7f80) & ((o & 0x7f) != 0)).any()   # bf16 NaNs are planted
         stats = parity(inp, path=path, what=f"poisoned/{path}")
         assert stats["empty_rows"] > 0
 
@@ -57,7 +59,7 @@ def test_empty_shards_poisoned_with_nan():
 def test_dtype_pairs(in_dt, out_dt):
     base = W["r8_b1_h8_d128"]
     inp = synth.make_inputs(base, in_dtype=in_dt, out_dtype=out_dt, B=3, H=7, R=5, D=96)
-    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR):
+    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM):
         parity(inp, path=path, what=f"{in_dt}->{out_dt}/{path}")
 
 
@@ -68,6 +70,8 @@ def test_ragged_shapes(R, D):
     inp = synth.make_inputs(base, R=R, D=D, B=3, H=5, lse_args=(-30.0, 30.0), seed=R * 1000 + D)
     parity(inp, what=f"R{R}/D{D}")
     parity(inp, path=nat.PATH_SCALAR, what=f"R{R}/D{D}/scalar")
+    if R <= 16 and D % 8 == 0:
+        parity(inp, path=nat.PATH_STREAM, what=f"R{R}/D{D}/stream")
 
 
 @pytest.mark.parametrize("layout", ["bhrd", "rbhd"])
@@ -76,6 +80,15 @@ def test_many_rows_ragged_tail(layout):
     inp = synth.make_inputs(W["r2_b1_h2_d64"], R=6, B=37, H=41, D=192, layout=layout, seed=5)
     parity(inp, what=layout)
     parity(inp, path=nat.PATH_VECTOR, what=layout + "/vector")
+    parity(inp, path=nat.PATH_STREAM, what=layout + "/stream")
+
+
+@pytest.mark.parametrize("B,H", [(5, 1031), (1000, 3), (1, 65536)])
+def test_row_index_arithmetic(B, H):
+    # prime, small and power-of-two head counts: the row/head split of every group
+    inp = synth.make_inputs(W["r2_b1_h2_d64"], R=3, B=B, H=H, D=256, seed=B + H)
+    parity(inp, what=f"B{B}/H{H}")
+    parity(inp, path=nat.PATH_STREAM, what=f"B{B}/H{H}/stream")
 
 
 def test_r1_is_identity_on_gpu():
@@ -90,7 +103,7 @@ def test_r1_is_identity_on_gpu():
 def test_all_rows_empty():
     inp = synth.make_inputs(W["r8_b256_h64_d128_rankmajor"], B=2, H=3)
     inp["lse"][:] = -np.inf
-    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR):
+    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM):
         got, got_lse, _ = run_gpu(inp, path)
         assert np.all(got == 0.0) and not np.signbit(got).any()
         assert np.all(got_lse == -np.inf)
@@ -146,7 +159,7 @@ def test_outputs_written_exactly_in_bounds():
     d_o = torch.from_numpy(inp["o"].view(np.int16)).cuda()
     d_l = torch.from_numpy(inp["lse"]).cuda()
     pad = 4096
-    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR):
+    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM):
         canvas = torch.full((pad + B * H * D + pad,), 12345, dtype=torch.int16, device="cuda")
         lcanvas = torch.full((pad + B * H + pad,), 7.0, dtype=torch.float32, device="cuda")
         nat.merge_raw(d_o.data_ptr(), d_l.data_ptr(), R, B, H, D, (inp["o_strides"], inp["lse_strides"]),
@@ -165,6 +178,10 @@ def test_deterministic_and_stream_ordered():
     s = torch.cuda.Stream()
     b, bl, _ = run_gpu(inp, stream=s)
     assert np.array_equal(a, b) and np.array_equal(al, bl)
+    # every vector-family path computes the same sums in the same order
+    for path in (nat.PATH_VECTOR, nat.PATH_STREAM):
+        c, cl, _ = run_gpu(inp, path)
+        assert np.array_equal(a, c) and np.array_equal(al, cl)
 
 
 def test_split_attention_tiny_check():
