@@ -12,9 +12,9 @@ R*B*H*(D*2+4) + B*H*(D*4+4).  Rank 0 prints one JSON line.
             inputs resident in HBM; K eager launches timed with CUDA events on
             the launch stream, inputs and outputs rotated over enough buffer
             sets that each step misses L2 (max over ranks for N > 1).
-  e2e       the same metric through the public torch call with the step's
-            inputs copied from pinned host memory and the result copied back
-            inside the timed region.
+  e2e       the same metric through the public host-buffer call merge_host:
+            each step copies its partials from pinned host memory to the GPU
+            and the result back, in 8 batch slices overlapped with the merge.
   roofline  the kernel's achieved GB/s against the measured HBM copy peak.
   latency   eager and CUDA-graph-replayed us/call of the two tiny decode
             shapes; per-workload GB/s of the other shapes.
@@ -209,7 +209,7 @@ def profiled_traffic(workload: str):
     if fields.get("source_sha256") != kernel_source_sha():
         return None, "kernel changed since the ncu capture"
     try:
-        return int(fields["dram_bytes_per_launch"]), path
+        return int(fields["dram_bytes_per_launch"]), os.path.relpath(path, ROOT)
     except (KeyError, ValueError):
         return None, "summary has no dram_bytes_per_launch"
 
@@ -314,37 +314,28 @@ def time_graph(sets: DeviceSets, calls: int, replays: int, device) -> float:
     return us
 
 
-def time_e2e(inp: dict, steps: int, device) -> dict:
-    """Public torch call with per-step host->device inputs and device->host results."""
+def time_e2e(inp: dict, steps: int, device, chunks: int = 8) -> dict:
+    """The public host-buffer call (merge_host): every step copies the step's
+    partials from pinned host memory to the GPU, merges, and copies the result
+    back to pinned host memory, the copies overlapped with the merge."""
     import numpy as np
     import torch
-    from lse_weighted_merge_b200 import merge
+    from lse_weighted_merge_b200 import merge_host
     R, B, H, D = inp["R"], inp["B"], inp["H"], inp["D"]
     o = inp["o"]
     tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
     raw = torch.from_numpy(o.view(np.int16) if o.dtype == np.uint16 else o.view(np.int32))
-    h_o = raw.view(tdt[inp["in_dtype"]]).pin_memory()
-    h_l = torch.from_numpy(inp["lse"]).pin_memory()
-    d_o = torch.empty_like(h_o, device=device)
-    d_l = torch.empty_like(h_l, device=device)
-    out = torch.empty((B, H, D), dtype=tdt[inp["out_dtype"]], device=device)
-    out_lse = torch.empty((B, H), dtype=torch.float32, device=device)
-    h_out = torch.empty_like(out, device="cpu").pin_memory()
-    h_out_lse = torch.empty_like(out_lse, device="cpu").pin_memory()
     layout = inp["workload"].layout
-
-    def view(t_o, t_l):
-        if layout == "bhrd":
-            return t_o.view(B, H, R, D), t_l.view(B, H, R)
-        return t_o.view(R, B, H, D), t_l.view(R, B, H)
+    shape_o = (B, H, R, D) if layout == "bhrd" else (R, B, H, D)
+    shape_l = (B, H, R) if layout == "bhrd" else (R, B, H)
+    h_o = raw.view(tdt[inp["in_dtype"]]).reshape(shape_o).pin_memory()
+    h_l = torch.from_numpy(inp["lse"]).reshape(shape_l).pin_memory()
+    h_out = torch.empty((B, H, D), dtype=tdt[inp["out_dtype"]]).pin_memory()
+    h_out_lse = torch.empty((B, H), dtype=torch.float32).pin_memory()
 
     def step():
-        d_o.copy_(h_o, non_blocking=True)
-        d_l.copy_(h_l, non_blocking=True)
-        vo, vl = view(d_o, d_l)
-        merge(vo, vl, layout=layout, out_dtype=tdt[inp["out_dtype"]], out=out, out_lse=out_lse)
-        h_out.copy_(out, non_blocking=True)
-        h_out_lse.copy_(out_lse, non_blocking=True)
+        merge_host(h_o, h_l, layout=layout, out_dtype=tdt[inp["out_dtype"]], chunks=chunks,
+                   device=device, out=h_out, out_lse=h_out_lse, sync=False)
 
     for _ in range(2):
         step()
@@ -361,7 +352,7 @@ def time_e2e(inp: dict, steps: int, device) -> dict:
     return {"ms_per_step": ms, "gbs": w.bytes_total() / (ms * 1e-3) / 1e9,
             "h2d_bytes_per_step": int(h_o.numel() * h_o.element_size() + h_l.numel() * 4),
             "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size() + h_out_lse.numel() * 4),
-            "steps": steps}
+            "steps": steps, "chunks": chunks}
 
 
 def sample_inputs(inp: dict, batches: int) -> dict:
@@ -507,7 +498,8 @@ def run_ours(args):
         e2e = {"value": bytes_step * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": r["h2d_bytes_per_step"],
                "d2h_bytes_per_step": r["d2h_bytes_per_step"], "ms_per_step": ms_e2e,
-               "steps": r["steps"], "api": "lse_weighted_merge_b200.merge (torch tensors)"}
+               "steps": r["steps"], "chunks": r["chunks"],
+               "api": "lse_weighted_merge_b200.merge_host (pinned host tensors in and out)"}
 
     extra = {}
     if not args.no_extra:

@@ -69,3 +69,117 @@ def merge(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, out=N
               dtype_code(partial_o.dtype), dtype_code(out_dtype), out.data_ptr(),
               out_lse.data_ptr(), stream, path)
     return out, out_lse
+
+
+_STREAMS: dict = {}
+_WORKSPACE: dict = {}
+
+
+def release_host_workspace() -> None:
+    """Free the device staging buffers merge_host keeps between calls."""
+    _WORKSPACE.clear()
+
+
+def _workspace(device, o_shape, o_dtype, l_shape, B, H, D, out_dtype):
+    """Device staging buffers of merge_host, kept per device for the last
+    shape used (allocating them on every call would stall the stream on the
+    allocator).  Reuse is ordered by the streams: a call's first copy waits
+    for the previous call's last copy."""
+    import torch
+    key = (o_shape, o_dtype, l_shape, B, H, D, out_dtype)
+    ws = _WORKSPACE.get(device)
+    if ws is None or ws["key"] != key:
+        if ws is not None:
+            ws["done"].synchronize()   # the old buffers may still be in use
+        ws = {"key": key, "done": torch.cuda.Event(),
+              "bufs": (torch.empty(o_shape, dtype=o_dtype, device=device),
+                       torch.empty(l_shape, dtype=torch.float32, device=device),
+                       torch.empty((B, H, D), dtype=out_dtype, device=device),
+                       torch.empty((B, H), dtype=torch.float32, device=device))}
+        ws["done"].record(torch.cuda.current_stream(device))
+        _WORKSPACE[device] = ws
+    return ws
+
+
+def _side_streams(device):
+    import torch
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    if key not in _STREAMS:
+        _STREAMS[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device),
+                         torch.cuda.Stream(device))
+    return _STREAMS[key]
+
+
+def merge_host(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, chunks: int = 8,
+               device=None, out=None, out_lse=None, sync: bool = True):
+    """Merge partials that live in (pinned) host memory; results land in host memory.
+
+    The batch is cut into ``chunks`` slices along B.  Slice i is copied to the
+    GPU on one stream while slice i-1 is merged (one kernel launch on a second
+    stream) and slice i-2's result is copied back on a third, so the merge and
+    the device-to-host copies hide behind the host-to-device copy of the
+    partials, which bounds the whole call.  Layouts and dtypes as in merge().
+
+    Device staging buffers for one call's shapes are kept between calls (see
+    release_host_workspace); pass pinned ``out``/``out_lse`` to avoid a host
+    allocation per call.
+
+    Returns pinned host tensors (out [B, H, D], out_lse [B, H]).  With
+    ``sync=False`` the call returns once everything is enqueued; the current
+    stream of ``device`` is made to wait for the last copy, so synchronising
+    that stream (or the device) makes the results valid.
+    """
+    import torch
+    if partial_o.is_cuda or partial_lse.is_cuda:
+        raise ValueError("merge_host takes host tensors; use merge() for device tensors")
+    if partial_lse.dtype != torch.float32:
+        raise TypeError("partial_lse must be float32")
+    (R, B, H, D), _ = _rbh_strides(partial_o, partial_lse, layout)
+    if not (partial_o.is_contiguous() and partial_lse.is_contiguous()):
+        raise ValueError("merge_host wants contiguous host tensors")
+    device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    out_dtype = out_dtype or partial_o.dtype
+    if out is None:
+        out = torch.empty((B, H, D), dtype=out_dtype).pin_memory()
+    if out_lse is None:
+        out_lse = torch.empty((B, H), dtype=torch.float32).pin_memory()
+    ws = _workspace(device, tuple(partial_o.shape), partial_o.dtype, tuple(partial_lse.shape),
+                    B, H, D, out_dtype)
+    d_o, d_l, d_out, d_out_lse = ws["bufs"]
+    cur = torch.cuda.current_stream(device)
+    s_in, s_merge, s_back = _side_streams(device)
+    # The staging buffers are free once the previous call's last copy is done
+    # (its `done` event); the host outputs may be in use on the current stream.
+    for s_ in (s_in, s_back):
+        s_.wait_event(ws["done"])
+        s_.wait_stream(cur)
+    nb = max(1, -(-B // max(1, int(chunks))))
+    for b0 in range(0, B, nb):
+        b1 = min(B, b0 + nb)
+        with torch.cuda.stream(s_in):
+            if layout == "bhrd":
+                d_o[b0:b1].copy_(partial_o[b0:b1], non_blocking=True)
+                d_l[b0:b1].copy_(partial_lse[b0:b1], non_blocking=True)
+                vo, vl = d_o[b0:b1], d_l[b0:b1]
+            else:
+                for r in range(R):
+                    d_o[r, b0:b1].copy_(partial_o[r, b0:b1], non_blocking=True)
+                    d_l[r, b0:b1].copy_(partial_lse[r, b0:b1], non_blocking=True)
+                vo, vl = d_o[:, b0:b1], d_l[:, b0:b1]
+            landed = torch.cuda.Event()
+            landed.record(s_in)
+        s_merge.wait_event(landed)
+        with torch.cuda.stream(s_merge):
+            merge(vo, vl, layout=layout, out_dtype=out_dtype, out=d_out[b0:b1],
+                  out_lse=d_out_lse[b0:b1])
+            merged = torch.cuda.Event()
+            merged.record(s_merge)
+        s_back.wait_event(merged)
+        with torch.cuda.stream(s_back):
+            out[b0:b1].copy_(d_out[b0:b1], non_blocking=True)
+            out_lse[b0:b1].copy_(d_out_lse[b0:b1], non_blocking=True)
+    ws["done"].record(s_back)
+    cur.wait_stream(s_back)
+    if sync:
+        s_back.synchronize()
+    return out, out_lse
