@@ -121,6 +121,7 @@ typedef struct {
     int vec;             /* elements per lane per partial load (16 B / elem size; 1 for scalar) */
     int lanes;           /* lanes that share one row slice (power of two, <= 32) */
     int rc;              /* partial rows whose loads are in flight together per lane */
+    int nv;              /* 16-byte columns per lane in every partial row (rc * nv <= 16) */
     int slices_per_row;  /* row slices (lane groups) that cover one row of D */
     int block;           /* threads per CTA */
     int64_t grid;        /* CTAs; 0 for STREAM, whose persistent grid is sized at
@@ -144,7 +145,7 @@ int lse_merge_last_cuda_error(void);
 /* ABI version of this header; bumped on any incompatible change. */
 int lse_merge_version(void);
 
-#define LSE_MERGE_ABI_VERSION 1
+#define LSE_MERGE_ABI_VERSION 2
 
 #ifdef __cplusplus
 }

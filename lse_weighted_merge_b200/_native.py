@@ -22,7 +22,7 @@ OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH = 0, -1, -2, -
 # Every symbol include/lse_merge.h declares.
 EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merge_strerror",
            "lse_merge_last_cuda_error", "lse_merge_version")
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 
 class Strides(ctypes.Structure):
@@ -32,7 +32,8 @@ class Strides(ctypes.Structure):
 
 class Plan(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int), ("vec", ctypes.c_int), ("lanes", ctypes.c_int),
-                ("rc", ctypes.c_int), ("slices_per_row", ctypes.c_int), ("block", ctypes.c_int),
+                ("rc", ctypes.c_int), ("nv", ctypes.c_int), ("slices_per_row", ctypes.c_int),
+                ("block", ctypes.c_int),
                 ("grid", ctypes.c_int64), ("groups", ctypes.c_int64)]
 
     def as_dict(self) -> dict:

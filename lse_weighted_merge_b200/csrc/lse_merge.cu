@@ -266,8 +266,43 @@ __device__ __forceinline__ float group_sum(float v, int lanes) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
+// Fold partial x (NV 16-byte columns) with weight w into acc.
+template <typename TIn, int NV, int N2>
+__device__ __forceinline__ void fold(uint64_t (&acc)[NV][N2], const uint4 (&x)[NV], float w) {
+    const uint64_t ww = pack2f(w, w);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        uint64_t xx[N2];
+        Elem<TIn>::unpack2(x[k], xx);
+#pragma unroll
+        for (int q = 0; q < N2; ++q) fma2(acc[k][q], xx[q], ww);
+    }
+}
+
+// Scale acc by inv and store the NV columns of this lane (those inside the row).
+template <typename TOut, int NV, int N, int N2>
+__device__ __forceinline__ void store_cols(const KParams& p, int64_t row, int v0, bool live,
+                                           const uint64_t (&acc)[NV][N2], float inv) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int v = v0 + k * p.lanes;
+        if (live && v < p.dv) {
+            float f[N];
+#pragma unroll
+            for (int q = 0; q < N2; ++q) {
+                unpack2f(acc[k][q], f[2 * q], f[2 * q + 1]);
+                f[2 * q] *= inv;
+                f[2 * q + 1] *= inv;
+            }
+            store_vec<TOut, N>(p.out + (row * p.D + (int64_t)v * N) * (int64_t)sizeof(TOut), f);
+        }
+    }
+}
+
+// One 16-byte column per lane (NV = 1), the form used whenever the planner
+// gives a lane a single column.
 template <typename TIn, typename TOut, int RC>
-__global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KParams p) {
+__global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec1_kernel(const KParams p) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
     pdl_wait();
@@ -356,15 +391,104 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KPa
 }
 
 
+// One group of p.lanes lanes merges one slice of one (b,h) row.  Lane j owns
+// the NV 16-byte columns v0 + k*lanes (v0 = slice*lanes*NV + j, k < NV) of
+// every partial row, so each warp load instruction reads lanes*16 contiguous
+// bytes of a partial row.  Control flow that reaches a shuffle depends only
+// on R, lanes, RC and NV, which are the same for every thread of the grid,
+// so every shuffle sees all 32 lanes.
+template <typename TIn, typename TOut, int RC, int NV>
+__global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KParams p) {
+    constexpr int N = Elem<TIn>::kVec;
+    constexpr int N2 = N / 2;
+    pdl_wait();
+    pdl_release();
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t grp = t >> p.lg;
+    const int j = (int)(t & (p.lanes - 1));
+    const bool live = grp < p.groups;
+    const RowIdx ri = row_of(p, live ? grp : 0);
+    const int v0 = ri.slice * p.lanes * NV + j;
+    const char* orow = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)v0 * 16;
+    const float* lrow = p.lse + ri.b * p.l_b + ri.h * p.l_h;
+    bool cl[NV];   // column k of this lane lies inside the row
+#pragma unroll
+    for (int k = 0; k < NV; ++k) cl[k] = live && v0 + k * p.lanes < p.dv;
+
+    // Partial rows 0..RC-1 go in flight first; nothing here waits on lse.
+    uint4 x[RC][NV];
+#pragma unroll
+    for (int i = 0; i < RC; ++i)
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            x[i][k] = make_uint4(0u, 0u, 0u, 0u);
+            if (cl[k] && i < p.R) x[i][k] = ld_stream16(orow + (int64_t)i * p.o_r + k * p.lanes * 16);
+        }
+
+    // m = max_r lse_r over the group (lane j reads lse_j, lse_{j+lanes}, ...).
+    float l0 = -INFINITY;
+    if (live && j < p.R) l0 = __ldg(lrow + (int64_t)j * p.l_r);
+    float m = l0;
+    for (int c = p.lanes; c < p.R; c += p.lanes)
+        if (live && c + j < p.R) m = fmaxf(m, __ldg(lrow + (int64_t)(c + j) * p.l_r));
+    m = group_max(m, p.lanes);
+    // An all-empty row has m = -inf; subtracting 0 instead keeps every weight
+    // exp(-inf) = 0 rather than exp(-inf + inf) = NaN.
+    const float mref = (m == -INFINITY) ? 0.f : m;
+
+    uint64_t acc[NV][N2];
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+        for (int q = 0; q < N2; ++q) acc[k][q] = 0ull;
+    float esum = 0.f;
+
+    for (int c = 0; c < p.R; c += p.lanes) {
+        float l = l0;
+        if (c > 0) {
+            l = -INFINITY;
+            if (live && c + j < p.R) l = __ldg(lrow + (int64_t)(c + j) * p.l_r);
+        }
+        const float e = expf(l - mref);  // weight of partial c+j; 0 for an empty shard
+        esum += e;
+        const int cn = min(p.R - c, p.lanes);
+        // Warp-uniform: does any group of this warp have a zero weight in this
+        // chunk?  Only then is the per-partial test needed (a partial of weight
+        // 0 may hold NaN and must not reach the sum).
+        const bool any_zero = __any_sync(kFull, j < cn && e == 0.f);
+        for (int s0 = 0; s0 < cn; s0 += RC) {
+            if (c > 0 || s0 > 0) {
+#pragma unroll
+                for (int i = 0; i < RC; ++i)
+#pragma unroll
+                    for (int k = 0; k < NV; ++k)
+                        if (cl[k] && s0 + i < cn)
+                            x[i][k] = ld_stream16(orow + (int64_t)(c + s0 + i) * p.o_r + k * p.lanes * 16);
+            }
+#pragma unroll
+            for (int i = 0; i < RC; ++i) {
+                const float w = __shfl_sync(kFull, e, s0 + i, p.lanes);
+                if (s0 + i < cn && (!any_zero || w != 0.f)) fold<TIn, NV, N2>(acc, x[i], w);
+            }
+        }
+    }
+    esum = group_sum(esum, p.lanes);
+
+    // esum >= 1 for a row with a finite max (its own weight is exp(0)).
+    const float inv = esum > 0.f ? 1.f / esum : 0.f;
+    store_cols<TOut, NV, N, N2>(p, ri.row, v0, live, acc, inv);
+    if (live && ri.slice == 0 && j == 0) p.out_lse[ri.row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+}
+
 // ------------------------------------------------------------------ stream kernel
 
 // Persistent form of the vector kernel for R <= RC: each lane group walks
 // the row slices grp, grp + G, grp + 2G, ... (G groups in the grid).  As soon
 // as partial i of the current slice has been folded into the accumulator,
-// its register is refilled with partial i of the next slice, so every lane
-// keeps up to R 16-byte loads in flight across slice boundaries and no warp
-// ever waits for a CTA to retire or launch.
-template <typename TIn, typename TOut, int RC>
+// its registers are refilled with partial i of the next slice, so every lane
+// keeps up to R*NV 16-byte loads in flight across slice boundaries and no
+// warp ever waits for a CTA to retire or launch.
+template <typename TIn, typename TOut, int RC, int NV>
 __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const KParams p, const int64_t G) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
@@ -382,8 +506,9 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const 
         const char* o;
         const float* l;
         int64_t row;
-        int v, slice;
-        bool live, vlive;
+        int v0, slice;
+        bool live;
+        bool cl[NV];
     };
     auto locate = [&](int64_t g) {
         Slice s;
@@ -391,24 +516,27 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const 
         const RowIdx ri = row_of(p, s.live ? g : 0);
         s.row = ri.row;
         s.slice = ri.slice;
-        s.v = ri.slice * p.lanes + j;
-        s.vlive = s.live && s.v < p.dv;
-        s.o = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)s.v * 16;
+        s.v0 = ri.slice * p.lanes * NV + j;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) s.cl[k] = s.live && s.v0 + k * p.lanes < p.dv;
+        s.o = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)s.v0 * 16;
         s.l = p.lse + ri.b * p.l_b + ri.h * p.l_h;
         return s;
     };
 
     Slice cur = locate(grp0);
-    uint4 x[RC];
+    uint4 x[RC][NV];
 #pragma unroll
-    for (int i = 0; i < RC; ++i) {
-        x[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (cur.vlive && i < p.R) x[i] = ld_stream16(cur.o + (int64_t)i * p.o_r);
-    }
+    for (int i = 0; i < RC; ++i)
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            x[i][k] = make_uint4(0u, 0u, 0u, 0u);
+            if (cur.cl[k] && i < p.R) x[i][k] = ld_stream16(cur.o + (int64_t)i * p.o_r + k * p.lanes * 16);
+        }
     float l = (cur.live && j < p.R) ? __ldg(cur.l + (int64_t)j * p.l_r) : -INFINITY;
 
-    for (int64_t k = 0; k < trips; ++k) {
-        const Slice nxt = locate(grp0 + (k + 1) * G);
+    for (int64_t it = 0; it < trips; ++it) {
+        const Slice nxt = locate(grp0 + (it + 1) * G);
         const float ln = (nxt.live && j < p.R) ? __ldg(nxt.l + (int64_t)j * p.l_r) : -INFINITY;
 
         const float m = group_max(l, p.lanes);
@@ -417,34 +545,23 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const 
         const float esum = group_sum(e, p.lanes);
         const bool any_zero = __any_sync(kFull, j < p.R && e == 0.f);
 
-        uint64_t acc[N2];
+        uint64_t acc[NV][N2];
 #pragma unroll
-        for (int q = 0; q < N2; ++q) acc[q] = 0ull;
+        for (int k = 0; k < NV; ++k)
+#pragma unroll
+            for (int q = 0; q < N2; ++q) acc[k][q] = 0ull;
 #pragma unroll
         for (int i = 0; i < RC; ++i) {
             const float w = __shfl_sync(kFull, e, i, p.lanes);
             if (i < p.R) {
-                if (!any_zero || w != 0.f) {
-                    uint64_t xx[N2];
-                    Elem<TIn>::unpack2(x[i], xx);
-                    const uint64_t ww = pack2f(w, w);
+                if (!any_zero || w != 0.f) fold<TIn, NV, N2>(acc, x[i], w);
 #pragma unroll
-                    for (int q = 0; q < N2; ++q) fma2(acc[q], xx[q], ww);
-                }
-                if (nxt.vlive) x[i] = ld_stream16(nxt.o + (int64_t)i * p.o_r);
+                for (int k = 0; k < NV; ++k)
+                    if (nxt.cl[k]) x[i][k] = ld_stream16(nxt.o + (int64_t)i * p.o_r + k * p.lanes * 16);
             }
         }
         const float inv = esum > 0.f ? 1.f / esum : 0.f;
-        if (cur.vlive) {
-            float f[N];
-#pragma unroll
-            for (int q = 0; q < N2; ++q) {
-                unpack2f(acc[q], f[2 * q], f[2 * q + 1]);
-                f[2 * q] *= inv;
-                f[2 * q + 1] *= inv;
-            }
-            store_vec<TOut, N>(p.out + (cur.row * p.D + (int64_t)cur.v * N) * (int64_t)sizeof(TOut), f);
-        }
+        store_cols<TOut, NV, N, N2>(p, cur.row, cur.v0, cur.live, acc, inv);
         if (cur.live && cur.slice == 0 && j == 0)
             p.out_lse[cur.row] = esum > 0.f ? m + logf(esum) : -INFINITY;
         cur = nxt;
@@ -511,27 +628,27 @@ __global__ void __launch_bounds__(kBlock) merge_scalar_kernel(const KParams p) {
 using KernelFn = void (*)(KParams);
 using StreamFn = void (*)(KParams, int64_t);
 
+// (rc, nv) pairs the planner produces: rc * nv <= 16 loads of 16 bytes per lane.
 template <typename TIn, typename TOut>
-StreamFn pick_stream_kernel(int rc) {
-    switch (rc) {
-        case 4: return merge_stream_kernel<TIn, TOut, 4>;
-        case 8: return merge_stream_kernel<TIn, TOut, 8>;
-        default: return merge_stream_kernel<TIn, TOut, 16>;
-    }
+StreamFn pick_stream_kernel(int rc, int nv) {
+    if (rc == 4) return nv == 4 ? merge_stream_kernel<TIn, TOut, 4, 4>
+                      : nv == 2 ? merge_stream_kernel<TIn, TOut, 4, 2> : merge_stream_kernel<TIn, TOut, 4, 1>;
+    if (rc == 8) return nv == 2 ? merge_stream_kernel<TIn, TOut, 8, 2> : merge_stream_kernel<TIn, TOut, 8, 1>;
+    return merge_stream_kernel<TIn, TOut, 16, 1>;
 }
 template <typename TIn>
-StreamFn pick_stream_out(int rc, int out_dtype) {
+StreamFn pick_stream_out(int rc, int nv, int out_dtype) {
     switch (out_dtype) {
-        case LSE_MERGE_F32: return pick_stream_kernel<TIn, float>(rc);
-        case LSE_MERGE_F16: return pick_stream_kernel<TIn, __half>(rc);
-        default: return pick_stream_kernel<TIn, __nv_bfloat16>(rc);
+        case LSE_MERGE_F32: return pick_stream_kernel<TIn, float>(rc, nv);
+        case LSE_MERGE_F16: return pick_stream_kernel<TIn, __half>(rc, nv);
+        default: return pick_stream_kernel<TIn, __nv_bfloat16>(rc, nv);
     }
 }
-StreamFn pick_stream(int rc, int in_dtype, int out_dtype) {
+StreamFn pick_stream(int rc, int nv, int in_dtype, int out_dtype) {
     switch (in_dtype) {
-        case LSE_MERGE_F32: return pick_stream_out<float>(rc, out_dtype);
-        case LSE_MERGE_F16: return pick_stream_out<__half>(rc, out_dtype);
-        default: return pick_stream_out<__nv_bfloat16>(rc, out_dtype);
+        case LSE_MERGE_F32: return pick_stream_out<float>(rc, nv, out_dtype);
+        case LSE_MERGE_F16: return pick_stream_out<__half>(rc, nv, out_dtype);
+        default: return pick_stream_out<__nv_bfloat16>(rc, nv, out_dtype);
     }
 }
 
@@ -546,6 +663,16 @@ OccEntry g_occ[kOccSlots];
 int g_occ_n = 0;
 std::mutex g_occ_mu;
 
+// Grid of a persistent kernel that would need `want_ctas` CTAs one-shot: at
+// most what fits on the device at once; with kBalance, the fewest CTAs that
+// still need the same number of rounds, so no round is left partial.
+int64_t balanced(int64_t want_ctas, int64_t capacity) {
+    if (want_ctas <= capacity) return want_ctas;
+    if (!kBalance) return capacity;
+    const int64_t rounds = (want_ctas + capacity - 1) / capacity;
+    return (want_ctas + rounds - 1) / rounds;
+}
+
 int persistent_grid(const void* fn, int block, int64_t want_ctas, int* grid_out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -554,8 +681,7 @@ int persistent_grid(const void* fn, int block, int64_t want_ctas, int* grid_out)
         std::lock_guard<std::mutex> lk(g_occ_mu);
         for (int i = 0; i < g_occ_n; ++i)
             if (g_occ[i].fn == fn && g_occ[i].dev == dev) {
-                const int64_t g = (int64_t)g_occ[i].ctas * g_occ[i].sms;
-                *grid_out = (int)(want_ctas < g ? want_ctas : g);
+                *grid_out = (int)balanced(want_ctas, (int64_t)g_occ[i].ctas * g_occ[i].sms);
                 return 0;
             }
     }
@@ -569,19 +695,18 @@ int persistent_grid(const void* fn, int block, int64_t want_ctas, int* grid_out)
         std::lock_guard<std::mutex> lk(g_occ_mu);
         if (g_occ_n < kOccSlots) g_occ[g_occ_n++] = OccEntry{fn, dev, ctas, sms};
     }
-    const int64_t g = (int64_t)ctas * sms;
-    *grid_out = (int)(want_ctas < g ? want_ctas : g);
+    *grid_out = (int)balanced(want_ctas, (int64_t)ctas * sms);
     return 0;
 }
 
 template <typename TIn, typename TOut>
 KernelFn pick_kernel(const lse_merge_plan& pl) {
     if (pl.path == LSE_MERGE_PATH_SCALAR) return merge_scalar_kernel<TIn, TOut>;
-    switch (pl.rc) {
-        case 4: return merge_vec_kernel<TIn, TOut, 4>;
-        case 8: return merge_vec_kernel<TIn, TOut, 8>;
-        default: return merge_vec_kernel<TIn, TOut, 16>;
-    }
+    const int rc = pl.rc, nv = pl.nv;
+    if (rc == 4) return nv == 4 ? merge_vec_kernel<TIn, TOut, 4, 4>
+                      : nv == 2 ? merge_vec_kernel<TIn, TOut, 4, 2> : merge_vec1_kernel<TIn, TOut, 4>;
+    if (rc == 8) return nv == 2 ? merge_vec_kernel<TIn, TOut, 8, 2> : merge_vec1_kernel<TIn, TOut, 8>;
+    return merge_vec1_kernel<TIn, TOut, 16>;
 }
 
 template <typename TIn>
@@ -656,7 +781,7 @@ int run(const void* partial_o, const float* partial_lse, int R, int B, int H, in
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e;
     if (pl.path == LSE_MERGE_PATH_STREAM) {
-        const StreamFn fn = pick_stream(pl.rc, in_dtype, out_dtype);
+        const StreamFn fn = pick_stream(pl.rc, pl.nv, in_dtype, out_dtype);
         const int64_t want = (pl.groups * pl.lanes + pl.block - 1) / pl.block;
         int grid = 0;
         const int qe = persistent_grid((const void*)fn, pl.block, want, &grid);

@@ -2,12 +2,14 @@
 //
 // Geometry of the vector kernels (the merge of one (b,h) row is spread over
 // a group of `lanes` consecutive lanes of one warp):
-//   * vec     = 16 bytes / element size: one 16-byte load per lane per partial;
-//   * lanes   = the power of two >= D/vec (at most 32), and at least rc so the
-//               lanes of a group can hold one lse value each for a batch;
-//   * slices  = ceil((D/vec) / lanes) groups per row when D/vec > 32;
-//   * rc      = 4, 8 or 16 partial rows loaded before the first FMA, so up to
-//               rc * 16 bytes per lane are in flight.
+//   * vec     = 16 bytes / element size: one 16-byte column of a row;
+//   * rc      = 4, 8 or 16 partial rows loaded before the first FMA;
+//   * nv      = 16-byte columns per lane in each partial row, 16 / rc, halved
+//               while it would leave fewer than rc lanes with work, so that a
+//               lane keeps rc * nv <= 16 loads (256 bytes) in flight;
+//   * lanes   = the power of two >= D / (vec * nv) (at most 32), and at least
+//               rc so the lanes of a group hold one lse value each per batch;
+//   * slices  = ceil((D/vec) / (lanes * nv)) groups per row.
 // The latency path is the same kernel launched as one CTA of exactly the
 // threads needed, for problems of at most kLatencyMaxThreads threads.
 #include "plan.h"
@@ -100,23 +102,42 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
     if (vec_ok && path != LSE_MERGE_PATH_SCALAR) {
         const int dv = D / vec;
         const int rc = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
-        int lanes = next_pow2(dv < 32 ? dv : 32);
-        if (lanes < rc) lanes = rc;
-        const int slices = (dv + lanes - 1) / lanes;
-        const i128 groups = rows * slices;
-        const i128 threads = groups * lanes;
-        const bool small = threads <= kLatencyMaxThreads;
+        // lanes and slices for nv columns per lane
+        auto shape = [&](int nv, int* lanes, int* slices) {
+            const int cols = (dv + nv - 1) / nv;
+            *lanes = next_pow2(cols < 32 ? cols : 32);
+            if (*lanes < rc) *lanes = rc;
+            *slices = (dv + *lanes * nv - 1) / (*lanes * nv);
+        };
+        // The latency path (one CTA) keeps one column per lane: for a
+        // problem that small, more threads beat more loads per thread.
+        int lanes1, slices1;
+        shape(1, &lanes1, &slices1);
+        const bool small = rows * slices1 * lanes1 <= kLatencyMaxThreads;
         const bool stream_ok = R <= rc;   // every partial of a row slice in one batch
+        const i128 in_bytes = (i128)R * rows * D * ib;
         int chosen = path;
         if (chosen == LSE_MERGE_PATH_AUTO)
             chosen = small ? LSE_MERGE_PATH_LATENCY
-                           : (kAutoStream && stream_ok ? LSE_MERGE_PATH_STREAM : LSE_MERGE_PATH_VECTOR);
+                           : (kAutoStream && stream_ok && in_bytes <= kStreamMaxBytes
+                                  ? LSE_MERGE_PATH_STREAM
+                                  : LSE_MERGE_PATH_VECTOR);
         if (chosen == LSE_MERGE_PATH_LATENCY && !small) return LSE_MERGE_EPATH;
         if (chosen == LSE_MERGE_PATH_STREAM && !stream_ok) return LSE_MERGE_EPATH;
+        int nv = 1;
+        if (chosen != LSE_MERGE_PATH_LATENCY) {
+            nv = 16 / rc < kMaxNv ? 16 / rc : kMaxNv;
+            while (nv > 1 && (dv + nv - 1) / nv < rc) nv >>= 1;
+        }
+        int lanes, slices;
+        shape(nv, &lanes, &slices);
+        const i128 groups = rows * slices;
+        const i128 threads = groups * lanes;
         p.path = chosen;
         p.vec = vec;
         p.lanes = lanes;
         p.rc = rc;
+        p.nv = nv;
         p.slices_per_row = slices;
         p.groups = (int64_t)groups;
         if (chosen == LSE_MERGE_PATH_LATENCY) {
@@ -139,6 +160,7 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
         p.vec = 1;
         p.lanes = 32;
         p.rc = 0;
+        p.nv = 1;
         p.slices_per_row = 1;
         p.groups = (int64_t)rows;
         p.block = kBlock;

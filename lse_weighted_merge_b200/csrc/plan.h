@@ -28,11 +28,30 @@ constexpr int kMinBlocks = LSEM_MINB;
 #define LSEM_PDL 1
 #endif
 constexpr int kPdl = LSEM_PDL;
-// Let AUTO pick the persistent STREAM kernel for problems beyond one CTA.
+// AUTO picks the persistent STREAM kernel for problems beyond one CTA whose
+// partials fit in kStreamMaxBytes, and the one-shot VECTOR kernel above that.
+// Measured on B200: STREAM is 4-6 % faster up to ~150 MB of partials, VECTOR
+// 3-6 % faster from ~300 MB on.
 #ifndef LSEM_AUTO_STREAM
-#define LSEM_AUTO_STREAM 0
+#define LSEM_AUTO_STREAM 1
 #endif
 constexpr int kAutoStream = LSEM_AUTO_STREAM;
+#ifndef LSEM_STREAM_MAX_MB
+#define LSEM_STREAM_MAX_MB 256
+#endif
+constexpr long long kStreamMaxBytes = (long long)LSEM_STREAM_MAX_MB << 20;
+// Upper bound on the 16-byte columns per lane (1, 2 or 4).
+#ifndef LSEM_MAX_NV
+#define LSEM_MAX_NV 2
+#endif
+constexpr int kMaxNv = LSEM_MAX_NV;
+// Size the persistent grid so that every CTA gets the same number of rounds
+// (ceil(work / capacity) rounds, spread evenly), instead of filling the
+// device and leaving a partial last round.
+#ifndef LSEM_BALANCE
+#define LSEM_BALANCE 1
+#endif
+constexpr int kBalance = LSEM_BALANCE;
 // Largest launch the latency path runs as a single CTA (the kernels are
 // compiled with __launch_bounds__(kBlock), so one CTA holds at most kBlock).
 constexpr int kLatencyMaxThreads = kBlock;

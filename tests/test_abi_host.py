@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strerror():
-    assert nat.lib.lse_merge_version() == nat.ABI_VERSION == 1
+    assert nat.lib.lse_merge_version() == nat.ABI_VERSION == 2
     for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
         assert nat.strerror(code) and "unknown lse_merge error" not in nat.strerror(code)
     assert "unknown lse_merge error" in nat.strerror(-99)
@@ -63,7 +63,7 @@ def q(R=2, B=1, H=2, D=64, strides=None, i=nat.BF16, o=nat.BF16, po=PO, pl=PL, o
     (dict(R=17, B=64, H=64, path=nat.PATH_STREAM), nat.EPATH),
     (dict(D=60, path=nat.PATH_STREAM), nat.EPATH),
     (dict(B=64, H=64, path=nat.PATH_LATENCY), nat.EPATH),
-    (dict(B=1, H=16, path=nat.PATH_LATENCY), nat.EPATH),     # 128 threads > one 64-thread CTA
+    (dict(B=1, H=32, path=nat.PATH_LATENCY), nat.EPATH),     # 128 threads > one 64-thread CTA
     (dict(D=60, path=nat.PATH_VECTOR), nat.EPATH),
     (dict(po=PO + 2, path=nat.PATH_VECTOR), nat.EPATH),
     (dict(R=2 ** 30, B=2 ** 30, H=2 ** 30, D=2 ** 30), nat.EDIMS),
@@ -88,23 +88,27 @@ def test_rejected_calls_return_before_any_cuda_call():
 
 def test_plans_of_the_five_workloads():
     blk = 64
-    expect = {  # name -> (path, lanes, rc, slices, block, grid)
-        "r2_b1_h2_d64": (nat.PATH_LATENCY, 8, 4, 1, 32, 1),
-        "r8_b1_h8_d128": (nat.PATH_VECTOR, 16, 8, 1, blk, 8 * 16 // blk),
-        "r4_b64_h32_d128_masked": (nat.PATH_VECTOR, 16, 4, 1, blk, 64 * 32 * 16 // blk),
-        "r8_b256_h64_d128_rankmajor": (nat.PATH_VECTOR, 16, 8, 1, blk, 256 * 64 * 16 // blk),
-        "r16_b512_h16_d512": (nat.PATH_VECTOR, 32, 16, 2, blk, 512 * 16 * 2 * 32 // blk),
+    expect = {  # name -> (path, lanes, rc, nv, slices, block, grid); STREAM grids are sized at launch
+        "r2_b1_h2_d64": (nat.PATH_LATENCY, 8, 4, 1, 1, 32, 1),
+        "r8_b1_h8_d128": (nat.PATH_STREAM, 8, 8, 2, 1, blk, 0),
+        "r4_b64_h32_d128_masked": (nat.PATH_STREAM, 8, 4, 2, 1, blk, 0),
+        "r8_b256_h64_d128_rankmajor": (nat.PATH_STREAM, 8, 8, 2, 1, blk, 0),
+        "r16_b512_h16_d512": (nat.PATH_STREAM, 32, 16, 1, 2, blk, 0),
     }
     for name, w in synth.WORKLOADS.items():
         st = synth.strides(w.layout, w.R, w.B, w.H, w.D)
         rc, plan = nat.plan_query(PO, PL, w.R, w.B, w.H, w.D, st, synth.DTYPES[w.in_dtype],
                                   synth.DTYPES[w.out_dtype], OUT, OUTL)
         assert rc == 0, name
-        got = (plan["path"], plan["lanes"], plan["rc"], plan["slices_per_row"], plan["block"],
-               plan["grid"])
+        got = (plan["path"], plan["lanes"], plan["rc"], plan["nv"], plan["slices_per_row"],
+               plan["block"], plan["grid"])
         assert got == expect[name], (name, got)
-        assert plan["vec"] == 8
+        assert plan["vec"] == 8 and plan["rc"] * plan["nv"] <= 16
         assert plan["groups"] == w.B * w.H * plan["slices_per_row"]
+        # every 16-byte column of a row is owned by exactly one lane slot
+        dv = w.D // 8
+        assert plan["slices_per_row"] * plan["lanes"] * plan["nv"] >= dv
+        assert (plan["slices_per_row"] - 1) * plan["lanes"] * plan["nv"] < dv
 
 
 def test_fallback_to_scalar_and_forced_paths():
@@ -126,15 +130,33 @@ def test_fallback_to_scalar_and_forced_paths():
     assert plan["grid"] == 64 * 64 * 32 // plan["block"] and plan["lanes"] == 32
 
 
-@pytest.mark.parametrize("R,want_rc,want_lanes", [(1, 4, 8), (3, 4, 8), (5, 8, 8), (9, 16, 16),
-                                                   (16, 16, 16), (33, 16, 16)])
-def test_rc_and_lanes_follow_R(R, want_rc, want_lanes):
-    rc, plan = q(R=R, D=64)      # 8 vectors per row
-    assert rc == 0 and plan["rc"] == want_rc and plan["lanes"] == want_lanes
+@pytest.mark.parametrize("R,want_rc,want_nv,want_lanes", [(1, 4, 2, 4), (3, 4, 2, 4), (5, 8, 1, 8),
+                                                           (9, 16, 1, 16), (16, 16, 1, 16),
+                                                           (33, 16, 1, 16)])
+def test_rc_nv_and_lanes_follow_R(R, want_rc, want_nv, want_lanes):
+    rc, plan = q(R=R, D=64, B=64, H=64)      # 8 vectors per row, beyond one CTA
+    assert rc == 0 and (plan["rc"], plan["nv"], plan["lanes"]) == (want_rc, want_nv, want_lanes)
 
 
-@pytest.mark.parametrize("D,lanes,slices", [(8, 4, 1), (24, 4, 1), (128, 16, 1), (256, 32, 1),
-                                             (264, 32, 2), (1024, 32, 4)])
-def test_lanes_and_slices_follow_D(D, lanes, slices):
+def test_latency_path_keeps_one_column_per_lane():
+    rc, plan = q(R=2, D=64, B=1, H=2)
+    assert plan["path"] == nat.PATH_LATENCY and plan["nv"] == 1 and plan["lanes"] == 8
+    assert plan["block"] == 32 and plan["grid"] == 1
+
+
+def test_stream_only_below_its_size_limit():
+    # 16 partials of 512 bf16 in 1100 batches x 16 heads = 288 MB of partials: one-shot VECTOR
+    big = q(R=16, B=1100, H=16, D=512, o=nat.F32, out=0x7fa000000000, outl=0x7fb000000000)[1]
+    assert big["path"] == nat.PATH_VECTOR and big["grid"] > 0
+    small = q(R=16, B=512, H=16, D=512, o=nat.F32)[1]
+    assert small["path"] == nat.PATH_STREAM and small["grid"] == 0
+    # R > 16 needs several batches of partials per slice: VECTOR
+    assert q(R=17, B=64, H=64)[1]["path"] == nat.PATH_VECTOR
+
+
+@pytest.mark.parametrize("D,lanes,nv,slices", [(8, 4, 1, 1), (24, 4, 1, 1), (128, 8, 2, 1),
+                                                (256, 16, 2, 1), (264, 32, 2, 1), (1024, 32, 2, 2),
+                                                (4096, 32, 2, 8)])
+def test_lanes_and_slices_follow_D(D, lanes, nv, slices):
     rc, plan = q(R=2, D=D, B=8, H=64)
-    assert rc == 0 and plan["lanes"] == lanes and plan["slices_per_row"] == slices
+    assert rc == 0 and (plan["lanes"], plan["nv"], plan["slices_per_row"]) == (lanes, nv, slices)
