@@ -562,7 +562,47 @@ def extra_workloads(device, l2: int, dist) -> dict:
         res[name] = row
         del sets
         torch.cuda.empty_cache()
-    return {"workloads": res}
+    return {"workloads": res, "state_update": time_state_update(device, l2, peak)}
+
+
+def time_state_update(device, l2: int, peak: float, B: int = 512, H: int = 16, D: int = 512) -> dict:
+    """In-place fold of one bf16 partial into an fp32 accumulator of B*H rows
+    (lse_merge_state_update), eager, inputs rotated past L2.  Algorithmic bytes
+    per call: B*H*(D*(4+2+4) + 12) (accumulator read and written, partial
+    read, three lse values).  lse_new starts equal to lse_acc, so the new
+    partial keeps a weight of about 1/k after k folds and is always read."""
+    import torch
+    from lse_weighted_merge_b200 import _native as nat
+    per = B * H * (D * 10 + 12)
+    nset = n_sets(per, l2)
+    gen = torch.Generator(device=device).manual_seed(2024)
+    accs = [torch.randn((B, H, D), generator=gen, device=device) for _ in range(nset)]
+    news = [torch.randn((B, H, D), generator=gen, device=device).to(torch.bfloat16) for _ in range(nset)]
+    las = [torch.rand((B, H), generator=gen, device=device) * 8 for _ in range(nset)]
+    lns = [la.clone() for la in las]
+    s = torch.cuda.current_stream(device).cuda_stream
+
+    def launch(i):
+        j = i % nset
+        nat.state_update_raw(accs[j].data_ptr(), las[j].data_ptr(), news[j].data_ptr(),
+                             lns[j].data_ptr(), B, H, D, None, nat.F32, nat.BF16, s)
+
+    for i in range(20):
+        launch(i)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n = 200
+    e0.record()
+    for i in range(n):
+        launch(i)
+    e1.record()
+    torch.cuda.synchronize(device)
+    us = e0.elapsed_time(e1) * 1e3 / n
+    gbs = per / (us * 1e-6) / 1e9
+    return {"shape": f"B={B} H={H} D={D}, fp32 accumulator, bf16 partial",
+            "eager_us_per_call": us, "gbs": gbs, "frac_of_measured_hbm": gbs / peak,
+            "bytes_per_call": per, "l2": f"rotating {nset} sets"}
 
 
 def main(argv=None):

@@ -88,7 +88,8 @@ typedef struct {
  *   out_dtype    element type of out_o (lse_merge_dtype)
  *   out_o        device pointer, dense [B,H,D] of out_dtype, written
  *   out_lse      device pointer, dense [B,H] fp32, written
- *   stream       CUDA stream the kernel is enqueued on
+ *   stream       CUDA stream the kernel is enqueued on; it and every pointer
+ *                belong to the calling thread's current CUDA device
  *
  * The caller owns every buffer.  Pointers must be aligned to their element
  * size; the fast path additionally wants 16-byte aligned partial_o rows and
@@ -135,6 +136,41 @@ int lse_merge_plan_query(const void* partial_o, const float* partial_lse,
                          int in_dtype, int out_dtype,
                          const void* out_o, const float* out_lse,
                          int path, lse_merge_plan* plan);
+
+/*
+ * Fold one new partial into an accumulator, in place (the merge above with
+ * R = 2 whose first partial is the accumulator; applied shard after shard it
+ * gives the R-way merge, because the log-sum-exp combine is associative).
+ * Per row (b, h):
+ *
+ *     m       = max(lse_acc, lse_new)
+ *     e_a     = exp(lse_acc - m),  e_n = exp(lse_new - m)    (0 for -inf)
+ *     o_acc   = (e_a * o_acc + e_n * o_new) / (e_a + e_n)
+ *     lse_acc = m + log(e_a + e_n)
+ *
+ * and 0, -inf when both sides are empty.  An empty side is never read, so an
+ * accumulator can start as lse_acc = -inf with o_acc uninitialised.  The pages
+ * describe the R-way merge only; this entry point is derived from it.
+ *
+ *   o_acc, lse_acc  device pointers, dense [B,H,D] of acc_dtype and [B,H] fp32;
+ *                   read and overwritten
+ *   o_new, lse_new  device pointers; element (b,h,d) of o_new at
+ *                   b*o_b + h*o_h + d, element (b,h) of lse_new at
+ *                   b*lse_b + h*lse_h (new_strides; NULL = dense [B,H,D], [B,H])
+ *   acc_dtype, new_dtype   lse_merge_dtype of o_acc and o_new
+ *   stream          as for lse_merge
+ *
+ * The new partial must not overlap the accumulator, nor o_acc lse_acc.
+ * Returns the codes of lse_merge (LSE_MERGE_EPATH does not occur).
+ */
+typedef struct {
+    int64_t o_b, o_h;
+    int64_t lse_b, lse_h;
+} lse_merge_state_strides;
+
+int lse_merge_state_update(void* o_acc, float* lse_acc, const void* o_new, const float* lse_new,
+                           int B, int H, int D, const lse_merge_state_strides* new_strides,
+                           int acc_dtype, int new_dtype, lse_merge_stream_t stream);
 
 /* A static, human-readable description of a return code. */
 const char* lse_merge_strerror(int code);

@@ -20,14 +20,19 @@ PATH_NAMES = {PATH_VECTOR: "vector", PATH_LATENCY: "latency", PATH_SCALAR: "scal
 OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH = 0, -1, -2, -3, -4, -5, -6, -7, -8
 
 # Every symbol include/lse_merge.h declares.
-EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merge_strerror",
-           "lse_merge_last_cuda_error", "lse_merge_version")
+EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merge_state_update",
+           "lse_merge_strerror", "lse_merge_last_cuda_error", "lse_merge_version")
 ABI_VERSION = 2
 
 
 class Strides(ctypes.Structure):
     _fields_ = [("o_r", ctypes.c_int64), ("o_b", ctypes.c_int64), ("o_h", ctypes.c_int64),
                 ("lse_r", ctypes.c_int64), ("lse_b", ctypes.c_int64), ("lse_h", ctypes.c_int64)]
+
+
+class StateStrides(ctypes.Structure):
+    _fields_ = [("o_b", ctypes.c_int64), ("o_h", ctypes.c_int64),
+                ("lse_b", ctypes.c_int64), ("lse_h", ctypes.c_int64)]
 
 
 class Plan(ctypes.Structure):
@@ -63,6 +68,9 @@ def _load() -> ctypes.CDLL:
     lib.lse_merge_plan_query.argtypes = [vp, vp, i, i, i, i, ctypes.POINTER(Strides), i, i, vp, vp,
                                          i, ctypes.POINTER(Plan)]
     lib.lse_merge_plan_query.restype = i
+    lib.lse_merge_state_update.argtypes = [vp, vp, vp, vp, i, i, i, ctypes.POINTER(StateStrides),
+                                           i, i, vp]
+    lib.lse_merge_state_update.restype = i
     lib.lse_merge_strerror.argtypes = [i]
     lib.lse_merge_strerror.restype = ctypes.c_char_p
     lib.lse_merge_last_cuda_error.argtypes = []
@@ -112,3 +120,18 @@ def plan_query(o_ptr: int, lse_ptr: int, R: int, B: int, H: int, D: int, strides
     rc = lib.lse_merge_plan_query(o_ptr, lse_ptr, R, B, H, D, _strides(strides), in_dtype,
                                   out_dtype, out_ptr, out_lse_ptr, path, ctypes.byref(plan))
     return rc, (plan.as_dict() if rc == OK else None)
+
+
+def state_update_raw(acc_ptr: int, lse_acc_ptr: int, new_ptr: int, lse_new_ptr: int, B: int,
+                     H: int, D: int, new_strides, acc_dtype: int, new_dtype: int,
+                     stream: int = 0, check: bool = True) -> int:
+    """Call lse_merge_state_update; ``new_strides`` = (o_b, o_h, lse_b, lse_h) or None."""
+    st = None if new_strides is None else ctypes.pointer(StateStrides(*[int(x) for x in new_strides]))
+    rc = lib.lse_merge_state_update(acc_ptr, lse_acc_ptr, new_ptr, lse_new_ptr, B, H, D, st,
+                                    acc_dtype, new_dtype, stream or None)
+    if check and rc != OK:
+        extra = ""
+        if rc == ELAUNCH:
+            extra = f" (cudaError {lib.lse_merge_last_cuda_error()})"
+        raise LseMergeError(rc, strerror(rc) + extra)
+    return rc

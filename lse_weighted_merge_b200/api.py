@@ -3,7 +3,7 @@ from __future__ import annotations
 
 from ._native import (BF16, F16, F32, PATH_AUTO, PATH_LATENCY, PATH_SCALAR, PATH_STREAM,
                       PATH_VECTOR,
-                      LseMergeError, merge_raw, plan_query, strerror)
+                      LseMergeError, merge_raw, plan_query, state_update_raw, strerror)
 
 
 def dtype_code(dtype) -> int:
@@ -64,10 +64,14 @@ def merge(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, out=N
         raise ValueError("out must be a contiguous [B, H, D] tensor of out_dtype")
     if tuple(out_lse.shape) != (B, H) or not out_lse.is_contiguous() or out_lse.dtype != torch.float32:
         raise ValueError("out_lse must be a contiguous float32 [B, H] tensor")
-    stream = torch.cuda.current_stream(dev).cuda_stream
-    merge_raw(partial_o.data_ptr(), partial_lse.data_ptr(), R, B, H, D, st,
-              dtype_code(partial_o.dtype), dtype_code(out_dtype), out.data_ptr(),
-              out_lse.data_ptr(), stream, path)
+    if partial_lse.device != dev or out.device != dev or out_lse.device != dev:
+        raise ValueError("all tensors must be on the same CUDA device")
+    # The library launches on the current device: make it the tensors' one.
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev).cuda_stream
+        merge_raw(partial_o.data_ptr(), partial_lse.data_ptr(), R, B, H, D, st,
+                  dtype_code(partial_o.dtype), dtype_code(out_dtype), out.data_ptr(),
+                  out_lse.data_ptr(), stream, path)
     return out, out_lse
 
 
@@ -183,3 +187,35 @@ def merge_host(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, 
     if sync:
         s_back.synchronize()
     return out, out_lse
+
+
+def merge_state_(o_acc, lse_acc, o_new, lse_new):
+    """Fold one new partial into an accumulator, in place, on the GPU.
+
+    o_acc [B, H, D] (contiguous; float32 / float16 / bfloat16) and lse_acc
+    [B, H] (contiguous float32) are read and overwritten with the merge of
+    themselves and (o_new [B, H, D], any strides with stride 1 along D;
+    lse_new [B, H] float32).  An accumulator with lse_acc = -inf is empty: its
+    o_acc is never read.  Returns (o_acc, lse_acc).
+    """
+    import torch
+    for t in (o_acc, lse_acc, o_new, lse_new):
+        if not t.is_cuda:
+            raise ValueError("merge_state_ runs on CUDA tensors only (there is no CPU path)")
+    if lse_acc.dtype != torch.float32 or lse_new.dtype != torch.float32:
+        raise TypeError("lse tensors must be float32")
+    if o_acc.dim() != 3 or not o_acc.is_contiguous() or not lse_acc.is_contiguous():
+        raise ValueError("o_acc must be a contiguous [B, H, D] tensor, lse_acc contiguous [B, H]")
+    B, H, D = o_acc.shape
+    if tuple(o_new.shape) != (B, H, D) or tuple(lse_acc.shape) != (B, H) or \
+            tuple(lse_new.shape) != (B, H) or o_new.stride(-1) != 1:
+        raise ValueError("shapes must be o [B, H, D] (stride 1 along D) and lse [B, H]")
+    dev = o_acc.device
+    if any(t.device != dev for t in (lse_acc, o_new, lse_new)):
+        raise ValueError("all tensors must be on the same CUDA device")
+    st = (o_new.stride(0), o_new.stride(1), lse_new.stride(0), lse_new.stride(1))
+    with torch.cuda.device(dev):
+        state_update_raw(o_acc.data_ptr(), lse_acc.data_ptr(), o_new.data_ptr(),
+                         lse_new.data_ptr(), B, H, D, st, dtype_code(o_acc.dtype),
+                         dtype_code(o_new.dtype), torch.cuda.current_stream(dev).cuda_stream)
+    return o_acc, lse_acc

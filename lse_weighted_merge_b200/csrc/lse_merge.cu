@@ -170,9 +170,9 @@ struct Elem<__nv_bfloat16> {
         x[2] = pack2u(v.z << 16, v.z & 0xffff0000u);
         x[3] = pack2u(v.w << 16, v.w & 0xffff0000u);
     }
+    __device__ static float widen(unsigned short u) { return __uint_as_float((uint32_t)u << 16); }
     __device__ static float load1(const char* p) {
-        const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
-        return __uint_as_float((uint32_t)u << 16);
+        return widen(__ldg(reinterpret_cast<const unsigned short*>(p)));
     }
     __device__ static void store1(char* p, float x) {
         *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x);
@@ -200,11 +200,9 @@ struct Elem<__half> {
 #pragma unroll
         for (int k = 0; k < 4; ++k) x[k] = pack2f(f[2 * k], f[2 * k + 1]);
     }
+    __device__ static float widen(unsigned short u) { return __half2float(__ushort_as_half(u)); }
     __device__ static float load1(const char* p) {
-        const unsigned short u = __ldg(reinterpret_cast<const unsigned short*>(p));
-        __half h;
-        memcpy(&h, &u, 2);
-        return __half2float(h);
+        return widen(__ldg(reinterpret_cast<const unsigned short*>(p)));
     }
     __device__ static void store1(char* p, float x) {
         *reinterpret_cast<__half*>(p) = __float2half_rn(x);
@@ -623,6 +621,126 @@ __global__ void __launch_bounds__(kBlock) merge_scalar_kernel(const KParams p) {
     if (live && j == 0) p.out_lse[row] = esum > 0.f ? m + logf(esum) : -INFINITY;
 }
 
+
+// ------------------------------------------------------------------ state update
+
+struct SParams {
+    char* acc;             // o_acc, dense [B,H,D]
+    float* lse_acc;        // dense [B,H]
+    const char* nw;        // o_new
+    const float* lse_new;
+    int64_t n_b, n_h;      // o_new strides in BYTES
+    int64_t l_b, l_h;      // lse_new strides in elements
+    int H, D, chunks;
+    int lanes, lg;
+    int64_t rows;
+};
+
+// 8 consecutive elements of type T at p as fp32; VEC: 16-byte accesses (p is
+// 16-byte aligned and all 8 elements exist), else element accesses for the
+// first `n`.  STREAM selects the read-only streaming load, only for data that
+// this kernel never writes.
+template <typename T, bool VEC, bool STREAM>
+__device__ __forceinline__ void load8(const char* p, int n, float* f) {
+    if constexpr (VEC) {
+#pragma unroll
+        for (int k = 0; k < (int)sizeof(T); k += 2) {   // 1 (16-bit) or 2 (fp32) vectors
+            const uint4 v = STREAM ? ld_stream16(p + k * 8) : *reinterpret_cast<const uint4*>(p + k * 8);
+            Elem<T>::unpack(v, f + k * 2);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            f[k] = 0.f;
+            if (k < n) {
+                if constexpr (STREAM) {
+                    f[k] = Elem<T>::load1(p + k * (int)sizeof(T));
+                } else if constexpr (sizeof(T) == 4) {
+                    f[k] = *reinterpret_cast<const float*>(p + k * 4);
+                } else {
+                    f[k] = Elem<T>::widen(*reinterpret_cast<const unsigned short*>(p + k * 2));
+                }
+            }
+        }
+    }
+}
+
+template <typename T, bool VEC>
+__device__ __forceinline__ void store8(char* p, int n, const float* f) {
+    if constexpr (VEC) {
+        store_vec<T, 8>(p, f);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (k < n) Elem<T>::store1(p + k * (int)sizeof(T), f[k]);
+    }
+}
+
+// A group of p.lanes lanes per row.  Lane 0 of the group reads both lse values
+// and hands them to the group by shuffle, so no lane reads lse_acc after lane
+// 0 has overwritten it; each element of o_acc is read and written by one lane.
+template <typename TA, typename TN, bool VEC>
+__global__ void __launch_bounds__(kBlock) state_update_kernel(const SParams p) {
+    pdl_wait();
+    pdl_release();
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = t >> p.lg;
+    const int j = (int)(t & (p.lanes - 1));
+    const bool live = row < p.rows;
+    const int64_t r = live ? row : 0;
+    const int64_t b = r / p.H, h = r - b * p.H;
+    float la = -INFINITY, ln = -INFINITY;
+    if (live && j == 0) {
+        la = p.lse_acc[r];
+        ln = __ldg(p.lse_new + b * p.l_b + h * p.l_h);
+    }
+    la = __shfl_sync(kFull, la, 0, p.lanes);
+    ln = __shfl_sync(kFull, ln, 0, p.lanes);
+    const float m = fmaxf(la, ln);
+    const float mref = (m == -INFINITY) ? 0.f : m;
+    const float ea = expf(la - mref), en = expf(ln - mref);   // 0 for an empty side
+    const float esum = ea + en;
+    const float inv = esum > 0.f ? 1.f / esum : 0.f;
+    if (!live) return;
+    char* arow = p.acc + r * p.D * (int64_t)sizeof(TA);
+    const char* nrow = p.nw + b * p.n_b + h * p.n_h;
+    for (int c = j; c < p.chunks; c += p.lanes) {
+        const int d0 = c * 8;
+        const int n = min(8, p.D - d0);
+        float fa[8], fn[8], o[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) fa[k] = fn[k] = 0.f;
+        if (ea != 0.f) load8<TA, VEC, false>(arow + (int64_t)d0 * sizeof(TA), n, fa);
+        if (en != 0.f) load8<TN, VEC, true>(nrow + (int64_t)d0 * sizeof(TN), n, fn);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[k] = fmaf(ea, fa[k], en * fn[k]) * inv;
+        store8<TA, VEC>(arow + (int64_t)d0 * sizeof(TA), n, o);
+    }
+    if (j == 0) p.lse_acc[r] = esum > 0.f ? m + logf(esum) : -INFINITY;
+}
+
+using StateFn = void (*)(SParams);
+
+template <typename TA, typename TN>
+StateFn pick_state_v(bool vec) {
+    return vec ? state_update_kernel<TA, TN, true> : state_update_kernel<TA, TN, false>;
+}
+template <typename TA>
+StateFn pick_state_n(int new_dtype, bool vec) {
+    switch (new_dtype) {
+        case LSE_MERGE_F32: return pick_state_v<TA, float>(vec);
+        case LSE_MERGE_F16: return pick_state_v<TA, __half>(vec);
+        default: return pick_state_v<TA, __nv_bfloat16>(vec);
+    }
+}
+StateFn pick_state(int acc_dtype, int new_dtype, bool vec) {
+    switch (acc_dtype) {
+        case LSE_MERGE_F32: return pick_state_n<float>(new_dtype, vec);
+        case LSE_MERGE_F16: return pick_state_n<__half>(new_dtype, vec);
+        default: return pick_state_n<__nv_bfloat16>(new_dtype, vec);
+    }
+}
+
 // ------------------------------------------------------------------------ dispatch
 
 using KernelFn = void (*)(KParams);
@@ -804,6 +922,57 @@ int run(const void* partial_o, const float* partial_lse, int R, int B, int H, in
     return LSE_MERGE_OK;
 }
 
+int run_state(void* o_acc, float* lse_acc, const void* o_new, const float* lse_new, int B,
+              int H, int D, const lse_merge_state_strides* strides, int acc_dtype, int new_dtype,
+              cudaStream_t stream) {
+    if (B < 1 || H < 1 || D < 1) return LSE_MERGE_EDIMS;
+    lse_merge_state_strides st;
+    if (strides) {
+        st = *strides;
+    } else {
+        st.o_b = (int64_t)H * D;
+        st.o_h = D;
+        st.lse_b = H;
+        st.lse_h = 1;
+    }
+    StatePlan pl;
+    const int rc = make_state_plan(o_acc, lse_acc, o_new, lse_new, B, H, D, st, acc_dtype,
+                                   new_dtype, &pl);
+    if (rc != LSE_MERGE_OK) return rc;
+    const int nb = elem_bytes(new_dtype);
+    SParams sp;
+    sp.acc = static_cast<char*>(o_acc);
+    sp.lse_acc = lse_acc;
+    sp.nw = static_cast<const char*>(o_new);
+    sp.lse_new = lse_new;
+    sp.n_b = st.o_b * nb;
+    sp.n_h = st.o_h * nb;
+    sp.l_b = st.lse_b;
+    sp.l_h = st.lse_h;
+    sp.H = H;
+    sp.D = D;
+    sp.chunks = pl.chunks;
+    sp.lanes = pl.lanes;
+    sp.lg = log2i(pl.lanes);
+    sp.rows = (int64_t)B * H;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pl.grid);
+    cfg.blockDim = dim3((unsigned)pl.block);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = kPdl ? attr : nullptr;
+    cfg.numAttrs = kPdl ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, pick_state(acc_dtype, new_dtype, pl.vec != 0), sp);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = (int)e;
+        (void)cudaGetLastError();
+        return LSE_MERGE_ELAUNCH;
+    }
+    return LSE_MERGE_OK;
+}
+
 }  // namespace
 }  // namespace lsem
 
@@ -821,6 +990,13 @@ int lse_merge_with_path(const void* partial_o, const float* partial_lse, int R, 
                         void* out_o, float* out_lse, lse_merge_stream_t stream, int path) {
     return lsem::run(partial_o, partial_lse, R, B, H, D, strides, in_dtype, out_dtype, out_o,
                      out_lse, reinterpret_cast<cudaStream_t>(stream), path);
+}
+
+int lse_merge_state_update(void* o_acc, float* lse_acc, const void* o_new, const float* lse_new,
+                           int B, int H, int D, const lse_merge_state_strides* new_strides,
+                           int acc_dtype, int new_dtype, lse_merge_stream_t stream) {
+    return lsem::run_state(o_acc, lse_acc, o_new, lse_new, B, H, D, new_strides, acc_dtype,
+                           new_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int lse_merge_last_cuda_error(void) { return lsem::g_last_cuda_error; }

@@ -172,6 +172,42 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
     return LSE_MERGE_OK;
 }
 
+int make_state_plan(const void* o_acc, const float* lse_acc, const void* o_new,
+                    const float* lse_new, int B, int H, int D, const lse_merge_state_strides& st,
+                    int acc_dtype, int new_dtype, StatePlan* plan) {
+    const int ab = elem_bytes(acc_dtype), nb = elem_bytes(new_dtype);
+    if (ab == 0 || nb == 0) return LSE_MERGE_EDTYPE;
+    if (B < 1 || H < 1 || D < 1) return LSE_MERGE_EDIMS;
+    if (!o_acc || !lse_acc || !o_new || !lse_new || !plan) return LSE_MERGE_ENULL;
+    if (st.o_b < 0 || st.o_h < 0 || st.lse_b < 0 || st.lse_h < 0) return LSE_MERGE_ESTRIDE;
+    if (!aligned(o_acc, ab) || !aligned(o_new, nb) || !aligned(lse_acc, 4) || !aligned(lse_new, 4))
+        return LSE_MERGE_EALIGN;
+    const i128 rows = (i128)B * H;
+    const i128 lim = (i128)1 << 62;
+    const i128 acc_bytes = rows * D * ab, lacc_bytes = rows * 4;
+    const i128 new_bytes = ((i128)(B - 1) * st.o_b + (i128)(H - 1) * st.o_h + D) * nb;
+    const i128 lnew_bytes = ((i128)(B - 1) * st.lse_b + (i128)(H - 1) * st.lse_h + 1) * 4;
+    if (acc_bytes > lim || new_bytes > lim || lnew_bytes > lim) return LSE_MERGE_EDIMS;
+    const Span sa{(uintptr_t)o_acc, (i128)(uintptr_t)o_acc + acc_bytes};
+    const Span sla{(uintptr_t)lse_acc, (i128)(uintptr_t)lse_acc + lacc_bytes};
+    const Span sn{(uintptr_t)o_new, (i128)(uintptr_t)o_new + new_bytes};
+    const Span sln{(uintptr_t)lse_new, (i128)(uintptr_t)lse_new + lnew_bytes};
+    if (overlap(sa, sla) || overlap(sa, sn) || overlap(sa, sln) || overlap(sla, sn) ||
+        overlap(sla, sln))
+        return LSE_MERGE_EALIAS;
+    StatePlan p{};
+    p.vec = (D % 8) == 0 && aligned(o_acc, 16) && aligned(o_new, 16) && ((st.o_b * nb) % 16) == 0 &&
+            ((st.o_h * nb) % 16) == 0;
+    p.chunks = (D + 7) / 8;
+    p.lanes = next_pow2(p.chunks < 32 ? p.chunks : 32);
+    p.block = kBlock;
+    const i128 grid = (rows * p.lanes + kBlock - 1) / kBlock;
+    if (grid > 0x7fffffff) return LSE_MERGE_EDIMS;
+    p.grid = (int64_t)grid;
+    *plan = p;
+    return LSE_MERGE_OK;
+}
+
 }  // namespace lsem
 
 extern "C" {

@@ -67,4 +67,19 @@ int make_plan(const void* partial_o, const float* partial_lse, int R, int B, int
 // Dense [B,H,R,D] / [B,H,R] strides, used when the caller passes NULL.
 lse_merge_strides default_strides(int R, int B, int H, int D);
 
+// Launch geometry of the in-place state update: a group of `lanes` lanes per
+// row, lane j folding the 8-element chunks j, j + lanes, ... of the row.
+struct StatePlan {
+    int vec;        // 1: 16-byte loads and stores; 0: element accesses
+    int lanes;      // power of two <= 32
+    int chunks;     // 8-element chunks per row, ceil(D / 8)
+    int block;
+    int64_t grid;
+};
+
+// Validate the arguments of lse_merge_state_update and fill *plan.
+int make_state_plan(const void* o_acc, const float* lse_acc, const void* o_new,
+                    const float* lse_new, int B, int H, int D, const lse_merge_state_strides& st,
+                    int acc_dtype, int new_dtype, StatePlan* plan);
+
 }  // namespace lsem

@@ -50,6 +50,11 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
         dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
         ctypes.c_int, dp, dp]
     lib.oracle_mutant.restype = ctypes.c_int
+    lib.oracle_state_update.restype = ctypes.c_int
+    lib.oracle_state_update.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_int64, ctypes.c_int64, dp, dp]
     return lib
 
 
@@ -117,3 +122,31 @@ def attention_shard(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
                                v.ctypes.data_as(dp), L, D, float(scale), begin, end,
                                o.ctypes.data_as(dp), lse.ctypes.data_as(dp))
     return o, float(lse[0])
+
+
+def state_update(acc: np.ndarray, lse_acc: np.ndarray, acc_dtype: int, new: np.ndarray,
+                 lse_new: np.ndarray, new_dtype: int, B: int, H: int, D: int,
+                 new_strides=None, lse_new_strides=None, lib: ctypes.CDLL | None = None):
+    """Fold ``new`` into the accumulator ``acc`` (fp64 result, nothing modified).
+
+    acc: flat dense [B, H, D] storage (uint16 bits or float32); lse_acc: [B, H]
+    float32; new: flat storage with (b, h) element strides ``new_strides``
+    (default dense [B, H, D]); lse_new with ``lse_new_strides`` (default
+    dense [B, H]).  Returns (out [B, H, D] float64, out_lse [B, H] float64).
+    """
+    lib = lib or load()
+    nb, nh = new_strides or (H * D, D)
+    lb, lh = lse_new_strides or (H, 1)
+    a = np.ascontiguousarray(acc)
+    n = np.ascontiguousarray(new)
+    la = np.ascontiguousarray(lse_acc, dtype=np.float32)
+    ln = np.ascontiguousarray(lse_new, dtype=np.float32)
+    out = np.empty((B, H, D), dtype=np.float64)
+    out_lse = np.empty((B, H), dtype=np.float64)
+    dp = ctypes.POINTER(ctypes.c_double)
+    rc = lib.oracle_state_update(a.ctypes.data, la.ctypes.data, acc_dtype, n.ctypes.data,
+                                 ln.ctypes.data, new_dtype, B, H, D, nb, nh, lb, lh,
+                                 out.ctypes.data_as(dp), out_lse.ctypes.data_as(dp))
+    if rc != 0:
+        raise ValueError(f"oracle_state_update returned {rc}")
+    return out, out_lse

@@ -227,3 +227,56 @@ void oracle_attention_shard(const double* q, const double* k, const double* v,
     for (int d = 0; d < D; ++d) o[d] /= z;
     *lse = mx + log(z);
 }
+
+/*
+ * Fold one new partial into an accumulator: the merge above with R = 2, the
+ * first partial being the accumulator (the combine the page's merge is built
+ * from; applying it shard by shard gives the R-way merge, by associativity of
+ * the log-sum-exp combine).  Per row (b, h):
+ *     m   = max(lse_acc, lse_new)
+ *     e_a = exp(lse_acc - m), e_n = exp(lse_new - m)   (0 for an lse of -inf)
+ *     out = (e_a * acc + e_n * new) / (e_a + e_n),  out_lse = m + log(e_a + e_n)
+ * and 0, -inf when both are empty.  acc is dense [B, H, D] of acc_dtype with
+ * lse_acc dense [B, H]; new has element strides nb, nh (d stride 1) and lse_new
+ * strides lb, lh.  Results in fp64: out [B, H, D], out_lse [B, H].
+ */
+int oracle_state_update(const void* acc, const float* lse_acc, int acc_dtype,
+                        const void* nw, const float* lse_new, int new_dtype,
+                        int B, int H, int D, int64_t nb, int64_t nh, int64_t lb, int64_t lh,
+                        double* out, double* out_lse) {
+    if ((acc_dtype != ORACLE_F32 && acc_dtype != ORACLE_F16 && acc_dtype != ORACLE_BF16) ||
+        (new_dtype != ORACLE_F32 && new_dtype != ORACLE_F16 && new_dtype != ORACLE_BF16))
+        return -1;
+    if (B < 1 || H < 1 || D < 1) return -2;
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            const int64_t row = (int64_t)b * H + h;
+            const double la = (double)lse_acc[row];
+            const double ln = (double)lse_new[(int64_t)b * lb + (int64_t)h * lh];
+            double* o = out + row * D;
+            const double m = la > ln ? la : ln;
+            if (m == -INFINITY) {
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                out_lse[row] = -INFINITY;
+                continue;
+            }
+#if ORACLE_MUTANT == 7
+            /* planted mistake: the two weights swapped */
+            const double en = (la == -INFINITY) ? 0.0 : exp(la - m);
+            const double ea = (ln == -INFINITY) ? 0.0 : exp(ln - m);
+#else
+            const double ea = (la == -INFINITY) ? 0.0 : exp(la - m);
+            const double en = (ln == -INFINITY) ? 0.0 : exp(ln - m);
+#endif
+            const double denom = ea + en;
+            for (int d = 0; d < D; ++d) {
+                double s = 0.0;
+                if (ea != 0.0) s += ea * load_elem(acc, row * D + d, acc_dtype);
+                if (en != 0.0) s += en * load_elem(nw, (int64_t)b * nb + (int64_t)h * nh + d, new_dtype);
+                o[d] = s / denom;
+            }
+            out_lse[row] = m + log(denom);
+        }
+    }
+    return 0;
+}

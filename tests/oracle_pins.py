@@ -26,6 +26,8 @@ from lse_weighted_merge_b200 import synth
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
                       "merge_hand_cases.json")
+GOLDEN_STATE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                            "state_update_hand_cases.json")
 
 
 def _num(x):
@@ -299,9 +301,64 @@ def pin_extreme_spread(lib):
     assert out_lse[0, 0] == 500.0 and out_lse[0, 1] == 30.0
 
 
+def pin_state_golden(lib):
+    """Hand-derived folds of one partial into an accumulator."""
+    with open(GOLDEN_STATE) as fh:
+        cases = json.load(fh)["cases"]
+    for c in cases:
+        D = c["D"]
+        acc = synth.pack(np.array([_num(x) for x in c["acc"]], np.float32), c["acc_dtype"])
+        new = synth.pack(np.array([_num(x) for x in c["new"]], np.float32), c["new_dtype"])
+        la = np.array([_num(c["lse_acc"])], np.float32)
+        ln = np.array([_num(c["lse_new"])], np.float32)
+        out, out_lse = oracle.state_update(acc, la, synth.DTYPES[c["acc_dtype"]], new, ln,
+                                           synth.DTYPES[c["new_dtype"]], 1, 1, D, lib=lib)
+        want = np.array([_num(x) for x in c["out"]])
+        assert not np.isnan(out).any(), c["name"]
+        assert np.all(np.abs(out[0, 0] - want) <= c["tol"]), (c["name"], out, want)
+        wl = _num(c["out_lse"])
+        if wl == -math.inf:
+            assert out_lse[0, 0] == -math.inf, c["name"]
+        else:
+            assert abs(out_lse[0, 0] - wl) <= c["tol"], (c["name"], out_lse, wl)
+
+
+def pin_state_chain_is_the_merge(lib):
+    """Folding R shards one by one into an empty accumulator (fp32 in between)
+    gives the R-way merge, by associativity of the combine; and one fold of
+    same-dtype partials is the R = 2 merge exactly."""
+    rng = np.random.Generator(np.random.PCG64(21))
+    R, B, H, D = 6, 2, 3, 10
+    o = rng.standard_normal((R, B, H, D)).astype(np.float32)
+    lse = rng.uniform(-8, 8, (R, B, H)).astype(np.float32)
+    lse[2, 1, 1] = -np.inf
+    full, full_lse = run(lib, o, lse)
+    acc = np.full((B, H, D), np.nan, np.float32)
+    la = np.full((B, H), -np.inf, np.float32)
+    for r in range(R):
+        out, ol = oracle.state_update(acc.ravel(), la, oracle.F32, o[r].ravel(), lse[r], oracle.F32,
+                                      B, H, D, lib=lib)
+        acc, la = out.astype(np.float32), ol.astype(np.float32)
+    assert np.allclose(acc, full, rtol=0, atol=2e-6)
+    assert np.allclose(la, full_lse, rtol=0, atol=2e-6)
+    two, two_lse = run(lib, o[:2], lse[:2])
+    one, one_lse = oracle.state_update(o[0].ravel(), lse[0], oracle.F32, o[1].ravel(), lse[1],
+                                       oracle.F32, B, H, D, lib=lib)
+    assert np.array_equal(one, two) and np.array_equal(one_lse, two_lse)
+    # strided new operand: the same data laid out with padded rows
+    padded = np.zeros((B, H, D + 5), np.float32)
+    padded[..., :D] = o[1]
+    lhm = np.ascontiguousarray(lse[1].T)     # [H, B]
+    alt, alt_lse = oracle.state_update(o[0].ravel(), lse[0], oracle.F32, padded.ravel(), lhm.ravel(),
+                                       oracle.F32, B, H, D, new_strides=(H * (D + 5), D + 5),
+                                       lse_new_strides=(1, B), lib=lib)
+    assert np.array_equal(alt, one) and np.array_equal(alt_lse, one_lse)
+
+
 ALL_PINS = [
     pin_decoders, pin_golden, pin_r1_identity, pin_equal_lse_mean,
     pin_empty_shards_drop_out, pin_shift_invariance, pin_permutation_invariance,
     pin_associativity, pin_attention_shard, pin_split_attention_identity,
-    pin_layout_and_row_independence, pin_extreme_spread,
+    pin_layout_and_row_independence, pin_extreme_spread, pin_state_golden,
+    pin_state_chain_is_the_merge,
 ]

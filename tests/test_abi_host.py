@@ -160,3 +160,23 @@ def test_stream_only_below_its_size_limit():
 def test_lanes_and_slices_follow_D(D, lanes, nv, slices):
     rc, plan = q(R=2, D=D, B=8, H=64)
     assert rc == 0 and (plan["lanes"], plan["nv"], plan["slices_per_row"]) == (lanes, nv, slices)
+
+
+
+def sq(B=2, H=3, D=64, st=None, a=nat.BF16, n=nat.BF16, acc=OUT, lacc=OUTL, new=PO, lnew=PL):
+    return nat.state_update_raw(acc, lacc, new, lnew, B, H, D, st, a, n, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(a=5), nat.EDTYPE), (dict(n=-1), nat.EDTYPE),
+    (dict(B=0), nat.EDIMS), (dict(D=0), nat.EDIMS),
+    (dict(acc=0), nat.ENULL), (dict(lacc=0), nat.ENULL), (dict(new=0), nat.ENULL), (dict(lnew=0), nat.ENULL),
+    (dict(st=(-64, 64, 3, 1)), nat.ESTRIDE), (dict(st=(192, 64, 3, -1)), nat.ESTRIDE),
+    (dict(acc=OUT + 1), nat.EALIGN), (dict(lacc=OUTL + 2), nat.EALIGN), (dict(a=nat.F32, acc=OUT + 2), nat.EALIGN),
+    (dict(new=OUT + 64), nat.EALIAS), (dict(lacc=OUT + 4), nat.EALIAS), (dict(lnew=OUTL), nat.EALIAS),
+    (dict(lnew=OUT), nat.EALIAS),
+    (dict(B=2 ** 30, H=2 ** 30, D=2 ** 30), nat.EDIMS),
+])
+def test_state_update_validation(kw, code):
+    # rejected before any CUDA call
+    assert sq(**kw) == code, (kw, nat.strerror(code))

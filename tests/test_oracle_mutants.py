@@ -20,6 +20,7 @@ MUTANTS = {
     4: "empty shards not skipped (0 * NaN leaks)",
     5: "plain mean instead of lse weights",
     6: "first shard dropped",
+    7: "state update with its two weights swapped",
 }
 
 CHILD = r"""
