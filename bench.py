@@ -15,9 +15,11 @@ R*B*H*(D*2+4) + B*H*(D*4+4).  Rank 0 prints one JSON line.
   e2e       the same metric through the public host-buffer call merge_host:
             each step copies its partials from pinned host memory to the GPU
             and the result back, in 8 batch slices overlapped with the merge.
-  roofline  the kernel's achieved GB/s against the measured HBM copy peak.
-  latency   eager and CUDA-graph-replayed us/call of the two tiny decode
-            shapes; per-workload GB/s of the other shapes.
+  roofline  the kernel's achieved GB/s against the measured HBM copy peak,
+            and its DRAM traffic from the committed ncu summary.
+  workloads eager us/call, GB/s and fraction of peak of every workload; the
+            two tiny decode shapes also CUDA-graph-replayed us/call.
+  state_update  the in-place fold of one partial into an accumulator.
   cpu_baseline  the fp64 CPU oracle on a bounded sample (rank 0, N = 1).
 
 With --gpus N under torchrun every rank merges its own batch (the rows are
