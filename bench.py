@@ -66,6 +66,8 @@ def parse_args(argv=None):
     p.add_argument("--no-extra", action="store_true", help="skip latency / per-workload lines")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--decode-only", default=None, metavar="SHAPE",
+                   help="only time the decode-attention shape SHAPE (for profiling)")
     return p.parse_args(argv)
 
 
@@ -564,7 +566,72 @@ def extra_workloads(device, l2: int, dist) -> dict:
         res[name] = row
         del sets
         torch.cuda.empty_cache()
-    return {"workloads": res, "state_update": time_state_update(device, l2, peak)}
+    return {"workloads": res, "state_update": time_state_update(device, l2, peak),
+            "decode_attention": time_decode_attention(device, peak)}
+
+
+DECODE_SHAPES = (  # name, B, Hq, Hkv, L, D, R
+    ("b64_hq32_hkv8_l4096_d128_r4", 64, 32, 8, 4096, 128, 4),
+    ("b8_hq8_hkv8_l32768_d128_r8", 8, 8, 8, 32768, 128, 8),
+)
+
+
+def time_decode_attention(device, peak: float, only: str | None = None) -> dict:
+    """Split-KV decode attention producing and merging the partials: fused
+    (one cluster kernel, the merge in distributed shared memory) against
+    unfused (the partials kernel, then lse_merge).  Algorithmic bytes per call:
+    K and V once (B*Hkv*L*D*2*2), q and the output once; the caches exceed L2,
+    so no rotation is needed."""
+    import torch
+    from lse_weighted_merge_b200 import _native as nat
+    res = {}
+    for name, B, Hq, Hkv, L, D, R in DECODE_SHAPES:
+        if only is not None and name != only:
+            continue
+        gen = torch.Generator(device=device).manual_seed(7)
+        q = torch.randn((B, Hq, D), generator=gen, device=device).to(torch.bfloat16)
+        k = torch.randn((B, Hkv, L, D), generator=gen, device=device).to(torch.bfloat16)
+        v = torch.randn((B, Hkv, L, D), generator=gen, device=device).to(torch.bfloat16)
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=device)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
+        po = torch.empty((B, Hq, R, D), dtype=torch.float32, device=device)
+        pl = torch.empty((B, Hq, R), dtype=torch.float32, device=device)
+        s = torch.cuda.current_stream(device).cuda_stream
+        scale = 1.0 / math.sqrt(D)
+        byts = B * Hkv * L * D * 2 * 2 + B * Hq * D * 2 * 2 + B * Hq * 4
+
+        def fused():
+            nat.decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), 0, B, Hq, Hkv, L, D, R,
+                           scale, None, nat.BF16, out.data_ptr(), lse.data_ptr(), s, fused=True,
+                           out_dtype=nat.BF16)
+
+        def unfused():
+            nat.decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), 0, B, Hq, Hkv, L, D, R,
+                           scale, None, nat.BF16, po.data_ptr(), pl.data_ptr(), s, fused=False)
+            nat.merge_raw(po.data_ptr(), pl.data_ptr(), R, B, Hq, D, None, nat.F32, nat.BF16,
+                          out.data_ptr(), lse.data_ptr(), s)
+
+        row = {"shape": f"B={B} Hq={Hq} Hkv={Hkv} L={L} D={D} splits={R}, bf16",
+               "bytes_per_call": byts}
+        for tag, fn, n in (("fused", fused, 50), ("unfused", unfused, 50)):
+            for _ in range(5):
+                fn()
+            torch.cuda.synchronize(device)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                fn()
+            e1.record()
+            torch.cuda.synchronize(device)
+            us = e0.elapsed_time(e1) * 1e3 / n
+            row[tag] = {"us_per_call": us, "gbs": byts / (us * 1e-6) / 1e9,
+                        "frac_of_measured_hbm": byts / (us * 1e-6) / 1e9 / peak,
+                        "launches_per_call": 1 if tag == "fused" else 2}
+        res[name] = row
+        del q, k, v
+        torch.cuda.empty_cache()
+    return res
 
 
 def time_state_update(device, l2: int, peak: float, B: int = 512, H: int = 16, D: int = 512) -> dict:
@@ -611,6 +678,12 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.decode_only:
+        import torch
+        device = torch.device("cuda", 0)
+        peak, _ = hbm_peak()
+        print(json.dumps({"decode_attention": time_decode_attention(device, peak, args.decode_only)}))
+        return 0
     return run_ours(args)
 
 

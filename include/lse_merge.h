@@ -67,6 +67,7 @@ typedef struct {
 #define LSE_MERGE_ELAUNCH (-6)  /* the CUDA launch failed (see lse_merge_last_cuda_error) */
 #define LSE_MERGE_EALIGN (-7)   /* a pointer not aligned to its element size */
 #define LSE_MERGE_EPATH (-8)    /* the requested path cannot take these arguments */
+#define LSE_MERGE_EUNSUP (-9)   /* a shape the decode-attention kernels do not implement */
 
 /* Kernel paths.  AUTO picks one from the sizes, dtypes and alignment. */
 #define LSE_MERGE_PATH_AUTO 0
@@ -171,6 +172,57 @@ typedef struct {
 int lse_merge_state_update(void* o_acc, float* lse_acc, const void* o_new, const float* lse_new,
                            int B, int H, int D, const lse_merge_state_strides* new_strides,
                            int acc_dtype, int new_dtype, lse_merge_stream_t stream);
+
+/*
+ * Split-KV decode attention, the producer of the partials (the CP-decode
+ * page's introduction: each rank attends over its own KV shard and returns
+ * o_r and lse_r).  One query token per sequence, grouped heads: query head h
+ * attends over KV head h / (Hq / Hkv).  The keys [0, len_b) of sequence b
+ * (len_b = kv_len[b] clamped to [0, L], or L when kv_len is NULL) are cut into
+ * R splits of ceil(len_b / R) keys; split r is the shard [r*ceil, min(len_b,
+ * (r+1)*ceil)).  For a split with keys j:
+ *
+ *     s_j = scale * <q, k_j>,  lse_r = log sum_j exp(s_j),
+ *     o_r = sum_j exp(s_j - lse_r) * v_j        (empty split: 0 and -inf)
+ *
+ *   q        [B, Hq, D]: element (b,h,d) at b*q_b + h*q_h + d
+ *   k, v     [B, Hkv, L, D]: element (b,h,l,d) at b*k_b + h*k_h + l*k_l + d
+ *            (v likewise with v_*); strides in elements, d stride 1; NULL
+ *            strides = dense
+ *   dtype    LSE_MERGE_BF16 or LSE_MERGE_F16 (q, k and v)
+ *   D        64 or 128; Hq a multiple of Hkv with Hq / Hkv <= 16
+ *   q, k, v  16-byte aligned, with strides of whole 16-byte multiples
+ *
+ * lse_merge_decode_partials writes the R partials, fp32, into caller buffers
+ * dense [B, Hq, R, D] and [B, Hq, R] (the layout lse_merge takes as its
+ * default), for a separate merge.
+ *
+ * lse_merge_decode_attention also merges them, inside the same kernel: the
+ * R CTAs of one (b, KV head) form a thread-block cluster, each holds its
+ * split's partial in shared memory, and after a cluster barrier every CTA
+ * merges a slice of D from all R partials through distributed shared memory,
+ * so the partials never reach HBM.  R must be 1, 2, 4 or 8.  Output out_o
+ * dense [B, Hq, D] of out_dtype and out_lse dense [B, Hq] fp32: attention over
+ * keys [0, len_b).
+ *
+ * Both return the codes of lse_merge, and LSE_MERGE_EUNSUP for a D, group
+ * size, dtype or R outside the above.
+ */
+typedef struct {
+    int64_t q_b, q_h;
+    int64_t k_b, k_h, k_l;
+    int64_t v_b, v_h, v_l;
+} lse_merge_attn_strides;
+
+int lse_merge_decode_partials(const void* q, const void* k, const void* v, const int32_t* kv_len,
+                              int B, int Hq, int Hkv, int L, int D, int R, float scale,
+                              const lse_merge_attn_strides* strides, int dtype,
+                              float* partial_o, float* partial_lse, lse_merge_stream_t stream);
+
+int lse_merge_decode_attention(const void* q, const void* k, const void* v, const int32_t* kv_len,
+                               int B, int Hq, int Hkv, int L, int D, int R, float scale,
+                               const lse_merge_attn_strides* strides, int dtype, int out_dtype,
+                               void* out_o, float* out_lse, lse_merge_stream_t stream);
 
 /* A static, human-readable description of a return code. */
 const char* lse_merge_strerror(int code);

@@ -16,7 +16,7 @@ from __future__ import annotations
 # these names without liblse_merge.so raises ImportError: there is no
 # fallback.
 _API = ("merge", "merge_state_", "merge_host", "release_host_workspace", "merge_raw",
-        "state_update_raw", "plan_query", "strerror", "LseMergeError", "dtype_code",
+        "state_update_raw", "decode_attention", "decode_raw", "plan_query", "strerror", "LseMergeError", "dtype_code",
         "F32", "F16", "BF16", "PATH_AUTO", "PATH_VECTOR", "PATH_LATENCY", "PATH_SCALAR",
         "PATH_STREAM")
 __all__ = list(_API)

@@ -17,11 +17,13 @@ PATH_AUTO, PATH_VECTOR, PATH_LATENCY, PATH_SCALAR, PATH_STREAM = 0, 1, 2, 3, 4
 PATH_NAMES = {PATH_VECTOR: "vector", PATH_LATENCY: "latency", PATH_SCALAR: "scalar",
               PATH_STREAM: "stream"}
 
-OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH = 0, -1, -2, -3, -4, -5, -6, -7, -8
+OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH, EUNSUP = (
+    0, -1, -2, -3, -4, -5, -6, -7, -8, -9)
 
 # Every symbol include/lse_merge.h declares.
 EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merge_state_update",
-           "lse_merge_strerror", "lse_merge_last_cuda_error", "lse_merge_version")
+           "lse_merge_decode_partials", "lse_merge_decode_attention", "lse_merge_strerror",
+           "lse_merge_last_cuda_error", "lse_merge_version")
 ABI_VERSION = 2
 
 
@@ -33,6 +35,10 @@ class Strides(ctypes.Structure):
 class StateStrides(ctypes.Structure):
     _fields_ = [("o_b", ctypes.c_int64), ("o_h", ctypes.c_int64),
                 ("lse_b", ctypes.c_int64), ("lse_h", ctypes.c_int64)]
+
+
+class AttnStrides(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("q_b", "q_h", "k_b", "k_h", "k_l", "v_b", "v_h", "v_l")]
 
 
 class Plan(ctypes.Structure):
@@ -71,6 +77,11 @@ def _load() -> ctypes.CDLL:
     lib.lse_merge_state_update.argtypes = [vp, vp, vp, vp, i, i, i, ctypes.POINTER(StateStrides),
                                            i, i, vp]
     lib.lse_merge_state_update.restype = i
+    attn = [vp, vp, vp, vp, i, i, i, i, i, i, ctypes.c_float, ctypes.POINTER(AttnStrides), i]
+    lib.lse_merge_decode_partials.argtypes = attn + [vp, vp, vp]
+    lib.lse_merge_decode_partials.restype = i
+    lib.lse_merge_decode_attention.argtypes = attn + [i, vp, vp, vp]
+    lib.lse_merge_decode_attention.restype = i
     lib.lse_merge_strerror.argtypes = [i]
     lib.lse_merge_strerror.restype = ctypes.c_char_p
     lib.lse_merge_last_cuda_error.argtypes = []
@@ -135,3 +146,28 @@ def state_update_raw(acc_ptr: int, lse_acc_ptr: int, new_ptr: int, lse_new_ptr: 
             extra = f" (cudaError {lib.lse_merge_last_cuda_error()})"
         raise LseMergeError(rc, strerror(rc) + extra)
     return rc
+
+
+def _check(rc: int, check: bool) -> int:
+    if check and rc != OK:
+        extra = ""
+        if rc == ELAUNCH:
+            extra = f" (cudaError {lib.lse_merge_last_cuda_error()})"
+        raise LseMergeError(rc, strerror(rc) + extra)
+    return rc
+
+
+def decode_raw(q_ptr: int, k_ptr: int, v_ptr: int, kv_len_ptr: int, B: int, Hq: int, Hkv: int,
+               L: int, D: int, R: int, scale: float, strides, dtype: int, out_ptr: int,
+               out_lse_ptr: int, stream: int = 0, fused: bool = True, out_dtype: int = BF16,
+               check: bool = True) -> int:
+    """lse_merge_decode_attention (fused) or lse_merge_decode_partials (fp32
+    partials [B,Hq,R,D] / [B,Hq,R] into out_ptr / out_lse_ptr).  ``strides`` =
+    (q_b, q_h, k_b, k_h, k_l, v_b, v_h, v_l) in elements, or None (dense)."""
+    st = None if strides is None else ctypes.pointer(AttnStrides(*[int(x) for x in strides]))
+    args = (q_ptr, k_ptr, v_ptr, kv_len_ptr or None, B, Hq, Hkv, L, D, R, float(scale), st, dtype)
+    if fused:
+        rc = lib.lse_merge_decode_attention(*args, out_dtype, out_ptr, out_lse_ptr, stream or None)
+    else:
+        rc = lib.lse_merge_decode_partials(*args, out_ptr, out_lse_ptr, stream or None)
+    return _check(rc, check)

@@ -3,7 +3,8 @@ from __future__ import annotations
 
 from ._native import (BF16, F16, F32, PATH_AUTO, PATH_LATENCY, PATH_SCALAR, PATH_STREAM,
                       PATH_VECTOR,
-                      LseMergeError, merge_raw, plan_query, state_update_raw, strerror)
+                      LseMergeError, decode_raw, merge_raw, plan_query, state_update_raw,
+                      strerror)
 
 
 def dtype_code(dtype) -> int:
@@ -219,3 +220,73 @@ def merge_state_(o_acc, lse_acc, o_new, lse_new):
                          lse_new.data_ptr(), B, H, D, st, dtype_code(o_acc.dtype),
                          dtype_code(o_new.dtype), torch.cuda.current_stream(dev).cuda_stream)
     return o_acc, lse_acc
+
+
+def decode_attention(q, k, v, *, splits: int | None = None, scale: float | None = None,
+                     kv_len=None, out_dtype=None, fused: bool | None = None):
+    """Split-KV decode attention on the GPU, its partials merged by LSE weight.
+
+    q [B, Hq, D]; k, v [B, Hkv, L, D] (bf16 or fp16, stride 1 along D, other
+    strides free); Hq a multiple of Hkv; D 64 or 128; kv_len an optional int32
+    CUDA tensor [B] of valid key counts.  The keys of each sequence are cut
+    into ``splits`` shards (default: enough shards for about two CTAs per SM,
+    a power of two of at least 64 keys each).  fused=True merges the shards
+    inside the attention kernel through a thread-block cluster (splits 1, 2,
+    4 or 8); fused=False writes the fp32 partials and merges them with
+    merge(), two launches.  By default the fused kernel is used below 128 MB
+    of keys and values when its splits still give every SM a CTA, where
+    saving a launch matters (measured on B200: 27.4 vs 28.9 us at B=4,
+    L=8192), and the two launches otherwise: above that size cluster
+    scheduling costs more than the second launch (166 vs 176 us at B=64,
+    L=4096), and few sequences need more than 8 splits (B=1 with one KV head
+    and 32768 keys: 15 us at 64 splits, 42 us at 8).  Returns (out [B, Hq, D],
+    lse [B, Hq]) with the natural-log lse of the scaled scores.
+    """
+    import math
+    import torch
+    B, Hq, D = q.shape
+    _, Hkv, L, _ = k.shape
+    if tuple(v.shape) != tuple(k.shape) or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k and v must be [B, Hkv, L, D] with q [B, Hq, D]")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("decode_attention runs on CUDA tensors only")
+    if q.stride(-1) != 1 or k.stride(-1) != 1 or v.stride(-1) != 1:
+        raise ValueError("q, k and v must be contiguous along D")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    dev = q.device
+    kv_bytes = 2 * B * Hkv * L * D * q.element_size()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    if fused is None:
+        # fused: its (at most 8) splits must still give every SM a CTA
+        fused = (kv_bytes <= (128 << 20) and B * Hkv * 8 >= sms
+                 and (splits is None or splits in (1, 2, 4, 8)))
+    if splits is None:
+        want = max(1, -(-2 * sms // (B * Hkv)))
+        splits = 1
+        while splits < want and splits < (8 if fused else 64) and splits * 64 < L:
+            splits *= 2
+    scale = (1.0 / math.sqrt(D)) if scale is None else float(scale)
+    out_dtype = out_dtype or q.dtype
+    st = (q.stride(0), q.stride(1), k.stride(0), k.stride(1), k.stride(2),
+          v.stride(0), v.stride(1), v.stride(2))
+    klen = 0
+    if kv_len is not None:
+        if kv_len.dtype != torch.int32 or not kv_len.is_cuda or kv_len.numel() != B:
+            raise ValueError("kv_len must be an int32 CUDA tensor of B lengths")
+        kv_len = kv_len.contiguous()
+        klen = kv_len.data_ptr()
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev).cuda_stream
+        if fused:
+            out = torch.empty((B, Hq, D), dtype=out_dtype, device=dev)
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+            decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), klen, B, Hq, Hkv, L, D, splits,
+                       scale, st, dtype_code(q.dtype), out.data_ptr(), lse.data_ptr(), s,
+                       fused=True, out_dtype=dtype_code(out_dtype))
+            return out, lse
+        po = torch.empty((B, Hq, splits, D), dtype=torch.float32, device=dev)
+        pl = torch.empty((B, Hq, splits), dtype=torch.float32, device=dev)
+        decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), klen, B, Hq, Hkv, L, D, splits,
+                   scale, st, dtype_code(q.dtype), po.data_ptr(), pl.data_ptr(), s, fused=False)
+        return merge(po, pl, out_dtype=out_dtype)

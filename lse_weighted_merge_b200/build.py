@@ -13,7 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblse_merge.so")
-SOURCES = [os.path.join(CSRC, "plan.cpp"), os.path.join(CSRC, "lse_merge.cu")]
+SOURCES = [os.path.join(CSRC, "plan.cpp"), os.path.join(CSRC, "lse_merge.cu"),
+           os.path.join(CSRC, "decode_attention.cu")]
 HEADERS = [os.path.join(INCLUDE, "lse_merge.h"), os.path.join(CSRC, "plan.h")]
 
 NVCC_FLAGS = [

@@ -1,0 +1,549 @@
+// decode_attention.cu -- split-KV decode attention on sm_100a, optionally with
+// the LSE-weighted merge of its partials fused in through a thread-block
+// cluster.
+//
+// The producer of the merge's inputs (page "[flashinfer] FlashInfer의
+// Context-Parallel Decode 최적화: Fused A2A + LSE Reduce", section "들어가며":
+// each rank attends over its own KV shard and returns o_r and lse_r).  Here
+// the shards are the R splits of one sequence's keys, computed by R CTAs.
+//
+// One CTA = one (batch b, KV head, split r), kAttnWarps warps.  The G query
+// heads that share the KV head are the rows of a 16-row tile, so both
+// products are tensor-core mma.sync m16n8k16 (bf16/fp16 in, fp32 accumulate):
+//   S = Q K^T   A = Q (16 x D, registers), B = K^T from a shared-memory tile
+//   O += P V    A = P (the S accumulators, exponentiated, as bf16/fp16),
+//               B = V from a shared-memory tile (ldmatrix .trans)
+// Each warp owns the key tiles w, w + kAttnWarps, ... of the split and a
+// private ring of kAttnStages K/V tiles filled with cp.async (16-byte
+// chunks, XOR-swizzled so ldmatrix rows hit distinct banks).  An online
+// softmax (running max m and sum l in log2 units) keeps O unnormalised.
+// After the key loop the warps' states are merged in shared memory (the
+// LSE merge again, over the warps), giving the split's (o_r, lse_r).
+//
+//  * lse_merge_decode_partials writes (o_r, lse_r) to global memory.
+//  * lse_merge_decode_attention launches the R splits of one (b, KV head) as
+//    a cluster: after a cluster barrier CTA r merges columns
+//    [r*D/R, (r+1)*D/R) of every head from all R partials, read from the
+//    other CTAs' shared memory (distributed shared memory), and a second
+//    barrier keeps every CTA alive until the others have read it.
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "lse_merge.h"
+#include "plan.h"
+
+namespace cg = cooperative_groups;
+
+namespace lsem {
+namespace attn {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AParams {
+    const char* q;
+    const char* k;
+    const char* v;
+    const int32_t* kv_len;
+    int64_t q_b, q_h, k_b, k_h, k_l, v_b, v_h, v_l;   // BYTE strides
+    int Hq, G, L, R;
+    float scale_log2;      // scale * log2(e)
+    float* po;             // partials [B, Hq, R, D] (unfused)
+    float* pl;             // [B, Hq, R]
+    char* out;             // merged output [B, Hq, D] (fused)
+    float* out_lse;        // [B, Hq]
+};
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// 16-byte global -> shared copy; `bytes` = 0 writes zeros without reading.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+template <typename T>
+struct Mma;
+
+template <>
+struct Mma<__nv_bfloat16> {
+    __device__ static void run(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+            "{%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ static uint32_t pack(float lo, float hi) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+};
+
+template <>
+struct Mma<__half> {
+    __device__ static void run(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+            "{%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    }
+    __device__ static uint32_t pack(float lo, float hi) {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+};
+
+template <typename TOut>
+__device__ __forceinline__ void store_out(char* p, float x);
+template <>
+__device__ __forceinline__ void store_out<float>(char* p, float x) { *reinterpret_cast<float*>(p) = x; }
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(char* p, float x) {
+    *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ void store_out<__half>(char* p, float x) {
+    *reinterpret_cast<__half*>(p) = __float2half_rn(x);
+}
+
+// Shared-memory byte offset of 16-byte chunk `ch` of tile row `row` (rows of
+// D*2 bytes): chunks are XOR-swizzled within groups of 8 so that the 8 rows
+// one ldmatrix 8x8 matrix reads fall in 8 different bank groups.
+template <int D>
+__device__ __forceinline__ uint32_t tile_off(int row, int ch) {
+    return (uint32_t)(row * (D * 2) + ((ch ^ (row & 7)) * 16));
+}
+
+template <typename T, int D, bool FUSED, typename TOut>
+__global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const AParams p) {
+    constexpr int TK = kAttnTileKeys;
+    constexpr int S = kAttnStages;
+    constexpr int KS = D / 16;         // k-steps of Q K^T
+    constexpr int NT = D / 8;          // n-tiles of P V
+    constexpr int CPR = D / 8;         // 16-byte chunks per K/V row
+    constexpr int TILE = TK * D * 2;   // bytes of one K (or V) tile
+    constexpr int NJ = TK / 8;         // n-tiles of Q K^T (8 keys each)
+    constexpr int KK = TK / 16;        // k-steps of P V (16 keys each)
+    static_assert(TK == 16 || TK == 32, "key tile of 16 or 32");
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    pdl_wait();
+    pdl_release();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int r = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int G = p.G, R = p.R;
+    const int h0 = hk * G;
+
+    int len = p.L;
+    if (p.kv_len) len = min(max(__ldg(p.kv_len + b), 0), p.L);
+    const int per = (len + R - 1) / R;
+    const int lo = min(len, r * per), hi = min(len, lo + per);
+    const int ntiles = (hi - lo + TK - 1) / TK;
+    const int mine = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
+
+    const char* kb = p.k + (int64_t)b * p.k_b + (int64_t)hk * p.k_h;
+    const char* vb = p.v + (int64_t)b * p.v_b + (int64_t)hk * p.v_h;
+    unsigned char* ring = smem + (size_t)warp * S * 2 * TILE;
+    const uint32_t ring_u = smem_u32(ring);
+
+    // Q as the A operand: rows g and g+8 are query heads h0+g, h0+g+8 (zero
+    // beyond the group), columns 16*ks + 2t (+1) and + 8.
+    uint32_t qa[KS][4];
+    {
+        const char* qb = p.q + (int64_t)b * p.q_b;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int c0 = (ks * 16 + 2 * t) * 2;
+            qa[ks][0] = qa[ks][1] = qa[ks][2] = qa[ks][3] = 0u;
+            if (g < G) {
+                const char* row = qb + (int64_t)(h0 + g) * p.q_h;
+                qa[ks][0] = __ldg(reinterpret_cast<const unsigned int*>(row + c0));
+                qa[ks][2] = __ldg(reinterpret_cast<const unsigned int*>(row + c0 + 16));
+            }
+            if (g + 8 < G) {
+                const char* row = qb + (int64_t)(h0 + g + 8) * p.q_h;
+                qa[ks][1] = __ldg(reinterpret_cast<const unsigned int*>(row + c0));
+                qa[ks][3] = __ldg(reinterpret_cast<const unsigned int*>(row + c0 + 16));
+            }
+        }
+    }
+
+    // Copy key tile `i` of this warp (keys lo + (warp + i*kAttnWarps)*TK ...)
+    // into ring stage `s`; keys at or past `hi` are zero-filled.
+    auto issue = [&](int i, int s) {
+        const int key0 = lo + (warp + i * kAttnWarps) * TK;
+        const uint32_t kd = ring_u + (uint32_t)(s * 2 * TILE);
+        const uint32_t vd = kd + TILE;
+#pragma unroll 4
+        for (int c = lane; c < TK * CPR; c += 32) {
+            const int row = c / CPR, ch = c - row * CPR;
+            const int key = key0 + row;
+            const bool ok = key < hi;
+            const int64_t src_key = ok ? key : lo;
+            cp_async16(kd + tile_off<D>(row, ch), kb + src_key * p.k_l + ch * 16, ok ? 16 : 0);
+            cp_async16(vd + tile_off<D>(row, ch), vb + src_key * p.v_l + ch * 16, ok ? 16 : 0);
+        }
+    };
+
+    float m0 = -INFINITY, m1 = -INFINITY;   // running max (log2 units) of rows g, g+8
+    float l0 = 0.f, l1 = 0.f;               // this thread's share of the running sums
+    float oacc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+
+#pragma unroll
+    for (int s = 0; s < S - 1; ++s) {
+        if (s < mine) issue(s, s);
+        cp_commit();
+    }
+    for (int i = 0; i < mine; ++i) {
+        if (i + S - 1 < mine) issue(i + S - 1, (i + S - 1) % S);
+        cp_commit();
+        cp_wait<S - 1>();
+        __syncwarp();
+        const uint32_t ks_u = ring_u + (uint32_t)((i % S) * 2 * TILE);
+        const uint32_t vs_u = ks_u + TILE;
+        const int key0 = lo + (warp + i * kAttnWarps) * TK;
+
+        // ---- S = Q K^T: NJ n-tiles of 8 keys
+        float sacc[NJ][4];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+            for (int jp = 0; jp < NJ / 2; ++jp) {
+                const int mi = lane >> 3, rr = lane & 7;
+                const int row = (2 * jp + (mi >> 1)) * 8 + rr;
+                const int ch = 2 * ks + (mi & 1);
+                uint32_t bf[4];
+                ldsm_x4(ks_u + tile_off<D>(row, ch), bf);
+                Mma<T>::run(sacc[2 * jp], qa[ks], bf[0], bf[1]);
+                Mma<T>::run(sacc[2 * jp + 1], qa[ks], bf[2], bf[3]);
+            }
+        }
+
+        // ---- online softmax over this tile (scores in log2 units)
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const bool ok = key0 + 8 * j + 2 * t + e < hi;
+                sacc[j][e] = ok ? sacc[j][e] * p.scale_log2 : -INFINITY;
+                sacc[j][e + 2] = ok ? sacc[j][e + 2] * p.scale_log2 : -INFINITY;
+                mx0 = fmaxf(mx0, sacc[j][e]);
+                mx1 = fmaxf(mx1, sacc[j][e + 2]);
+            }
+        }
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
+        // every tile holds at least one valid key, so the new maxima are finite
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);   // 0 on the first tile
+        m0 = n0;
+        m1 = n1;
+        l0 *= a0;
+        l1 *= a1;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            oacc[n][0] *= a0;
+            oacc[n][1] *= a0;
+            oacc[n][2] *= a1;
+            oacc[n][3] *= a1;
+        }
+        uint32_t pa[KK][4];   // P as the A operand of the 16-key k-steps
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const float p0 = exp2f(sacc[j][0] - n0), p1 = exp2f(sacc[j][1] - n0);
+            const float p2 = exp2f(sacc[j][2] - n1), p3 = exp2f(sacc[j][3] - n1);
+            l0 += p0 + p1;
+            l1 += p2 + p3;
+            pa[j >> 1][(j & 1) * 2 + 0] = Mma<T>::pack(p0, p1);
+            pa[j >> 1][(j & 1) * 2 + 1] = Mma<T>::pack(p2, p3);
+        }
+
+        // ---- O += P V: D/8 n-tiles, KK k-steps of 16 keys
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+#pragma unroll
+            for (int np = 0; np < NT / 2; ++np) {
+                const int mi = lane >> 3, rr = lane & 7;
+                const int row = 16 * kk + (mi & 1) * 8 + rr;
+                const int ch = 2 * np + (mi >> 1);
+                uint32_t bf[4];
+                ldsm_x4_t(vs_u + tile_off<D>(row, ch), bf);
+                Mma<T>::run(oacc[2 * np], pa[kk], bf[0], bf[1]);
+                Mma<T>::run(oacc[2 * np + 1], pa[kk], bf[2], bf[3]);
+            }
+        }
+        __syncwarp();
+    }
+    cp_wait<0>();
+    l0 += __shfl_xor_sync(kFull, l0, 1);
+    l0 += __shfl_xor_sync(kFull, l0, 2);
+    l1 += __shfl_xor_sync(kFull, l1, 1);
+    l1 += __shfl_xor_sync(kFull, l1, 2);
+    __syncthreads();   // every warp is done with its ring: reuse the shared memory
+
+    // ---- merge the warps' states: per warp m[16], l[16], O[16][D]
+    float* st_m = reinterpret_cast<float*>(smem);
+    float* st_l = st_m + kAttnWarps * 16;
+    float* st_o = st_l + kAttnWarps * 16;
+    float* sp_o = st_o + kAttnWarps * 16 * D;   // the split's partial o [16][D]
+    float* sp_l = sp_o + 16 * D;                // and its lse [16] (natural log)
+    if (t == 0) {
+        st_m[warp * 16 + g] = m0;
+        st_m[warp * 16 + g + 8] = m1;
+        st_l[warp * 16 + g] = l0;
+        st_l[warp * 16 + g + 8] = l1;
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        float* o0 = st_o + (warp * 16 + g) * D + 8 * n + 2 * t;
+        float* o1 = st_o + (warp * 16 + g + 8) * D + 8 * n + 2 * t;
+        o0[0] = oacc[n][0];
+        o0[1] = oacc[n][1];
+        o1[0] = oacc[n][2];
+        o1[1] = oacc[n][3];
+    }
+    __syncthreads();
+    const int64_t rows_b = (int64_t)b * p.Hq + h0;
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int gg = idx / D, d = idx - gg * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, st_m[w * 16 + gg]);
+        float den = 0.f, num = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kAttnWarps; ++w) {
+                const float mw = st_m[w * 16 + gg];
+                if (mw != -INFINITY) {
+                    const float e = exp2f(mw - M);
+                    den += e * st_l[w * 16 + gg];
+                    num += e * st_o[(w * 16 + gg) * D + d];
+                }
+            }
+        }
+        const float o = den > 0.f ? num / den : 0.f;
+        const float lse = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+        if constexpr (FUSED) {
+            sp_o[gg * D + d] = o;
+            if (d == 0) sp_l[gg] = lse;
+        } else {
+            const int64_t row = rows_b + gg;
+            p.po[(row * R + r) * D + d] = o;
+            if (d == 0) p.pl[row * R + r] = lse;
+        }
+    }
+
+    if constexpr (FUSED) {
+        // ---- merge the R splits of this (b, KV head) across the cluster
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();   // every CTA's partial is in its shared memory
+        const int rank = (int)cluster.block_rank();
+        const int cols = D / R;
+        for (int idx = threadIdx.x; idx < G * cols; idx += blockDim.x) {
+            const int gg = idx / cols, d = rank * cols + (idx - gg * cols);
+            // all R remote loads of a kind are issued before any is used
+            float lj[8], oj[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                lj[j] = -INFINITY;
+                oj[j] = 0.f;
+                if (j < R) {
+                    lj[j] = *cluster.map_shared_rank(sp_l + gg, j);
+                    oj[j] = *cluster.map_shared_rank(sp_o + gg * D + d, j);
+                }
+            }
+            float M = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) M = fmaxf(M, lj[j]);
+            float den = 0.f, num = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (lj[j] != -INFINITY) {   // an empty split's o is not used
+                        const float e = expf(lj[j] - M);
+                        den += e;
+                        num += e * oj[j];
+                    }
+                }
+            }
+            const int64_t row = rows_b + gg;
+            store_out<TOut>(p.out + (row * D + d) * (int64_t)sizeof(TOut), den > 0.f ? num / den : 0.f);
+            if (rank == 0 && idx - gg * cols == 0)
+                p.out_lse[row] = den > 0.f ? M + logf(den) : -INFINITY;
+        }
+        cluster.sync();   // keep this CTA's shared memory alive until all have read it
+    }
+}
+
+using AttnFn = void (*)(AParams);
+
+template <typename T, int D>
+AttnFn pick_d(bool fused, int out_dtype) {
+    if (!fused) return decode_attn_kernel<T, D, false, float>;
+    switch (out_dtype) {
+        case LSE_MERGE_F32: return decode_attn_kernel<T, D, true, float>;
+        case LSE_MERGE_F16: return decode_attn_kernel<T, D, true, __half>;
+        default: return decode_attn_kernel<T, D, true, __nv_bfloat16>;
+    }
+}
+template <typename T>
+AttnFn pick_t(int D, bool fused, int out_dtype) {
+    return D == 64 ? pick_d<T, 64>(fused, out_dtype) : pick_d<T, 128>(fused, out_dtype);
+}
+AttnFn pick(int dtype, int D, bool fused, int out_dtype) {
+    return dtype == LSE_MERGE_F16 ? pick_t<__half>(D, fused, out_dtype)
+                                  : pick_t<__nv_bfloat16>(D, fused, out_dtype);
+}
+
+// cudaFuncSetAttribute once per (kernel, device) for dynamic shared memory
+// above 48 KB.
+std::mutex g_attr_mu;
+struct AttrDone {
+    const void* fn;
+    int dev;
+};
+AttrDone g_attr_done[128];
+int g_attr_n = 0;
+
+cudaError_t ensure_smem(AttnFn fn, int64_t bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    for (int i = 0; i < g_attr_n; ++i)
+        if (g_attr_done[i].fn == (const void*)fn && g_attr_done[i].dev == dev) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && g_attr_n < 128) g_attr_done[g_attr_n++] = AttrDone{(const void*)fn, dev};
+    return e;
+}
+
+
+int launch(const void* q, const void* k, const void* v, const int32_t* kv_len, int B, int Hq,
+           int Hkv, int L, int D, int R, float scale, const lse_merge_attn_strides* strides,
+           int dtype, int out_dtype, void* out_o, float* out_lse, bool fused, cudaStream_t stream) {
+    if (Hq < 1 || Hkv < 1 || L < 1 || D < 1) return LSE_MERGE_EDIMS;
+    const lse_merge_attn_strides st = strides ? *strides : default_attn_strides(Hq, Hkv, L, D);
+    AttnPlan pl;
+    const int rc = make_attn_plan(q, k, v, B, Hq, Hkv, L, D, R, scale, st, dtype,
+                                  fused ? out_dtype : LSE_MERGE_F32, out_o, out_lse, fused, &pl);
+    if (rc != LSE_MERGE_OK) return rc;
+    AParams ap;
+    ap.q = static_cast<const char*>(q);
+    ap.k = static_cast<const char*>(k);
+    ap.v = static_cast<const char*>(v);
+    ap.kv_len = kv_len;
+    ap.q_b = st.q_b * 2;
+    ap.q_h = st.q_h * 2;
+    ap.k_b = st.k_b * 2;
+    ap.k_h = st.k_h * 2;
+    ap.k_l = st.k_l * 2;
+    ap.v_b = st.v_b * 2;
+    ap.v_h = st.v_h * 2;
+    ap.v_l = st.v_l * 2;
+    ap.Hq = Hq;
+    ap.G = pl.G;
+    ap.L = L;
+    ap.R = R;
+    ap.scale_log2 = scale * kLog2e;
+    ap.po = fused ? nullptr : static_cast<float*>(out_o);
+    ap.pl = fused ? nullptr : out_lse;
+    ap.out = fused ? static_cast<char*>(out_o) : nullptr;
+    ap.out_lse = fused ? out_lse : nullptr;
+    const AttnFn fn = pick(dtype, D, fused, out_dtype);
+    cudaError_t e = ensure_smem(fn, pl.smem);
+    if (e == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)R, (unsigned)Hkv, (unsigned)B);
+        cfg.blockDim = dim3(kAttnWarps * 32);
+        cfg.dynamicSmemBytes = (size_t)pl.smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        int na = 0;
+        if (kPdl) {
+            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        if (fused) {
+            attr[na].id = cudaLaunchAttributeClusterDimension;
+            attr[na].val.clusterDim.x = (unsigned)R;
+            attr[na].val.clusterDim.y = 1;
+            attr[na].val.clusterDim.z = 1;
+            ++na;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        e = cudaLaunchKernelEx(&cfg, fn, ap);
+    }
+    if (e != cudaSuccess) {
+        set_last_cuda_error((int)e);
+        (void)cudaGetLastError();
+        return LSE_MERGE_ELAUNCH;
+    }
+    return LSE_MERGE_OK;
+}
+
+}  // namespace
+}  // namespace attn
+}  // namespace lsem
+
+extern "C" {
+
+int lse_merge_decode_partials(const void* q, const void* k, const void* v, const int32_t* kv_len,
+                              int B, int Hq, int Hkv, int L, int D, int R, float scale,
+                              const lse_merge_attn_strides* strides, int dtype,
+                              float* partial_o, float* partial_lse, lse_merge_stream_t stream) {
+    return lsem::attn::launch(q, k, v, kv_len, B, Hq, Hkv, L, D, R, scale, strides, dtype,
+                              LSE_MERGE_F32, partial_o, partial_lse, false,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+int lse_merge_decode_attention(const void* q, const void* k, const void* v, const int32_t* kv_len,
+                               int B, int Hq, int Hkv, int L, int D, int R, float scale,
+                               const lse_merge_attn_strides* strides, int dtype, int out_dtype,
+                               void* out_o, float* out_lse, lse_merge_stream_t stream) {
+    return lsem::attn::launch(q, k, v, kv_len, B, Hq, Hkv, L, D, R, scale, strides, dtype,
+                              out_dtype, out_o, out_lse, true,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -844,7 +844,6 @@ KernelFn pick(const lse_merge_plan& pl, int in_dtype, int out_dtype) {
     }
 }
 
-thread_local int g_last_cuda_error = 0;
 
 int log2i(int x) {
     int l = 0;
@@ -904,7 +903,7 @@ int run(const void* partial_o, const float* partial_lse, int R, int B, int H, in
         int grid = 0;
         const int qe = persistent_grid((const void*)fn, pl.block, want, &grid);
         if (qe != 0) {
-            g_last_cuda_error = qe;
+            set_last_cuda_error(qe);
             (void)cudaGetLastError();
             return LSE_MERGE_ELAUNCH;
         }
@@ -915,7 +914,7 @@ int run(const void* partial_o, const float* partial_lse, int R, int B, int H, in
         e = cudaLaunchKernelEx(&cfg, pick(pl, in_dtype, out_dtype), kp);
     }
     if (e != cudaSuccess) {
-        g_last_cuda_error = (int)e;
+        set_last_cuda_error((int)e);
         (void)cudaGetLastError();  // the failure belongs to this call; do not leave it pending
         return LSE_MERGE_ELAUNCH;
     }
@@ -966,7 +965,7 @@ int run_state(void* o_acc, float* lse_acc, const void* o_new, const float* lse_n
     cfg.numAttrs = kPdl ? 1 : 0;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, pick_state(acc_dtype, new_dtype, pl.vec != 0), sp);
     if (e != cudaSuccess) {
-        g_last_cuda_error = (int)e;
+        set_last_cuda_error((int)e);
         (void)cudaGetLastError();
         return LSE_MERGE_ELAUNCH;
     }
@@ -999,6 +998,6 @@ int lse_merge_state_update(void* o_acc, float* lse_acc, const void* o_new, const
                            new_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int lse_merge_last_cuda_error(void) { return lsem::g_last_cuda_error; }
+int lse_merge_last_cuda_error(void) { return lsem::last_cuda_error(); }
 
 }  // extern "C"

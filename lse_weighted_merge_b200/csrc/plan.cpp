@@ -18,6 +18,12 @@
 
 namespace lsem {
 
+namespace {
+thread_local int g_last_cuda_error = 0;
+}
+void set_last_cuda_error(int e) { g_last_cuda_error = e; }
+int last_cuda_error() { return g_last_cuda_error; }
+
 int elem_bytes(int dtype) {
     switch (dtype) {
         case LSE_MERGE_F32: return 4;
@@ -172,6 +178,72 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
     return LSE_MERGE_OK;
 }
 
+lse_merge_attn_strides default_attn_strides(int Hq, int Hkv, int L, int D) {
+    lse_merge_attn_strides s;
+    s.q_b = (int64_t)Hq * D;
+    s.q_h = D;
+    s.k_b = s.v_b = (int64_t)Hkv * L * D;
+    s.k_h = s.v_h = (int64_t)L * D;
+    s.k_l = s.v_l = D;
+    return s;
+}
+
+// out_o / out_lse: the merged outputs (fused) or the partial buffers
+// (dense [B,Hq,R,D] and [B,Hq,R] fp32) of the unfused producer.
+int make_attn_plan(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int L,
+                   int D, int R, float scale, const lse_merge_attn_strides& st, int dtype,
+                   int out_dtype, const void* out_o, const float* out_lse, int fused,
+                   AttnPlan* plan) {
+    const int ob = elem_bytes(out_dtype);
+    if (elem_bytes(dtype) == 0 || ob == 0) return LSE_MERGE_EDTYPE;
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || D < 1 || R < 1) return LSE_MERGE_EDIMS;
+    if (!q || !k || !v || !out_o || !out_lse || !plan) return LSE_MERGE_ENULL;
+    if (st.q_b < 0 || st.q_h < 0 || st.k_b < 0 || st.k_h < 0 || st.k_l < 0 || st.v_b < 0 ||
+        st.v_h < 0 || st.v_l < 0)
+        return LSE_MERGE_ESTRIDE;
+    if (dtype == LSE_MERGE_F32) return LSE_MERGE_EUNSUP;
+    if (D != 64 && D != 128) return LSE_MERGE_EUNSUP;
+    if (Hq % Hkv != 0 || Hq / Hkv > 16) return LSE_MERGE_EUNSUP;
+    if (fused && R != 1 && R != 2 && R != 4 && R != 8) return LSE_MERGE_EUNSUP;
+    if (B > 65535 || Hkv > 65535 || R > 65535) return LSE_MERGE_EDIMS;
+    if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return LSE_MERGE_EDIMS;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out_o, ob) ||
+        !aligned(out_lse, 4))
+        return LSE_MERGE_EALIGN;
+    const int64_t s16[8] = {st.q_b, st.q_h, st.k_b, st.k_h, st.k_l, st.v_b, st.v_h, st.v_l};
+    for (int i = 0; i < 8; ++i)
+        if ((s16[i] * 2) % 16 != 0) return LSE_MERGE_EALIGN;
+    const i128 lim = (i128)1 << 62;
+    const i128 q_bytes = ((i128)(B - 1) * st.q_b + (i128)(Hq - 1) * st.q_h + D) * 2;
+    const i128 k_bytes = ((i128)(B - 1) * st.k_b + (i128)(Hkv - 1) * st.k_h + (i128)(L - 1) * st.k_l + D) * 2;
+    const i128 v_bytes = ((i128)(B - 1) * st.v_b + (i128)(Hkv - 1) * st.v_h + (i128)(L - 1) * st.v_l + D) * 2;
+    const i128 rows = (i128)B * Hq;
+    const i128 o_bytes = fused ? rows * D * ob : rows * R * D * 4;
+    const i128 l_bytes = fused ? rows * 4 : rows * R * 4;
+    if (q_bytes > lim || k_bytes > lim || v_bytes > lim || o_bytes > lim || l_bytes > lim)
+        return LSE_MERGE_EDIMS;
+    const Span sq{(uintptr_t)q, (i128)(uintptr_t)q + q_bytes};
+    const Span sk{(uintptr_t)k, (i128)(uintptr_t)k + k_bytes};
+    const Span sv{(uintptr_t)v, (i128)(uintptr_t)v + v_bytes};
+    const Span so{(uintptr_t)out_o, (i128)(uintptr_t)out_o + o_bytes};
+    const Span sl{(uintptr_t)out_lse, (i128)(uintptr_t)out_lse + l_bytes};
+    if (overlap(so, sq) || overlap(so, sk) || overlap(so, sv) || overlap(sl, sq) ||
+        overlap(sl, sk) || overlap(sl, sv) || overlap(so, sl))
+        return LSE_MERGE_EALIAS;
+    AttnPlan p{};
+    p.G = Hq / Hkv;
+    p.fused = fused;
+    const int64_t ring = (int64_t)kAttnWarps * kAttnStages * 2 * kAttnTileKeys * D * 2;
+    // after the key loop the ring is reused: each warp's state (16 rows of m, l
+    // and D accumulators) and, behind it, the split's merged partial
+    const int64_t states = (int64_t)kAttnWarps * 16 * (D + 2) * 4;
+    const int64_t split = (int64_t)16 * (D + 1) * 4;
+    const int64_t need = states + split;
+    p.smem = ring > need ? ring : need;
+    *plan = p;
+    return LSE_MERGE_OK;
+}
+
 int make_state_plan(const void* o_acc, const float* lse_acc, const void* o_new,
                     const float* lse_new, int B, int H, int D, const lse_merge_state_strides& st,
                     int acc_dtype, int new_dtype, StatePlan* plan) {
@@ -233,6 +305,7 @@ const char* lse_merge_strerror(int code) {
         case LSE_MERGE_ELAUNCH: return "CUDA kernel launch failed";
         case LSE_MERGE_EALIGN: return "a pointer is not aligned to its element size";
         case LSE_MERGE_EPATH: return "the requested kernel path cannot take these arguments";
+        case LSE_MERGE_EUNSUP: return "shape not implemented by the decode-attention kernels (dtype, D, group, R)";
         default: return "unknown lse_merge error code";
     }
 }

@@ -58,6 +58,10 @@ constexpr int kLatencyMaxThreads = kBlock;
 
 int elem_bytes(int dtype);
 
+// The cudaError_t of the last failed launch on this host thread.
+void set_last_cuda_error(int e);
+int last_cuda_error();
+
 // Validate the arguments and fill *plan for `path` (LSE_MERGE_PATH_*).
 // Returns LSE_MERGE_OK or the error code lse_merge would return.
 int make_plan(const void* partial_o, const float* partial_lse, int R, int B, int H, int D,
@@ -76,6 +80,28 @@ struct StatePlan {
     int block;
     int64_t grid;
 };
+
+// Decode attention: validated geometry.
+struct AttnPlan {
+    int G;            // query heads per KV head
+    int fused;        // 1: cluster merge inside the kernel
+    int64_t smem;     // dynamic shared memory per CTA
+};
+constexpr int kAttnWarps = 4;     // warps per CTA, each a private K/V ring
+#ifndef LSEM_ATTN_TK
+#define LSEM_ATTN_TK 16
+#endif
+#ifndef LSEM_ATTN_STAGES
+#define LSEM_ATTN_STAGES 3
+#endif
+constexpr int kAttnTileKeys = LSEM_ATTN_TK;    // keys per K/V tile (16 or 32)
+constexpr int kAttnStages = LSEM_ATTN_STAGES;  // tiles per warp ring
+
+int make_attn_plan(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int L,
+                   int D, int R, float scale, const lse_merge_attn_strides& st, int dtype,
+                   int out_dtype, const void* out_o, const float* out_lse, int fused,
+                   AttnPlan* plan);
+lse_merge_attn_strides default_attn_strides(int Hq, int Hkv, int L, int D);
 
 // Validate the arguments of lse_merge_state_update and fill *plan.
 int make_state_plan(const void* o_acc, const float* lse_acc, const void* o_new,

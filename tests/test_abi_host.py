@@ -180,3 +180,32 @@ def sq(B=2, H=3, D=64, st=None, a=nat.BF16, n=nat.BF16, acc=OUT, lacc=OUTL, new=
 def test_state_update_validation(kw, code):
     # rejected before any CUDA call
     assert sq(**kw) == code, (kw, nat.strerror(code))
+
+
+def dq(B=2, Hq=8, Hkv=2, L=100, D=128, R=4, scale=0.1, st=None, dt=nat.BF16, q=PO, k=PL,
+       v=0x7f4000000000, out=OUT, outl=OUTL, fused=True, odt=nat.BF16):
+    return nat.decode_raw(q, k, v, 0, B, Hq, Hkv, L, D, R, scale, st, dt, out, outl,
+                          fused=fused, out_dtype=odt, check=False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dt=nat.F32), nat.EUNSUP), (dict(dt=7), nat.EDTYPE), (dict(odt=9), nat.EDTYPE),
+    (dict(D=96), nat.EUNSUP), (dict(D=256), nat.EUNSUP), (dict(Hq=6, Hkv=4), nat.EUNSUP),
+    (dict(Hq=34, Hkv=2), nat.EUNSUP), (dict(R=3), nat.EUNSUP), (dict(R=16), nat.EUNSUP),
+    (dict(B=0), nat.EDIMS), (dict(L=0), nat.EDIMS), (dict(R=0), nat.EDIMS), (dict(B=70000), nat.EDIMS),
+    (dict(scale=float("nan")), nat.EDIMS), (dict(scale=float("inf")), nat.EDIMS),
+    (dict(q=0), nat.ENULL), (dict(out=0), nat.ENULL),
+    (dict(q=PO + 8), nat.EALIGN), (dict(st=(8 * 128, 130, 2 * 100 * 128, 100 * 128, 128,
+                                            2 * 100 * 128, 100 * 128, 128)), nat.EALIGN),
+    (dict(st=(-1, 128, 0, 0, 128, 0, 0, 128)), nat.ESTRIDE),
+    (dict(out=PL + 64), nat.EALIAS), (dict(outl=PO), nat.EALIAS),
+    (dict(fused=False, out=PL), nat.EALIAS),
+])
+def test_decode_attention_validation(kw, code):
+    assert dq(**kw) == code, (kw, nat.strerror(code))
+
+
+def test_decode_valid_arguments_pass_validation():
+    # valid arguments get past validation (here, without a GPU, the launch itself fails)
+    for kw in (dict(), dict(R=3, fused=False), dict(R=64, fused=False), dict(D=64, Hq=16, Hkv=1)):
+        assert dq(**kw) in (nat.OK, nat.ELAUNCH), kw
