@@ -17,8 +17,8 @@ R*B*H*(D*2+4) + B*H*(D*4+4).  Rank 0 prints one JSON line.
             and the result back, in 8 batch slices overlapped with the merge.
   roofline  the kernel's achieved GB/s against the measured HBM copy peak,
             and its DRAM traffic from the committed ncu summary.
-  workloads eager us/call, GB/s and fraction of peak of every workload; the
-            two tiny decode shapes also CUDA-graph-replayed us/call.
+  workloads eager and CUDA-graph-replayed us/call, GB/s and fraction of
+            peak of every workload.
   state_update  the in-place fold of one partial into an accumulator.
   cpu_baseline  the fp64 CPU oracle on a bounded sample (rank 0, N = 1).
 
@@ -561,8 +561,8 @@ def extra_workloads(device, l2: int, dist) -> dict:
         row = {"eager_us_per_call": eager_us, "gbs": w.bytes_total() / (eager_us * 1e-6) / 1e9,
                "l2": "resident (latency shape)" if tiny else f"rotating {nset} sets"}
         row["frac_of_measured_hbm"] = row["gbs"] / peak
-        if tiny:
-            row["graph_us_per_call"] = time_graph(sets, 100, 20, device)
+        row["graph_us_per_call"] = time_graph(sets, 100, 20 if tiny else 5, device)
+        row["graph_gbs"] = w.bytes_total() / (row["graph_us_per_call"] * 1e-6) / 1e9
         res[name] = row
         del sets
         torch.cuda.empty_cache()

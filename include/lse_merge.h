@@ -76,6 +76,8 @@ typedef struct {
 #define LSE_MERGE_PATH_SCALAR 3   /* element loads, any alignment of strides and D */
 #define LSE_MERGE_PATH_STREAM 4   /* persistent vector kernel, loads of the next row slice
                                      issued as the current one is consumed (R <= 16) */
+#define LSE_MERGE_PATH_WIDE 5     /* one CTA per row slice, the partials spread over its
+                                     lane groups and their states merged (for large R) */
 
 /*
  * Merge R partials of B*H rows.
@@ -119,7 +121,7 @@ int lse_merge_with_path(const void* partial_o, const float* partial_lse,
  * arguments exactly as lse_merge does (pointers are only inspected, never
  * dereferenced) and fills *plan without touching the GPU. */
 typedef struct {
-    int path;            /* LSE_MERGE_PATH_VECTOR / _LATENCY / _SCALAR / _STREAM */
+    int path;            /* LSE_MERGE_PATH_VECTOR / _LATENCY / _SCALAR / _STREAM / _WIDE */
     int vec;             /* elements per lane per partial load (16 B / elem size; 1 for scalar) */
     int lanes;           /* lanes that share one row slice (power of two, <= 32) */
     int rc;              /* partial rows whose loads are in flight together per lane */

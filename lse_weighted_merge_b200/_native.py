@@ -13,9 +13,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "liblse_merge.so")
 
 F32, F16, BF16 = 0, 1, 2
-PATH_AUTO, PATH_VECTOR, PATH_LATENCY, PATH_SCALAR, PATH_STREAM = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_VECTOR, PATH_LATENCY, PATH_SCALAR, PATH_STREAM, PATH_WIDE = 0, 1, 2, 3, 4, 5
 PATH_NAMES = {PATH_VECTOR: "vector", PATH_LATENCY: "latency", PATH_SCALAR: "scalar",
-              PATH_STREAM: "stream"}
+              PATH_STREAM: "stream", PATH_WIDE: "wide"}
 
 OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH, EUNSUP = (
     0, -1, -2, -3, -4, -5, -6, -7, -8, -9)

@@ -567,6 +567,125 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const 
     }
 }
 
+
+// ------------------------------------------------------------------ wide kernel
+
+// For R > 16: one CTA of up to kWideWarps warps per row slice, so that every
+// partial of the row can be in flight at once.  The CTA's lane groups (of
+// p.lanes lanes, one 16-byte column each) are S sub-groups; sub-group s takes
+// the partials s, s + S, s + 2S, ... in batches of RC and keeps an online
+// state (running max m, weight sum, fp32 accumulator), rescaled when a batch
+// raises the max.  The S states are then merged -- the same LSE combine --
+// by shuffles inside each warp and through shared memory across warps.
+constexpr int kWideWarps = 4;
+
+__device__ __forceinline__ void combine_state(float& m, float& es, float* acc, float m2, float es2,
+                                              const float* acc2, int n) {
+    const float M = fmaxf(m, m2);
+    const float Mref = (M == -INFINITY) ? 0.f : M;
+    const float a = expf(m - Mref), a2 = expf(m2 - Mref);   // 0 for an empty state
+    for (int k = 0; k < n; ++k) acc[k] = acc[k] * a + acc2[k] * a2;
+    es = es * a + es2 * a2;
+    m = M;
+}
+
+template <typename TIn, typename TOut, int RC>
+__global__ void __launch_bounds__(kWideWarps * 32) merge_wide_kernel(const KParams p) {
+    constexpr int N = Elem<TIn>::kVec;
+    constexpr int N2 = N / 2;
+    __shared__ float sh_acc[kWideWarps][32][N];
+    __shared__ float sh_m[kWideWarps], sh_es[kWideWarps];
+    pdl_wait();
+    pdl_release();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int W = blockDim.x >> 5;                    // warps of this CTA (<= kWideWarps)
+    const int j = lane & (p.lanes - 1);
+    const int per_warp = 32 >> p.lg;                  // sub-groups per warp
+    const int S = W * per_warp;
+    const int s = warp * per_warp + (lane >> p.lg);
+    const int s_w = warp * per_warp;                  // the warp's first sub-group: most partials
+    const RowIdx ri = row_of(p, blockIdx.x);
+    const int v = ri.slice * p.lanes + j;
+    const bool vlive = v < p.dv;
+    const char* orow = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)v * 16;
+    const float* lrow = p.lse + ri.b * p.l_b + ri.h * p.l_h;
+    const int n_w = p.R > s_w ? (p.R - s_w + S - 1) / S : 0;   // partials of sub-group s_w
+    const int batches = (n_w + RC - 1) / RC;                    // warp-uniform
+
+    float m = -INFINITY, es = 0.f;
+    uint64_t acc[N2];
+#pragma unroll
+    for (int q = 0; q < N2; ++q) acc[q] = 0ull;
+    for (int bt = 0; bt < batches; ++bt) {
+        uint4 x[RC];
+#pragma unroll
+        for (int i = 0; i < RC; ++i) {
+            const int r = s + S * (bt * RC + i);
+            x[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (vlive && r < p.R) x[i] = ld_stream16(orow + (int64_t)r * p.o_r);
+        }
+        const int rj = s + S * (bt * RC + j);
+        const float l = (j < RC && rj < p.R) ? __ldg(lrow + (int64_t)rj * p.l_r) : -INFINITY;
+        const float mn = fmaxf(m, group_max(l, p.lanes));
+        const float mref = (mn == -INFINITY) ? 0.f : mn;
+        const float sc = expf(m - mref);   // rescale of the state so far (0 if it was empty)
+#pragma unroll
+        for (int q = 0; q < N2; ++q) {
+            float a, b;
+            unpack2f(acc[q], a, b);
+            acc[q] = pack2f(a * sc, b * sc);
+        }
+        const float e = expf(l - mref);
+        es = es * sc + group_sum(e, p.lanes);
+        m = mn;
+        const bool any_zero = __any_sync(kFull, j < RC && rj < p.R && e == 0.f);
+#pragma unroll
+        for (int i = 0; i < RC; ++i) {
+            const float w = __shfl_sync(kFull, e, i, p.lanes);
+            const int r = s + S * (bt * RC + i);
+            if (r < p.R && (!any_zero || w != 0.f)) {
+                uint64_t xx[N2];
+                Elem<TIn>::unpack2(x[i], xx);
+                const uint64_t ww = pack2f(w, w);
+#pragma unroll
+                for (int q = 0; q < N2; ++q) fma2(acc[q], xx[q], ww);
+            }
+        }
+    }
+    float f[N];
+#pragma unroll
+    for (int q = 0; q < N2; ++q) unpack2f(acc[q], f[2 * q], f[2 * q + 1]);
+    // merge the sub-groups of this warp: partners differ in the lane bits above lg
+    for (int off = p.lanes; off < 32; off <<= 1) {
+        float f2[N];
+#pragma unroll
+        for (int k = 0; k < N; ++k) f2[k] = __shfl_xor_sync(kFull, f[k], off);
+        const float m2 = __shfl_xor_sync(kFull, m, off);
+        const float es2 = __shfl_xor_sync(kFull, es, off);
+        combine_state(m, es, f, m2, es2, f2, N);
+    }
+    if (W > 1) {
+        if (lane < p.lanes) {
+#pragma unroll
+            for (int k = 0; k < N; ++k) sh_acc[warp][lane][k] = f[k];
+            if (lane == 0) {
+                sh_m[warp] = m;
+                sh_es[warp] = es;
+            }
+        }
+        __syncthreads();
+    }
+    if (warp == 0 && lane < p.lanes) {
+        for (int w = 1; w < W; ++w)
+            combine_state(m, es, f, sh_m[w], sh_es[w], sh_acc[w][lane], N);
+        const float inv = es > 0.f ? 1.f / es : 0.f;
+#pragma unroll
+        for (int k = 0; k < N; ++k) f[k] *= inv;
+        if (vlive) store_vec<TOut, N>(p.out + (ri.row * p.D + (int64_t)v * N) * (int64_t)sizeof(TOut), f);
+        if (ri.slice == 0 && lane == 0) p.out_lse[ri.row] = es > 0.f ? m + logf(es) : -INFINITY;
+    }
+}
+
 // ------------------------------------------------------------------ scalar kernel
 
 // Any alignment of strides and D: one warp per row, lane j handles the
@@ -820,6 +939,9 @@ int persistent_grid(const void* fn, int block, int64_t want_ctas, int* grid_out)
 template <typename TIn, typename TOut>
 KernelFn pick_kernel(const lse_merge_plan& pl) {
     if (pl.path == LSE_MERGE_PATH_SCALAR) return merge_scalar_kernel<TIn, TOut>;
+    if (pl.path == LSE_MERGE_PATH_WIDE)
+        return pl.rc == 4 ? merge_wide_kernel<TIn, TOut, 4>
+                          : pl.rc == 8 ? merge_wide_kernel<TIn, TOut, 8> : merge_wide_kernel<TIn, TOut, 16>;
     const int rc = pl.rc, nv = pl.nv;
     if (rc == 4) return nv == 4 ? merge_vec_kernel<TIn, TOut, 4, 4>
                       : nv == 2 ? merge_vec_kernel<TIn, TOut, 4, 2> : merge_vec1_kernel<TIn, TOut, 4>;

@@ -78,7 +78,7 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
     if (!o || !lse || !out_o || !out_lse || !plan) return LSE_MERGE_ENULL;
     if (st.o_r < 0 || st.o_b < 0 || st.o_h < 0 || st.lse_r < 0 || st.lse_b < 0 || st.lse_h < 0)
         return LSE_MERGE_ESTRIDE;
-    if (path < LSE_MERGE_PATH_AUTO || path > LSE_MERGE_PATH_STREAM) return LSE_MERGE_EPATH;
+    if (path < LSE_MERGE_PATH_AUTO || path > LSE_MERGE_PATH_WIDE) return LSE_MERGE_EPATH;
     if (!aligned(o, ib) || !aligned(out_o, ob) || !aligned(lse, 4) || !aligned(out_lse, 4))
         return LSE_MERGE_EALIGN;
 
@@ -125,11 +125,39 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
         int chosen = path;
         if (chosen == LSE_MERGE_PATH_AUTO)
             chosen = small ? LSE_MERGE_PATH_LATENCY
-                           : (kAutoStream && stream_ok && in_bytes <= kStreamMaxBytes
-                                  ? LSE_MERGE_PATH_STREAM
-                                  : LSE_MERGE_PATH_VECTOR);
+                           : !stream_ok ? LSE_MERGE_PATH_WIDE
+                           : (kAutoStream && in_bytes <= kStreamMaxBytes ? LSE_MERGE_PATH_STREAM
+                                                                         : LSE_MERGE_PATH_VECTOR);
         if (chosen == LSE_MERGE_PATH_LATENCY && !small) return LSE_MERGE_EPATH;
         if (chosen == LSE_MERGE_PATH_STREAM && !stream_ok) return LSE_MERGE_EPATH;
+        if (chosen == LSE_MERGE_PATH_WIDE) {
+            // One 16-byte column per lane, at least 4 lanes.  Just enough
+            // warps (at most 4) that the lane groups hold every partial of the
+            // row in one batch of at most min(16, lanes) per group; the batch
+            // size rc then shrinks to what the groups need (a power of two >= 4).
+            int lanes = next_pow2(dv < 32 ? dv : 32);
+            if (lanes < 4) lanes = 4;
+            const int rc_max = lanes < 16 ? lanes : 16;
+            const int per_warp = 32 / lanes;
+            int warps = (R + rc_max * per_warp - 1) / (rc_max * per_warp);
+            if (warps > kWideBlock / 32) warps = kWideBlock / 32;
+            const int groups_cta = warps * per_warp;
+            int rc = next_pow2((R + groups_cta - 1) / groups_cta);
+            if (rc < 4) rc = 4;
+            if (rc > rc_max) rc = rc_max;
+            p.path = chosen;
+            p.vec = vec;
+            p.lanes = lanes;
+            p.rc = rc;
+            p.nv = 1;
+            p.slices_per_row = (dv + lanes - 1) / lanes;
+            p.groups = (int64_t)(rows * p.slices_per_row);
+            p.block = warps * 32;
+            if ((i128)p.groups > 0x7fffffff) return LSE_MERGE_EDIMS;
+            p.grid = p.groups;
+            *plan = p;
+            return LSE_MERGE_OK;
+        }
         int nv = 1;
         if (chosen != LSE_MERGE_PATH_LATENCY) {
             nv = 16 / rc < kMaxNv ? 16 / rc : kMaxNv;
@@ -160,7 +188,7 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
         }
     } else {
         if (path == LSE_MERGE_PATH_VECTOR || path == LSE_MERGE_PATH_LATENCY ||
-            path == LSE_MERGE_PATH_STREAM)
+            path == LSE_MERGE_PATH_STREAM || path == LSE_MERGE_PATH_WIDE)
             return LSE_MERGE_EPATH;
         p.path = LSE_MERGE_PATH_SCALAR;
         p.vec = 1;

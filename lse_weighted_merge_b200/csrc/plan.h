@@ -40,6 +40,8 @@ constexpr int kAutoStream = LSEM_AUTO_STREAM;
 #define LSEM_STREAM_MAX_MB 256
 #endif
 constexpr long long kStreamMaxBytes = (long long)LSEM_STREAM_MAX_MB << 20;
+// Threads per CTA of the wide kernel (R > 16: one CTA per row slice).
+constexpr int kWideBlock = 128;
 // Upper bound on the 16-byte columns per lane (1, 2 or 4).
 #ifndef LSEM_MAX_NV
 #define LSEM_MAX_NV 2

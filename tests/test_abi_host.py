@@ -60,6 +60,7 @@ def q(R=2, B=1, H=2, D=64, strides=None, i=nat.BF16, o=nat.BF16, po=PO, pl=PL, o
     (dict(out=PO + 64), nat.EALIAS), (dict(outl=PL), nat.EALIAS), (dict(outl=OUT + 8), nat.EALIAS),
     (dict(out=PL), nat.EALIAS),
     (dict(path=7), nat.EPATH),
+    (dict(D=60, path=nat.PATH_WIDE), nat.EPATH),
     (dict(R=17, B=64, H=64, path=nat.PATH_STREAM), nat.EPATH),
     (dict(D=60, path=nat.PATH_STREAM), nat.EPATH),
     (dict(B=64, H=64, path=nat.PATH_LATENCY), nat.EPATH),
@@ -121,7 +122,8 @@ def test_fallback_to_scalar_and_forced_paths():
     # f32 input: 4 elements per vector; bf16 out then needs 8-byte alignment
     assert q(i=nat.F32, D=12)[1]["vec"] == 4
     assert q(i=nat.F32, o=nat.BF16, out=OUT + 8)[1]["path"] == nat.PATH_LATENCY
-    for path in (nat.PATH_VECTOR, nat.PATH_LATENCY, nat.PATH_SCALAR, nat.PATH_STREAM):
+    for path in (nat.PATH_VECTOR, nat.PATH_LATENCY, nat.PATH_SCALAR, nat.PATH_STREAM,
+                 nat.PATH_WIDE):
         rc, plan = q(path=path)
         assert rc == 0 and plan["path"] == path
     rc, plan = q(B=64, H=64, R=16, path=nat.PATH_STREAM)
@@ -130,12 +132,25 @@ def test_fallback_to_scalar_and_forced_paths():
     assert plan["grid"] == 64 * 64 * 32 // plan["block"] and plan["lanes"] == 32
 
 
-@pytest.mark.parametrize("R,want_rc,want_nv,want_lanes", [(1, 4, 2, 4), (3, 4, 2, 4), (5, 8, 1, 8),
-                                                           (9, 16, 1, 16), (16, 16, 1, 16),
-                                                           (33, 16, 1, 16)])
-def test_rc_nv_and_lanes_follow_R(R, want_rc, want_nv, want_lanes):
+@pytest.mark.parametrize("R,want_rc,want_nv,want_lanes,want_path", [
+    (1, 4, 2, 4, nat.PATH_STREAM), (3, 4, 2, 4, nat.PATH_STREAM), (5, 8, 1, 8, nat.PATH_STREAM),
+    (9, 16, 1, 16, nat.PATH_STREAM), (16, 16, 1, 16, nat.PATH_STREAM),
+    (17, 8, 1, 8, nat.PATH_WIDE), (33, 8, 1, 8, nat.PATH_WIDE), (100, 8, 1, 8, nat.PATH_WIDE)])
+def test_rc_nv_and_lanes_follow_R(R, want_rc, want_nv, want_lanes, want_path):
     rc, plan = q(R=R, D=64, B=64, H=64)      # 8 vectors per row, beyond one CTA
-    assert rc == 0 and (plan["rc"], plan["nv"], plan["lanes"]) == (want_rc, want_nv, want_lanes)
+    assert rc == 0 and (plan["rc"], plan["nv"], plan["lanes"], plan["path"]) == \
+        (want_rc, want_nv, want_lanes, want_path)
+
+
+@pytest.mark.parametrize("R,D,lanes,rc,slices,block", [
+    (64, 8, 4, 4, 1, 64), (64, 64, 8, 8, 1, 64), (64, 128, 16, 16, 1, 64), (64, 512, 32, 16, 2, 128),
+    (64, 1000, 32, 16, 4, 128), (32, 128, 16, 16, 1, 32), (17, 64, 8, 8, 1, 32),
+    (257, 512, 32, 16, 2, 128), (40, 128, 16, 16, 1, 64), (20, 128, 16, 16, 1, 32)])
+def test_wide_plan(R, D, lanes, rc, slices, block):
+    rc_, plan = q(R=R, D=D, B=3, H=5, path=nat.PATH_WIDE)
+    assert rc_ == 0
+    assert (plan["lanes"], plan["rc"], plan["slices_per_row"], plan["block"]) == (lanes, rc, slices, block)
+    assert plan["grid"] == plan["groups"] == 15 * slices
 
 
 def test_latency_path_keeps_one_column_per_lane():
@@ -150,8 +165,9 @@ def test_stream_only_below_its_size_limit():
     assert big["path"] == nat.PATH_VECTOR and big["grid"] > 0
     small = q(R=16, B=512, H=16, D=512, o=nat.F32)[1]
     assert small["path"] == nat.PATH_STREAM and small["grid"] == 0
-    # R > 16 needs several batches of partials per slice: VECTOR
-    assert q(R=17, B=64, H=64)[1]["path"] == nat.PATH_VECTOR
+    # R > 16: the partials of a row spread over one CTA (WIDE)
+    assert q(R=17, B=64, H=64)[1]["path"] == nat.PATH_WIDE
+    assert q(R=17, B=64, H=64, path=nat.PATH_VECTOR)[1]["path"] == nat.PATH_VECTOR
 
 
 @pytest.mark.parametrize("D,lanes,nv,slices", [(8, 4, 1, 1), (24, 4, 1, 1), (128, 8, 2, 1),

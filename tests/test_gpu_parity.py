@@ -34,7 +34,7 @@ def test_workload_full_size(name):
 
 @pytest.mark.parametrize("name", list(W))
 @pytest.mark.parametrize("path", [nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_LATENCY,
-                                  nat.PATH_STREAM])
+                                  nat.PATH_STREAM, nat.PATH_WIDE])
 def test_workload_every_path(name, path):
     w = W[name]
     # a reduced batch keeps the scalar path quick; the latency path is one CTA
@@ -46,7 +46,7 @@ def test_workload_every_path(name, path):
 
 def test_empty_shards_poisoned_with_nan():
     w = W["r4_b64_h32_d128_masked"]
-    for path in (nat.PATH_AUTO, nat.PATH_SCALAR, nat.PATH_VECTOR, nat.PATH_STREAM):
+    for path in (nat.PATH_AUTO, nat.PATH_SCALAR, nat.PATH_VECTOR, nat.PATH_STREAM, nat.PATH_WIDE):
         inp = synth.make_inputs(w, poison_empty=True)
         o = inp["o"]
         assert (((o & 0x7f80) == 0x7f80) & ((o & 0x7f) != 0)).any()   # bf16 NaNs are planted
@@ -59,19 +59,22 @@ def test_empty_shards_poisoned_with_nan():
 def test_dtype_pairs(in_dt, out_dt):
     base = W["r8_b1_h8_d128"]
     inp = synth.make_inputs(base, in_dtype=in_dt, out_dtype=out_dt, B=3, H=7, R=5, D=96)
-    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM):
+    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM, nat.PATH_WIDE):
         parity(inp, path=path, what=f"{in_dt}->{out_dt}/{path}")
 
 
-@pytest.mark.parametrize("R", [1, 2, 3, 5, 8, 9, 16, 17, 33, 40])
+@pytest.mark.parametrize("R", [1, 2, 3, 5, 8, 9, 16, 17, 33, 40, 64, 100, 257])
 @pytest.mark.parametrize("D", [4, 8, 24, 64, 100, 128, 256, 264, 512, 1024])
 def test_ragged_shapes(R, D):
     base = W["r2_b1_h2_d64"]
     inp = synth.make_inputs(base, R=R, D=D, B=3, H=5, lse_args=(-30.0, 30.0), seed=R * 1000 + D)
     parity(inp, what=f"R{R}/D{D}")
     parity(inp, path=nat.PATH_SCALAR, what=f"R{R}/D{D}/scalar")
-    if R <= 16 and D % 8 == 0:
-        parity(inp, path=nat.PATH_STREAM, what=f"R{R}/D{D}/stream")
+    if D % 8 == 0:
+        parity(inp, path=nat.PATH_VECTOR, what=f"R{R}/D{D}/vector")
+        parity(inp, path=nat.PATH_WIDE, what=f"R{R}/D{D}/wide")
+        if R <= 16:
+            parity(inp, path=nat.PATH_STREAM, what=f"R{R}/D{D}/stream")
 
 
 @pytest.mark.parametrize("layout", ["bhrd", "rbhd"])
@@ -103,7 +106,7 @@ def test_r1_is_identity_on_gpu():
 def test_all_rows_empty():
     inp = synth.make_inputs(W["r8_b256_h64_d128_rankmajor"], B=2, H=3)
     inp["lse"][:] = -np.inf
-    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM):
+    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM, nat.PATH_WIDE):
         got, got_lse, _ = run_gpu(inp, path)
         assert np.all(got == 0.0) and not np.signbit(got).any()
         assert np.all(got_lse == -np.inf)
@@ -159,7 +162,7 @@ def test_outputs_written_exactly_in_bounds():
     d_o = torch.from_numpy(inp["o"].view(np.int16)).cuda()
     d_l = torch.from_numpy(inp["lse"]).cuda()
     pad = 4096
-    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM):
+    for path in (nat.PATH_AUTO, nat.PATH_VECTOR, nat.PATH_SCALAR, nat.PATH_STREAM, nat.PATH_WIDE):
         canvas = torch.full((pad + B * H * D + pad,), 12345, dtype=torch.int16, device="cuda")
         lcanvas = torch.full((pad + B * H + pad,), 7.0, dtype=torch.float32, device="cuda")
         nat.merge_raw(d_o.data_ptr(), d_l.data_ptr(), R, B, H, D, (inp["o_strides"], inp["lse_strides"]),
@@ -261,3 +264,17 @@ def test_merge_host_pipelined(name, chunks):
     assert torch.equal(out_lse, dev_lse.cpu())
     want, want_lse = run_oracle(inp)
     check(out.double().numpy(), out_lse.double().numpy(), want, want_lse, inp["out_dtype"], name)
+
+
+@pytest.mark.parametrize("R,B,H,D", [(64, 1, 8, 128), (64, 64, 32, 128), (128, 4, 8, 512),
+                                     (48, 2, 3, 64)])
+def test_many_partials_wide_path(R, B, H, D):
+    """Large R (many KV splits): the AUTO (wide) path against the oracle, with
+    empty shards and an all-empty row among the inputs."""
+    w = W["r4_b64_h32_d128_masked"]
+    inp = synth.make_inputs(w, R=R, B=B, H=H, D=D, seed=R + B, poison_empty=True)
+    stats = parity(inp, what=f"wide R{R}")
+    rc, plan = nat.plan_query(0x7f0000000000, 0x7f1000000000, R, B, H, D,
+                              (inp["o_strides"], inp["lse_strides"]), nat.BF16, nat.BF16,
+                              0x7f2000000000, 0x7f3000000000)
+    assert plan["path"] == nat.PATH_WIDE
