@@ -123,11 +123,16 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
         const bool stream_ok = R <= rc;   // every partial of a row slice in one batch
         const i128 in_bytes = (i128)R * rows * D * ib;
         int chosen = path;
-        if (chosen == LSE_MERGE_PATH_AUTO)
-            chosen = small ? LSE_MERGE_PATH_LATENCY
-                           : !stream_ok ? LSE_MERGE_PATH_WIDE
-                           : (kAutoStream && in_bytes <= kStreamMaxBytes ? LSE_MERGE_PATH_STREAM
-                                                                         : LSE_MERGE_PATH_VECTOR);
+        if (chosen == LSE_MERGE_PATH_AUTO) {
+            if (small)
+                chosen = LSE_MERGE_PATH_LATENCY;
+            else if (!stream_ok || rows * slices1 <= kWideMaxSlices)
+                chosen = LSE_MERGE_PATH_WIDE;
+            else if (kAutoStream && in_bytes >= kStreamMinBytes && in_bytes <= kStreamMaxBytes)
+                chosen = LSE_MERGE_PATH_STREAM;
+            else
+                chosen = LSE_MERGE_PATH_VECTOR;
+        }
         if (chosen == LSE_MERGE_PATH_LATENCY && !small) return LSE_MERGE_EPATH;
         if (chosen == LSE_MERGE_PATH_STREAM && !stream_ok) return LSE_MERGE_EPATH;
         if (chosen == LSE_MERGE_PATH_WIDE) {

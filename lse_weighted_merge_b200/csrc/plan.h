@@ -28,10 +28,11 @@ constexpr int kMinBlocks = LSEM_MINB;
 #define LSEM_PDL 1
 #endif
 constexpr int kPdl = LSEM_PDL;
-// AUTO picks the persistent STREAM kernel for problems beyond one CTA whose
-// partials fit in kStreamMaxBytes, and the one-shot VECTOR kernel above that.
-// Measured on B200: STREAM is 4-6 % faster up to ~150 MB of partials, VECTOR
-// 3-6 % faster from ~300 MB on.
+// AUTO picks the persistent STREAM kernel for partials between
+// kStreamMinBytes and kStreamMaxBytes and the one-shot VECTOR kernel outside
+// that range.  Measured on B200: STREAM is 3-7 % faster from ~30 MB to
+// ~150 MB of partials; VECTOR is faster below one wave of work (2.1 MB:
+// 2.13 vs 2.36 us graph-replayed) and from ~300 MB on.
 #ifndef LSEM_AUTO_STREAM
 #define LSEM_AUTO_STREAM 1
 #endif
@@ -40,6 +41,11 @@ constexpr int kAutoStream = LSEM_AUTO_STREAM;
 #define LSEM_STREAM_MAX_MB 256
 #endif
 constexpr long long kStreamMaxBytes = (long long)LSEM_STREAM_MAX_MB << 20;
+constexpr long long kStreamMinBytes = 8ll << 20;
+// Row slices up to which AUTO spreads each row over a CTA (WIDE) even for
+// R <= 16: a handful of rows is latency-bound, and more threads per row beat
+// more loads per thread (8 rows of R=8: 2.03 us WIDE, 2.23 us VECTOR).
+constexpr long long kWideMaxSlices = 128;
 // Threads per CTA of the wide kernel (R > 16: one CTA per row slice).
 constexpr int kWideBlock = 128;
 // Upper bound on the 16-byte columns per lane (1, 2 or 4).

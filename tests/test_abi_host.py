@@ -91,8 +91,8 @@ def test_plans_of_the_five_workloads():
     blk = 64
     expect = {  # name -> (path, lanes, rc, nv, slices, block, grid); STREAM grids are sized at launch
         "r2_b1_h2_d64": (nat.PATH_LATENCY, 8, 4, 1, 1, 32, 1),
-        "r8_b1_h8_d128": (nat.PATH_STREAM, 8, 8, 2, 1, blk, 0),
-        "r4_b64_h32_d128_masked": (nat.PATH_STREAM, 8, 4, 2, 1, blk, 0),
+        "r8_b1_h8_d128": (nat.PATH_WIDE, 16, 4, 1, 1, 32, 8),
+        "r4_b64_h32_d128_masked": (nat.PATH_VECTOR, 8, 4, 2, 1, blk, 64 * 32 * 8 // blk),
         "r8_b256_h64_d128_rankmajor": (nat.PATH_STREAM, 8, 8, 2, 1, blk, 0),
         "r16_b512_h16_d512": (nat.PATH_STREAM, 32, 16, 1, 2, blk, 0),
     }
@@ -106,6 +106,8 @@ def test_plans_of_the_five_workloads():
         assert got == expect[name], (name, got)
         assert plan["vec"] == 8 and plan["rc"] * plan["nv"] <= 16
         assert plan["groups"] == w.B * w.H * plan["slices_per_row"]
+        if plan["path"] == nat.PATH_WIDE:
+            continue
         # every 16-byte column of a row is owned by exactly one lane slot
         dv = w.D // 8
         assert plan["slices_per_row"] * plan["lanes"] * plan["nv"] >= dv
@@ -133,11 +135,11 @@ def test_fallback_to_scalar_and_forced_paths():
 
 
 @pytest.mark.parametrize("R,want_rc,want_nv,want_lanes,want_path", [
-    (1, 4, 2, 4, nat.PATH_STREAM), (3, 4, 2, 4, nat.PATH_STREAM), (5, 8, 1, 8, nat.PATH_STREAM),
-    (9, 16, 1, 16, nat.PATH_STREAM), (16, 16, 1, 16, nat.PATH_STREAM),
+    (1, 4, 2, 4, nat.PATH_VECTOR), (3, 4, 2, 4, nat.PATH_VECTOR), (5, 8, 1, 8, nat.PATH_VECTOR),
+    (9, 16, 1, 16, nat.PATH_VECTOR), (16, 16, 1, 16, nat.PATH_STREAM),   # 16 x 0.5 MB = 8 MB
     (17, 8, 1, 8, nat.PATH_WIDE), (33, 8, 1, 8, nat.PATH_WIDE), (100, 8, 1, 8, nat.PATH_WIDE)])
 def test_rc_nv_and_lanes_follow_R(R, want_rc, want_nv, want_lanes, want_path):
-    rc, plan = q(R=R, D=64, B=64, H=64)      # 8 vectors per row, beyond one CTA
+    rc, plan = q(R=R, D=64, B=64, H=64)      # 8 vectors per row, beyond one CTA, < 8 MB
     assert rc == 0 and (plan["rc"], plan["nv"], plan["lanes"], plan["path"]) == \
         (want_rc, want_nv, want_lanes, want_path)
 
@@ -157,6 +159,15 @@ def test_latency_path_keeps_one_column_per_lane():
     rc, plan = q(R=2, D=64, B=1, H=2)
     assert plan["path"] == nat.PATH_LATENCY and plan["nv"] == 1 and plan["lanes"] == 8
     assert plan["block"] == 32 and plan["grid"] == 1
+
+
+def test_path_choice_by_size():
+    # a few rows: each spread over a CTA
+    assert q(R=8, B=2, H=8, D=128)[1]["path"] == nat.PATH_WIDE
+    # under one wave of work (< 8 MB of partials): one-shot VECTOR
+    assert q(R=4, B=64, H=32, D=128)[1]["path"] == nat.PATH_VECTOR
+    # 8 MB .. 256 MB: persistent STREAM
+    assert q(R=8, B=64, H=64, D=128, o=nat.F32)[1]["path"] == nat.PATH_STREAM
 
 
 def test_stream_only_below_its_size_limit():
