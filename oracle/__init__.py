@@ -55,6 +55,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
         ctypes.c_int64, ctypes.c_int64, dp, dp]
+    lib.oracle_cp_exchange_merge.restype = ctypes.c_int
+    lib.oracle_cp_exchange_merge.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, dp, dp]
     return lib
 
 
@@ -149,4 +153,34 @@ def state_update(acc: np.ndarray, lse_acc: np.ndarray, acc_dtype: int, new: np.n
                                  out.ctypes.data_as(dp), out_lse.ctypes.data_as(dp))
     if rc != 0:
         raise ValueError(f"oracle_state_update returned {rc}")
+    return out, out_lse
+
+
+def cp_exchange_merge(local_o: np.ndarray, local_lse: np.ndarray, world: int, B: int, H: int,
+                      D: int, in_dtype: int, lib: ctypes.CDLL | None = None):
+    """Exchange heads between ``world`` ranks, then merge (fp64).
+
+    local_o: flat [world, B, H, D] raw elements (uint16 bits or float32), rank
+    s's partials in block s; local_lse: [world, B, H] float32.  Rank q owns
+    heads [q*H/world, (q+1)*H/world).  Returns (out [world, B, H/world, D],
+    out_lse [world, B, H/world]) float64, block q being rank q's result.
+    """
+    lib = lib or load()
+    po = np.ascontiguousarray(local_o)
+    pl = np.ascontiguousarray(local_lse, dtype=np.float32)
+    want = np.float32 if in_dtype == F32 else np.uint16
+    if po.dtype != want:
+        raise TypeError(f"local_o must be {np.dtype(want).name} for dtype {in_dtype}")
+    if po.size != world * B * H * D or pl.size != world * B * H:
+        raise ValueError("local_o / local_lse sizes do not match world, B, H, D")
+    if H % world:
+        raise ValueError("H must be a multiple of world")
+    Hq = H // world
+    out = np.empty((world, B, Hq, D), dtype=np.float64)
+    out_lse = np.empty((world, B, Hq), dtype=np.float64)
+    dp = ctypes.POINTER(ctypes.c_double)
+    rc = lib.oracle_cp_exchange_merge(po.ctypes.data, pl.ctypes.data, world, B, H, D, in_dtype,
+                                      out.ctypes.data_as(dp), out_lse.ctypes.data_as(dp))
+    if rc != 0:
+        raise ValueError(f"oracle_cp_exchange_merge returned {rc}")
     return out, out_lse

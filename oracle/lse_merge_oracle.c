@@ -280,3 +280,43 @@ int oracle_state_update(const void* acc, const float* lse_acc, int acc_dtype,
     }
     return 0;
 }
+
+/*
+ * Context-parallel exchange followed by the merge (page "[flashinfer]
+ * FlashInfer의 Context-Parallel Decode 최적화: Fused A2A + LSE Reduce",
+ * sections "들어가며" and "코드 분석 / 1. Fused Kernel 구현": every rank holds
+ * the partials of its KV shard for all heads; the exchange hands each head to
+ * the rank that owns it, which then merges the partials of all ranks).
+ * Reading: heads are scattered in equal contiguous blocks, rank q owning heads
+ * [q*H/world, (q+1)*H/world).  So rank q's output row (b, j) is the merge over
+ * ranks s of rank s's partial at (b, q*H/world + j):
+ *     out[q][b][j] = merge_s (local_o[s][b][q*Hq + j], local_lse[s][b][q*Hq + j])
+ * local_o     [world, B, H, D] elements of in_dtype, contiguous
+ * local_lse   [world, B, H] float, contiguous
+ * out_o       double [world, B, H/world, D];  out_lse  double [world, B, H/world]
+ * Returns 0, -1 for an unknown dtype, -2 for a bad size (H % world != 0).
+ */
+int oracle_cp_exchange_merge(const void* local_o, const float* local_lse, int world,
+                             int B, int H, int D, int in_dtype,
+                             double* out_o, double* out_lse) {
+    if (in_dtype != ORACLE_F32 && in_dtype != ORACLE_F16 && in_dtype != ORACLE_BF16)
+        return -1;
+    if (world < 1 || B < 1 || H < 1 || D < 1 || H % world != 0) return -2;
+    const int Hq = H / world;
+    const int64_t esize = in_dtype == ORACLE_F32 ? 4 : 2;
+    const int64_t os[3] = {(int64_t)B * H * D, (int64_t)H * D, D};
+    const int64_t ls[3] = {(int64_t)B * H, H, 1};
+    for (int q = 0; q < world; ++q) {
+#if ORACLE_MUTANT == 8
+        const int64_t h0 = 0;                           /* planted mistake: owner's head offset dropped */
+#else
+        const int64_t h0 = (int64_t)q * Hq;             /* first head rank q owns */
+#endif
+        const char* o = (const char*)local_o + h0 * D * esize;
+        const float* l = local_lse + h0;
+        int rc = oracle_lse_merge(o, l, world, B, Hq, D, os, ls, in_dtype,
+                                  out_o + (int64_t)q * B * Hq * D, out_lse + (int64_t)q * B * Hq);
+        if (rc != 0) return rc;
+    }
+    return 0;
+}

@@ -28,6 +28,8 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
                       "merge_hand_cases.json")
 GOLDEN_STATE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
                             "state_update_hand_cases.json")
+GOLDEN_CP = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                         "cp_exchange_hand_cases.json")
 
 
 def _num(x):
@@ -355,10 +357,63 @@ def pin_state_chain_is_the_merge(lib):
     assert np.array_equal(alt, one) and np.array_equal(alt_lse, one_lse)
 
 
+def _nums(a):
+    return np.vectorize(_num, otypes=[np.float64])(np.array(a, dtype=object))
+
+
+def pin_cp_golden(lib):
+    """Hand-derived exchange + merge results (head ownership by rank)."""
+    with open(GOLDEN_CP) as fh:
+        cases = json.load(fh)["cases"]
+    for c in cases:
+        world, B, H, D = c["world"], c["B"], c["H"], c["D"]
+        o = synth.pack(_nums(c["o"]).astype(np.float32).ravel(), c["dtype"])
+        lse = _nums(c["lse"]).astype(np.float32).ravel()
+        out, out_lse = oracle.cp_exchange_merge(o, lse, world, B, H, D, synth.DTYPES[c["dtype"]],
+                                                lib=lib)
+        want, want_lse = _nums(c["out"]), _nums(c["out_lse"])
+        assert not np.isnan(out).any(), c["name"]
+        assert np.all(np.abs(out - want) <= c["tol"]), (c["name"], out, want)
+        fin = np.isfinite(want_lse)
+        assert np.array_equal(np.isneginf(out_lse), np.isneginf(want_lse)), c["name"]
+        assert np.all(np.abs(out_lse[fin] - want_lse[fin]) <= c["tol"]), (c["name"], out_lse)
+
+
+def pin_cp_partitions_the_merge(lib):
+    """The ranks' outputs, laid side by side along the head axis, are the
+    world-way merge of all heads (each head merged once, by its owner); with
+    one rank the exchange is the identity merge of that rank's partials; and
+    reordering the senders changes no output."""
+    rng = np.random.Generator(np.random.PCG64(33))
+    for world, B, H, D, dt in ((4, 3, 8, 5, "bf16"), (2, 2, 6, 3, "f32"), (8, 1, 8, 4, "f16")):
+        o = rng.standard_normal((world, B, H, D)).astype(np.float32)
+        lse = rng.uniform(-6, 6, (world, B, H)).astype(np.float32)
+        lse[world - 1, 0, H - 1] = -np.inf
+        packed = synth.pack(o.ravel(), dt)
+        out, out_lse = oracle.cp_exchange_merge(packed, lse, world, B, H, D, synth.DTYPES[dt],
+                                                lib=lib)
+        Hq = H // world
+        full, full_lse = oracle.merge(packed, lse, world, B, H, D, (B * H * D, H * D, D),
+                                      (B * H, H, 1), synth.DTYPES[dt], lib=lib)
+        side = np.concatenate([out[q] for q in range(world)], axis=1)       # [B, H, D]
+        side_lse = np.concatenate([out_lse[q] for q in range(world)], axis=1)
+        assert np.array_equal(side, full) and np.array_equal(side_lse, full_lse), (world, dt)
+        perm = rng.permutation(world)
+        po = synth.pack(o[perm].ravel(), dt)
+        pout, pout_lse = oracle.cp_exchange_merge(po, lse[perm], world, B, H, D,
+                                                  synth.DTYPES[dt], lib=lib)
+        assert np.allclose(pout, out, rtol=0, atol=1e-12) and np.allclose(pout_lse, out_lse,
+                                                                          rtol=0, atol=1e-12)
+        one, one_lse = oracle.cp_exchange_merge(synth.pack(o[0].ravel(), dt), lse[0], 1, B, H, D,
+                                                synth.DTYPES[dt], lib=lib)
+        assert np.array_equal(one[0], widened(o[0], dt))
+        assert np.array_equal(one_lse[0], lse[0].astype(np.float64))
+
+
 ALL_PINS = [
     pin_decoders, pin_golden, pin_r1_identity, pin_equal_lse_mean,
     pin_empty_shards_drop_out, pin_shift_invariance, pin_permutation_invariance,
     pin_associativity, pin_attention_shard, pin_split_attention_identity,
     pin_layout_and_row_independence, pin_extreme_spread, pin_state_golden,
-    pin_state_chain_is_the_merge,
+    pin_state_chain_is_the_merge, pin_cp_golden, pin_cp_partitions_the_merge,
 ]

@@ -21,6 +21,7 @@ MUTANTS = {
     5: "plain mean instead of lse weights",
     6: "first shard dropped",
     7: "state update with its two weights swapped",
+    8: "exchange: owner's head offset dropped",
 }
 
 CHILD = r"""
