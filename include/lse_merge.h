@@ -24,7 +24,8 @@
  * Everything runs on the GPU inside one kernel launch per call; the library
  * allocates nothing, keeps no pointer after returning, never synchronises
  * the host, and only enqueues work on `stream`, so a call can be captured in
- * a CUDA graph.
+ * a CUDA graph.  The exceptions are the set-up calls of the context-parallel
+ * exchange (lse_merge_cp_workspace_create and the IPC calls), which say so.
  */
 #ifndef LSE_MERGE_H
 #define LSE_MERGE_H
@@ -68,6 +69,7 @@ typedef struct {
 #define LSE_MERGE_EALIGN (-7)   /* a pointer not aligned to its element size */
 #define LSE_MERGE_EPATH (-8)    /* the requested path cannot take these arguments */
 #define LSE_MERGE_EUNSUP (-9)   /* a shape the decode-attention kernels do not implement */
+#define LSE_MERGE_ECUDA (-10)   /* a CUDA runtime call of a set-up function failed */
 
 /* Kernel paths.  AUTO picks one from the sizes, dtypes and alignment. */
 #define LSE_MERGE_PATH_AUTO 0
@@ -226,6 +228,99 @@ int lse_merge_decode_attention(const void* q, const void* k, const void* v, cons
                                const lse_merge_attn_strides* strides, int dtype, int out_dtype,
                                void* out_o, float* out_lse, lse_merge_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Context-parallel exchange and merge in one kernel.
+ *
+ * The step before the merge on the CP-decode page (section "코드 분석 / 1.
+ * Fused Kernel 구현": instead of an all-to-all followed by a separate merge,
+ * each rank writes its partials straight into the buffer of the rank that
+ * owns them, and the owner merges once everything has landed; the
+ * introduction, "들어가며", gives the partials themselves).  `world` ranks
+ * each hold the partials of their own KV shard for all B*H rows:
+ *   local_o [B,H,D] of in_dtype, dense;  local_lse [B,H] fp32, dense.
+ * Heads are scattered in equal contiguous blocks: rank q owns heads
+ * [q*Hq, (q+1)*Hq) with Hq = H / world, and produces
+ *   out_o [B,Hq,D] of out_dtype, dense;  out_lse [B,Hq] fp32, dense,
+ * the merge over all ranks' partials of its heads.  One launch, per rank:
+ *   1. every (b, h) row owned by another rank q is stored into q's workspace
+ *      (plain 16-byte stores; ws[q] may be a peer GPU's memory);
+ *   2. the rank adds the number of 16-byte units it stored for q to q's
+ *      landed counter for this sender (system-scope release);
+ *   3. it waits, bounded by timeout_ns of the GPU's global timer, until every
+ *      other rank's landed counter in its own workspace reached e * U, e the
+ *      number of this call since the workspace was zeroed (U = B*Hq*D*elem/16
+ *      units per sender);
+ *   4. it merges its rows: its own partial read in place from local_o, the
+ *      others from its workspace;
+ *   5. its last CTA to finish records call e as completed in the workspace.
+ * The call number lives in the workspace, so every rank must make the same
+ * calls since the workspaces were zeroed, each rank's calls ordered on one
+ * stream; a captured CUDA graph may replay a call.  Received rows alternate
+ * between two slots by the parity of e, so a rank may start call e + 1 while
+ * a peer still merges call e.  A wait that runs out ORs bit s (sender s) into
+ * the uint32 status word at byte LSE_MERGE_CP_STATUS_OFFSET of that rank's
+ * workspace, leaves that rank's outputs unwritten and returns; the
+ * workspaces are then out of step, and every rank must zero its workspace
+ * (lse_merge_cp_workspace_zero) before the next call.
+ *
+ * One launch may play several ranks: ranks rank_begin .. rank_begin +
+ * rank_count - 1 (local_o[i], local_lse[i], out_o[i], out_lse[i] belong to
+ * rank rank_begin + i).  All CTAs of a launch are co-resident (cooperative
+ * launch), so a single GPU can play all `world` ranks at once; in a multi-GPU
+ * job each process plays its own rank (rank_count = 1) and ws[] holds the
+ * peers' workspaces (lse_merge_cp_ipc_open).
+ *
+ * Requirements: 1 <= world <= LSE_MERGE_CP_MAX_WORLD; H % world == 0;
+ * D * elem(in_dtype) a multiple of 16 bytes; 0 <= rank_begin and
+ * rank_begin + rank_count <= world; local_o and out_o 16-byte aligned, lse
+ * pointers 4-byte aligned, workspaces 256-byte aligned and
+ * lse_merge_cp_workspace_bytes() long (zeroed before the first call);
+ * 0 < timeout_ns <= 60 s.  Outputs may not overlap inputs or workspaces.  The
+ * library keeps no pointer.  Returns the codes of lse_merge (EDIMS for the
+ * requirements on world, H, the ranks and the timeout, EALIGN for D and the
+ * pointers) and LSE_MERGE_ELAUNCH when the launch fails, e.g. a grid that
+ * cannot be co-resident.
+ */
+#define LSE_MERGE_CP_MAX_WORLD 8
+#define LSE_MERGE_CP_STATUS_OFFSET 64     /* uint32 in each workspace; 0 = no wait ran out */
+#define LSE_MERGE_CP_IPC_HANDLE_BYTES 64
+
+typedef struct {
+    int world, rank_begin, rank_count;
+    const void* local_o[LSE_MERGE_CP_MAX_WORLD];    /* per played rank */
+    const float* local_lse[LSE_MERGE_CP_MAX_WORLD];
+    void* out_o[LSE_MERGE_CP_MAX_WORLD];            /* per played rank */
+    float* out_lse[LSE_MERGE_CP_MAX_WORLD];
+    void* ws[LSE_MERGE_CP_MAX_WORLD];               /* workspace of every rank q < world */
+    int B, H, D, in_dtype, out_dtype;
+    int64_t timeout_ns;
+} lse_merge_cp_args;
+
+/* Bytes of one rank's workspace (the same on every rank). */
+int lse_merge_cp_workspace_bytes(int world, int B, int H, int D, int in_dtype, int64_t* bytes);
+/* Check the arguments as lse_merge_cp_exchange_merge does, without a GPU. */
+int lse_merge_cp_validate(const lse_merge_cp_args* args);
+int lse_merge_cp_exchange_merge(const lse_merge_cp_args* args, lse_merge_stream_t stream);
+
+/* Workspaces shared between processes (one GPU per process).  create:
+ * cudaMalloc of `bytes` on the current device, zeroed before it returns.
+ * ipc_handle: the cudaIpcMemHandle_t of a created workspace, copied into
+ * `handle` (LSE_MERGE_CP_IPC_HANDLE_BYTES bytes).  ipc_open: maps a peer's
+ * workspace into this process (peer access enabled), *peer_ws its address;
+ * ipc_close unmaps it.  These are set-up calls: they synchronise the device,
+ * and create is the one place the library allocates.  They return
+ * LSE_MERGE_ECUDA when the CUDA call fails (lse_merge_last_cuda_error). */
+int lse_merge_cp_workspace_create(int64_t bytes, void** ws);
+/* The status word of a workspace (a synchronous copy; 0 = no wait ran out,
+ * bit s = sender s never landed) and the restart after a wait ran out:
+ * zero `bytes` of the workspace, synchronously. */
+int lse_merge_cp_status(const void* ws, uint32_t* status);
+int lse_merge_cp_workspace_zero(void* ws, int64_t bytes);
+int lse_merge_cp_workspace_destroy(void* ws);
+int lse_merge_cp_ipc_handle(void* ws, void* handle);
+int lse_merge_cp_ipc_open(const void* handle, void** peer_ws);
+int lse_merge_cp_ipc_close(void* peer_ws);
+
 /* A static, human-readable description of a return code. */
 const char* lse_merge_strerror(int code);
 
@@ -235,7 +330,7 @@ int lse_merge_last_cuda_error(void);
 /* ABI version of this header; bumped on any incompatible change. */
 int lse_merge_version(void);
 
-#define LSE_MERGE_ABI_VERSION 2
+#define LSE_MERGE_ABI_VERSION 3
 
 #ifdef __cplusplus
 }

@@ -17,14 +17,20 @@ PATH_AUTO, PATH_VECTOR, PATH_LATENCY, PATH_SCALAR, PATH_STREAM, PATH_WIDE = 0, 1
 PATH_NAMES = {PATH_VECTOR: "vector", PATH_LATENCY: "latency", PATH_SCALAR: "scalar",
               PATH_STREAM: "stream", PATH_WIDE: "wide"}
 
-OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH, EUNSUP = (
-    0, -1, -2, -3, -4, -5, -6, -7, -8, -9)
+OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH, EUNSUP, ECUDA = (
+    0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10)
+CP_MAX_WORLD = 8
+CP_STATUS_OFFSET = 64
+CP_IPC_HANDLE_BYTES = 64
 
 # Every symbol include/lse_merge.h declares.
 EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merge_state_update",
            "lse_merge_decode_partials", "lse_merge_decode_attention", "lse_merge_strerror",
-           "lse_merge_last_cuda_error", "lse_merge_version")
-ABI_VERSION = 2
+           "lse_merge_last_cuda_error", "lse_merge_version", "lse_merge_cp_workspace_bytes",
+           "lse_merge_cp_validate", "lse_merge_cp_exchange_merge", "lse_merge_cp_workspace_create",
+           "lse_merge_cp_workspace_destroy", "lse_merge_cp_ipc_handle", "lse_merge_cp_ipc_open",
+           "lse_merge_cp_ipc_close", "lse_merge_cp_status", "lse_merge_cp_workspace_zero")
+ABI_VERSION = 3
 
 
 class Strides(ctypes.Structure):
@@ -51,6 +57,32 @@ class Plan(ctypes.Structure):
         d = {f: getattr(self, f) for f, _ in self._fields_}
         d["path_name"] = PATH_NAMES.get(self.path, "?")
         return d
+
+
+_P8 = ctypes.c_void_p * CP_MAX_WORLD
+
+
+class CpArgs(ctypes.Structure):
+    _fields_ = [("world", ctypes.c_int), ("rank_begin", ctypes.c_int), ("rank_count", ctypes.c_int),
+                ("local_o", _P8), ("local_lse", _P8), ("out_o", _P8), ("out_lse", _P8),
+                ("ws", _P8), ("B", ctypes.c_int), ("H", ctypes.c_int),
+                ("D", ctypes.c_int), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+                ("timeout_ns", ctypes.c_int64)]
+
+
+def cp_args(world: int, rank_begin: int, local_o, local_lse, out_o, out_lse, ws,
+            B: int, H: int, D: int, in_dtype: int, out_dtype: int, timeout_ns: int) -> CpArgs:
+    """Fill lse_merge_cp_args from lists of raw pointers (one per played rank / per rank)."""
+    def arr(ptrs):
+        if len(ptrs) > CP_MAX_WORLD:
+            raise ValueError(f"at most {CP_MAX_WORLD} ranks, got {len(ptrs)} pointers")
+        a = _P8()
+        for i, x in enumerate(ptrs):
+            a[i] = int(x) if x else None
+        return a
+    return CpArgs(int(world), int(rank_begin), len(local_o), arr(local_o), arr(local_lse),
+                  arr(out_o), arr(out_lse), arr(ws), int(B), int(H), int(D),
+                  int(in_dtype), int(out_dtype), int(timeout_ns))
 
 
 class LseMergeError(RuntimeError):
@@ -88,6 +120,26 @@ def _load() -> ctypes.CDLL:
     lib.lse_merge_last_cuda_error.restype = i
     lib.lse_merge_version.argtypes = []
     lib.lse_merge_version.restype = i
+    lib.lse_merge_cp_workspace_bytes.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_int64)]
+    lib.lse_merge_cp_workspace_bytes.restype = i
+    lib.lse_merge_cp_validate.argtypes = [ctypes.POINTER(CpArgs)]
+    lib.lse_merge_cp_validate.restype = i
+    lib.lse_merge_cp_exchange_merge.argtypes = [ctypes.POINTER(CpArgs), vp]
+    lib.lse_merge_cp_exchange_merge.restype = i
+    lib.lse_merge_cp_workspace_create.argtypes = [ctypes.c_int64, ctypes.POINTER(vp)]
+    lib.lse_merge_cp_workspace_create.restype = i
+    lib.lse_merge_cp_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.lse_merge_cp_status.restype = i
+    lib.lse_merge_cp_workspace_zero.argtypes = [vp, ctypes.c_int64]
+    lib.lse_merge_cp_workspace_zero.restype = i
+    lib.lse_merge_cp_workspace_destroy.argtypes = [vp]
+    lib.lse_merge_cp_workspace_destroy.restype = i
+    lib.lse_merge_cp_ipc_handle.argtypes = [vp, vp]
+    lib.lse_merge_cp_ipc_handle.restype = i
+    lib.lse_merge_cp_ipc_open.argtypes = [vp, ctypes.POINTER(vp)]
+    lib.lse_merge_cp_ipc_open.restype = i
+    lib.lse_merge_cp_ipc_close.argtypes = [vp]
+    lib.lse_merge_cp_ipc_close.restype = i
     if lib.lse_merge_version() != ABI_VERSION:
         raise ImportError(f"{LIB_PATH}: ABI version {lib.lse_merge_version()} != {ABI_VERSION}")
     return lib
@@ -171,3 +223,84 @@ def decode_raw(q_ptr: int, k_ptr: int, v_ptr: int, kv_len_ptr: int, B: int, Hq: 
     else:
         rc = lib.lse_merge_decode_partials(*args, out_ptr, out_lse_ptr, stream or None)
     return _check(rc, check)
+
+
+def _raise(rc: int):
+    extra = ""
+    if rc in (ELAUNCH, ECUDA):
+        extra = f" (cudaError {lib.lse_merge_last_cuda_error()})"
+    raise LseMergeError(rc, strerror(rc) + extra)
+
+
+def cp_workspace_bytes(world: int, B: int, H: int, D: int, in_dtype: int) -> int:
+    n = ctypes.c_int64(0)
+    rc = lib.lse_merge_cp_workspace_bytes(world, B, H, D, in_dtype, ctypes.byref(n))
+    if rc != OK:
+        _raise(rc)
+    return n.value
+
+
+def cp_validate(args: CpArgs) -> int:
+    """Host-only: the code lse_merge_cp_exchange_merge would return for ``args``
+    before launching (OK when it would launch)."""
+    return lib.lse_merge_cp_validate(ctypes.byref(args))
+
+
+def cp_exchange_merge_raw(args: CpArgs, stream: int = 0, check: bool = True) -> int:
+    rc = lib.lse_merge_cp_exchange_merge(ctypes.byref(args), stream or None)
+    if check and rc != OK:
+        _raise(rc)
+    return rc
+
+
+def cp_workspace_create(nbytes: int) -> int:
+    p = ctypes.c_void_p()
+    rc = lib.lse_merge_cp_workspace_create(int(nbytes), ctypes.byref(p))
+    if rc != OK:
+        _raise(rc)
+    return p.value
+
+
+def cp_status(ptr: int) -> int:
+    st = ctypes.c_uint32(0)
+    rc = lib.lse_merge_cp_status(ptr, ctypes.byref(st))
+    if rc != OK:
+        _raise(rc)
+    return st.value
+
+
+def cp_workspace_zero(ptr: int, nbytes: int) -> None:
+    rc = lib.lse_merge_cp_workspace_zero(ptr, int(nbytes))
+    if rc != OK:
+        _raise(rc)
+
+
+def cp_workspace_destroy(ptr: int) -> None:
+    rc = lib.lse_merge_cp_workspace_destroy(ptr)
+    if rc != OK:
+        _raise(rc)
+
+
+def cp_ipc_handle(ptr: int) -> bytes:
+    buf = ctypes.create_string_buffer(CP_IPC_HANDLE_BYTES)
+    rc = lib.lse_merge_cp_ipc_handle(ptr, buf)
+    if rc != OK:
+        _raise(rc)
+    return buf.raw
+
+
+def cp_ipc_open(handle: bytes) -> int:
+    if len(handle) != CP_IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {CP_IPC_HANDLE_BYTES} bytes, got {len(handle)}")
+    buf = ctypes.create_string_buffer(bytes(handle), CP_IPC_HANDLE_BYTES)
+    p = ctypes.c_void_p()
+    rc = lib.lse_merge_cp_ipc_open(buf, ctypes.byref(p))
+    if rc != OK:
+        _raise(rc)
+    return p.value
+
+
+def cp_ipc_close(ptr: int) -> None:
+    rc = lib.lse_merge_cp_ipc_close(ptr)
+    if rc != OK:
+        _raise(rc)

@@ -14,8 +14,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblse_merge.so")
 SOURCES = [os.path.join(CSRC, "plan.cpp"), os.path.join(CSRC, "lse_merge.cu"),
-           os.path.join(CSRC, "decode_attention.cu")]
-HEADERS = [os.path.join(INCLUDE, "lse_merge.h"), os.path.join(CSRC, "plan.h")]
+           os.path.join(CSRC, "decode_attention.cu"), os.path.join(CSRC, "cp_exchange.cu")]
+HEADERS = [os.path.join(INCLUDE, "lse_merge.h"), os.path.join(CSRC, "plan.h"),
+           os.path.join(CSRC, "device_common.cuh")]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",

@@ -1,0 +1,481 @@
+// cp_exchange.cu -- context-parallel exchange and merge in one kernel (sm_100a).
+//
+// Under context-parallel decode every rank holds the partials (o, lse) of its
+// own KV shard for all heads; the heads are then scattered so that each rank
+// merges the partials of the heads it owns (page "[flashinfer] FlashInfer의
+// Context-Parallel Decode 최적화: Fused A2A + LSE Reduce", section "들어가며"
+// for the partials; section "코드 분석 / 1. Fused Kernel 구현" for the fused
+// design in which the ranks write straight into the owner's buffer over
+// NVLink and the owner merges once everything has landed).
+//
+// One launch, per rank `me` (blockIdx.y picks the rank among those the launch
+// plays; blockIdx.x is the CTA within the rank):
+//   1. send: the rank's partial rows of heads owned by rank q != me are
+//      copied, 16 bytes per thread and step, into q's workspace (the slot of
+//      sender me, parity e & 1).  Each CTA owns a contiguous range of the
+//      (q, b, head, 16-byte column) units, so consecutive threads write
+//      consecutive addresses of one receiver;
+//   2. land: after a CTA barrier, one thread makes the CTA's stores visible
+//      system-wide and adds the number of units the CTA sent to q to q's
+//      landed counter of sender me.  The count does not depend on how many
+//      CTAs the sender used, so ranks may launch different grids;
+//   3. wait: one thread per CTA polls the landed counters in me's workspace
+//      (acquire, system scope) until every sender reached e * U units (e: the
+//      number of this call, kept in the workspace header),
+//      bounded by the GPU global timer and by a poll count.  A wait that runs
+//      out sets the sender's bit in me's status word and the CTA returns
+//      without writing its outputs;
+//   4. merge: each thread merges one 16-byte column of one owned row over all
+//      senders: its own partial read in place from local_o, the others from
+//      the workspace (L2-only loads, since other SMs or GPUs wrote them during
+//      this launch), fp32 accumulation, one reciprocal, conversion;
+//   5. the rank's last CTA to finish advances the rank's call count, so the
+//      next call (or the next replay of a captured graph) is call e + 1.
+// All CTAs of the launch are co-resident (cooperative launch), so a CTA that
+// waits never keeps a sending CTA of the same launch from running.
+//
+// The peer traffic is plain 16-byte stores and one atomic add per CTA and
+// receiver; no load reads another GPU's memory.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "device_common.cuh"
+#include "lse_merge.h"
+#include "plan.h"
+
+namespace lsem {
+namespace {
+
+constexpr int kMaxWorld = LSE_MERGE_CP_MAX_WORLD;
+constexpr int kSendUnroll = 4;   // 16-byte units in flight per thread while sending
+
+struct CpParams {
+    const char* local_o[kMaxWorld];   // per played rank, dense [B, H, D]
+    const float* local_lse[kMaxWorld];
+    char* out_o[kMaxWorld];           // per played rank, dense [B, Hq, D]
+    float* out_lse[kMaxWorld];
+    char* ws[kMaxWorld];              // every rank's workspace
+    int world, rank_begin, H, Hq;
+    uint32_t dv;                      // 16-byte units per row
+    int64_t U;                        // units per (sender, receiver) pair
+    int64_t rowbytes;                 // D * in_bytes
+    int64_t slot_o, slot_l, o_off, l_off;
+    int64_t chunk;                    // send units per CTA
+    int64_t timeout_ns, max_polls;
+    int idx32;                        // all unit indices fit in 32 bits
+    uint64_t c_U, c_dv, c_Hq;         // fastdiv constants (idx32 only)
+};
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_sys(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Loads of data written during this launch by other SMs or GPUs: cached in
+// L2 only (L1 is not coherent), 256-byte L2 prefetch for the row's neighbours.
+__device__ __forceinline__ uint4 ld_cg16(const char* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ float ld_cg_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// n / d and n % d, through the 32-bit constant division when idx32.
+__device__ __forceinline__ void divmod(const CpParams& p, int64_t n, uint64_t c, int64_t d,
+                                       int64_t& q, int64_t& r) {
+    if (p.idx32) {
+        const uint32_t qq = fastdiv((uint32_t)n, c, (uint32_t)d);
+        q = qq;
+        r = (int64_t)((uint32_t)n - qq * (uint32_t)d);
+    } else {
+        q = n / d;
+        r = n - q * d;
+    }
+}
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kCpBlock) cp_exchange_merge_kernel(const __grid_constant__ CpParams p) {
+    constexpr int N = Elem<TIn>::kVec;
+    constexpr int N2 = N / 2;
+    const int pr = blockIdx.y;
+    const int me = p.rank_begin + pr;
+    const int w1 = p.world - 1;
+    const int64_t cta = blockIdx.x;
+    const char* src_o = p.local_o[pr];
+    const float* src_l = p.local_lse[pr];
+    char* const mine = p.ws[me];
+    // This call's number e (1 for the first call after the workspace was
+    // zeroed), from the count of calls this rank has completed; the last CTA
+    // of the rank to finish advances the count, after every CTA read it.
+    const unsigned long long e =
+        *reinterpret_cast<volatile const unsigned long long*>(mine + kCpEpochOffset) + 1;
+    const int par = (int)(e & 1);   // receive slot of this call
+
+    // ---- 1. send the rows other ranks own
+    const int64_t total = (int64_t)w1 * p.U;
+    const int64_t u0 = min(total, cta * p.chunk);
+    const int64_t u1 = min(total, u0 + p.chunk);
+    for (int64_t u = u0 + threadIdx.x; u < u1; u += (int64_t)kCpBlock * kSendUnroll) {
+        uint4 x[kSendUnroll];
+        char* dst[kSendUnroll];
+        float lv[kSendUnroll];
+        float* ldst[kSendUnroll];
+#pragma unroll
+        for (int k = 0; k < kSendUnroll; ++k) {
+            const int64_t uk = u + (int64_t)k * kCpBlock;
+            dst[k] = nullptr;
+            ldst[k] = nullptr;
+            lv[k] = 0.f;
+            x[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (uk < u1) {
+                int64_t qi, rem, row, v, b, hq;
+                divmod(p, uk, p.c_U, p.U, qi, rem);
+                divmod(p, rem, p.c_dv, p.dv, row, v);
+                divmod(p, row, p.c_Hq, p.Hq, b, hq);
+                const int q = (int)qi + ((int)qi >= me ? 1 : 0);   // receiver
+                const int slot = me - (me > q ? 1 : 0);            // sender slot at q
+                const int64_t srow = b * p.H + (int64_t)q * p.Hq + hq;
+                x[k] = ld_stream16(src_o + srow * p.rowbytes + v * 16);
+                const int64_t blk = (int64_t)par * w1 + slot;
+                dst[k] = p.ws[q] + p.o_off + blk * p.slot_o + rem * 16;
+                if (v == 0) {
+                    lv[k] = __ldg(src_l + srow);
+                    ldst[k] = reinterpret_cast<float*>(p.ws[q] + p.l_off + blk * p.slot_l) + row;
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kSendUnroll; ++k) {
+            if (dst[k]) *reinterpret_cast<uint4*>(dst[k]) = x[k];
+            if (ldst[k]) *ldst[k] = lv[k];
+        }
+    }
+
+    // ---- 2. land: publish this CTA's units to each receiver
+    __syncthreads();
+    if (threadIdx.x == 0 && u1 > u0) {
+        __threadfence_system();
+        for (int qi = 0; qi < w1; ++qi) {
+            const int64_t lo = max(u0, (int64_t)qi * p.U), hi = min(u1, (int64_t)(qi + 1) * p.U);
+            if (hi > lo) {
+                const int q = qi + (qi >= me ? 1 : 0);
+                atomicAdd_system(reinterpret_cast<unsigned long long*>(p.ws[q]) + me,
+                                 (unsigned long long)(hi - lo));
+            }
+        }
+    }
+
+    // ---- 3. wait until every sender's units of calls 1..e have landed here (bounded)
+    __shared__ int s_ok;
+    const unsigned long long target = e * (unsigned long long)p.U;
+    if (threadIdx.x == 0) {
+        const unsigned long long* landed = reinterpret_cast<const unsigned long long*>(mine);
+        uint32_t missing = 0;
+        int64_t polls = 0;
+        const uint64_t t0 = global_ns();
+        for (int s = 0; s < p.world; ++s) {
+            if (s == me) continue;
+            unsigned ns = 64;
+            while (ld_acquire_sys(landed + s) < target) {
+                if (++polls > p.max_polls || global_ns() - t0 > (uint64_t)p.timeout_ns) {
+                    missing |= 1u << s;
+                    break;
+                }
+                __nanosleep(ns);
+                if (ns < 2048) ns <<= 1;
+            }
+        }
+        if (missing) atomicOr(reinterpret_cast<unsigned*>(mine + LSE_MERGE_CP_STATUS_OFFSET), missing);
+        s_ok = missing == 0;
+    }
+    __syncthreads();
+
+    // ---- 4. merge the owned rows over all senders (skipped after a timeout)
+    char* const dst_o = p.out_o[pr];
+    float* const dst_l = p.out_lse[pr];
+    const int64_t wend = s_ok ? p.U : 0;
+    for (int64_t w = cta * kCpBlock + threadIdx.x; w < wend; w += (int64_t)gridDim.x * kCpBlock) {
+        int64_t row, v, b, hq;
+        divmod(p, w, p.c_dv, p.dv, row, v);
+        divmod(p, row, p.c_Hq, p.Hq, b, hq);
+        const int64_t srow = b * p.H + (int64_t)me * p.Hq + hq;
+        uint4 x[kMaxWorld];
+        float l[kMaxWorld];
+#pragma unroll
+        for (int s = 0; s < kMaxWorld; ++s) {
+            x[s] = make_uint4(0u, 0u, 0u, 0u);
+            l[s] = -INFINITY;
+            if (s < p.world) {
+                if (s == me) {
+                    x[s] = ld_stream16(src_o + srow * p.rowbytes + v * 16);
+                    l[s] = __ldg(src_l + srow);
+                } else {
+                    const int64_t blk = (int64_t)par * w1 + (s - (s > me ? 1 : 0));
+                    x[s] = ld_cg16(mine + p.o_off + blk * p.slot_o + w * 16);
+                    l[s] = ld_cg_f32(reinterpret_cast<const float*>(mine + p.l_off + blk * p.slot_l) + row);
+                }
+            }
+        }
+        float m = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < kMaxWorld; ++s) m = fmaxf(m, l[s]);
+        // An all-empty row has m = -inf; subtracting 0 keeps every weight
+        // exp(-inf) = 0 instead of NaN.
+        const float mref = (m == -INFINITY) ? 0.f : m;
+        uint64_t acc[N2];
+#pragma unroll
+        for (int k = 0; k < N2; ++k) acc[k] = 0ull;
+        float esum = 0.f;
+#pragma unroll
+        for (int s = 0; s < kMaxWorld; ++s) {
+            const float e = expf(l[s] - mref);   // 0 for an empty partial or s >= world
+            esum += e;
+            if (e != 0.f) {                      // an empty partial's o (maybe NaN) is not read
+                uint64_t xx[N2];
+                Elem<TIn>::unpack2(x[s], xx);
+                const uint64_t ww = pack2f(e, e);
+#pragma unroll
+                for (int k = 0; k < N2; ++k) fma2(acc[k], xx[k], ww);
+            }
+        }
+        const float inv = esum > 0.f ? 1.f / esum : 0.f;
+        float f[N];
+#pragma unroll
+        for (int k = 0; k < N2; ++k) {
+            unpack2f(acc[k], f[2 * k], f[2 * k + 1]);
+            f[2 * k] *= inv;
+            f[2 * k + 1] *= inv;
+        }
+        store_vec<TOut, N>(dst_o + w * N * (int64_t)sizeof(TOut), f);
+        if (v == 0) dst_l[row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+    }
+
+    // ---- 5. the last CTA of this rank to finish records call e as completed
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned* done = reinterpret_cast<unsigned*>(mine + kCpDoneOffset);
+        __threadfence();
+        if (atomicAdd(done, 1u) == gridDim.x - 1) {
+            *done = 0u;
+            *reinterpret_cast<volatile unsigned long long*>(mine + kCpEpochOffset) = e;
+        }
+    }
+}
+
+using CpFn = void (*)(CpParams);
+
+template <typename TIn>
+CpFn pick_out(int out_dtype) {
+    switch (out_dtype) {
+        case LSE_MERGE_F32: return cp_exchange_merge_kernel<TIn, float>;
+        case LSE_MERGE_F16: return cp_exchange_merge_kernel<TIn, __half>;
+        default: return cp_exchange_merge_kernel<TIn, __nv_bfloat16>;
+    }
+}
+
+CpFn pick_cp(int in_dtype, int out_dtype) {
+    switch (in_dtype) {
+        case LSE_MERGE_F32: return pick_out<float>(out_dtype);
+        case LSE_MERGE_F16: return pick_out<__half>(out_dtype);
+        default: return pick_out<__nv_bfloat16>(out_dtype);
+    }
+}
+
+// Co-resident CTAs per SM and SM count, cached per (kernel, device).
+struct CoEntry {
+    const void* fn;
+    int dev, per_sm, sms;
+};
+constexpr int kCoSlots = 64;
+CoEntry g_co[kCoSlots];
+int g_co_n = 0;
+std::mutex g_co_mu;
+
+int co_resident(const void* fn, int64_t* capacity) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return (int)e;
+    {
+        std::lock_guard<std::mutex> lk(g_co_mu);
+        for (int i = 0; i < g_co_n; ++i)
+            if (g_co[i].fn == fn && g_co[i].dev == dev) {
+                *capacity = (int64_t)g_co[i].per_sm * g_co[i].sms;
+                return 0;
+            }
+    }
+    int per_sm = 0, sms = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kCpBlock, 0);
+    if (e != cudaSuccess) return (int)e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return (int)e;
+    {
+        std::lock_guard<std::mutex> lk(g_co_mu);
+        if (g_co_n < kCoSlots) g_co[g_co_n++] = CoEntry{fn, dev, per_sm, sms};
+    }
+    *capacity = (int64_t)per_sm * sms;
+    return 0;
+}
+
+int fail_cuda(int code, int e) {
+    set_last_cuda_error(e);
+    (void)cudaGetLastError();   // the failure belongs to this call; do not leave it pending
+    return code;
+}
+
+static_assert(sizeof(cudaIpcMemHandle_t) == LSE_MERGE_CP_IPC_HANDLE_BYTES, "IPC handle size");
+
+}  // namespace
+}  // namespace lsem
+
+extern "C" {
+
+int lse_merge_cp_exchange_merge(const lse_merge_cp_args* a, lse_merge_stream_t stream) {
+    using namespace lsem;
+    if (!a) return LSE_MERGE_ENULL;
+    CpPlan pl;
+    const int rc = make_cp_plan(*a, &pl);
+    if (rc != LSE_MERGE_OK) return rc;
+
+    CpParams kp{};
+    for (int i = 0; i < a->rank_count; ++i) {
+        kp.local_o[i] = static_cast<const char*>(a->local_o[i]);
+        kp.local_lse[i] = a->local_lse[i];
+        kp.out_o[i] = static_cast<char*>(a->out_o[i]);
+        kp.out_lse[i] = a->out_lse[i];
+    }
+    for (int q = 0; q < a->world; ++q) kp.ws[q] = static_cast<char*>(a->ws[q]);
+    kp.world = a->world;
+    kp.rank_begin = a->rank_begin;
+    kp.H = a->H;
+    kp.Hq = pl.Hq;
+    kp.dv = (uint32_t)pl.dv;
+    kp.U = pl.U;
+    kp.rowbytes = (int64_t)a->D * pl.in_bytes;
+    kp.slot_o = pl.slot_o;
+    kp.slot_l = pl.slot_l;
+    kp.o_off = pl.o_off;
+    kp.l_off = pl.l_off;
+    kp.timeout_ns = a->timeout_ns;
+    // Second bound on the wait, should the global timer not advance: with
+    // sleeps growing to ~2 us, this many polls take several times the timeout.
+    kp.max_polls = a->timeout_ns / 256 + 1024;
+    const int64_t send_units = (int64_t)(a->world - 1) * pl.U;
+    kp.idx32 = (send_units + pl.U) < ((int64_t)1 << 31);
+    kp.c_U = fastdiv_c((uint32_t)(kp.idx32 ? pl.U : 1));
+    kp.c_dv = fastdiv_c(kp.dv);
+    kp.c_Hq = fastdiv_c((uint32_t)pl.Hq);
+
+    const CpFn fn = pick_cp(a->in_dtype, a->out_dtype);
+    int64_t capacity = 0;
+    const int ce = co_resident((const void*)fn, &capacity);
+    if (ce != 0) return fail_cuda(LSE_MERGE_ELAUNCH, ce);
+    const int64_t cap = capacity / a->rank_count;
+    if (cap < 1) return fail_cuda(LSE_MERGE_ELAUNCH, (int)cudaErrorCooperativeLaunchTooLarge);
+    const int64_t work = send_units > pl.U ? send_units : pl.U;
+    int64_t ctas = (work + kCpBlock - 1) / kCpBlock;
+    if (ctas > cap) ctas = cap;
+    if (ctas < 1) ctas = 1;
+    kp.chunk = (send_units + ctas - 1) / ctas;
+
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)ctas, (unsigned)a->rank_count, 1);
+    cfg.blockDim = dim3(kCpBlock, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fn, kp);
+    if (e != cudaSuccess) return fail_cuda(LSE_MERGE_ELAUNCH, (int)e);
+    return LSE_MERGE_OK;
+}
+
+int lse_merge_cp_workspace_create(int64_t bytes, void** ws) {
+    if (!ws) return LSE_MERGE_ENULL;
+    if (bytes < lsem::kCpHeaderBytes) return LSE_MERGE_EDIMS;
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, (size_t)bytes);
+    if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    e = cudaMemset(p, 0, (size_t)bytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        (void)cudaFree(p);
+        return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    }
+    *ws = p;
+    return LSE_MERGE_OK;
+}
+
+int lse_merge_cp_status(const void* ws, uint32_t* status) {
+    if (!ws || !status) return LSE_MERGE_ENULL;
+    const cudaError_t e = cudaMemcpy(status, static_cast<const char*>(ws) + LSE_MERGE_CP_STATUS_OFFSET,
+                                     sizeof(uint32_t), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    return LSE_MERGE_OK;
+}
+
+int lse_merge_cp_workspace_zero(void* ws, int64_t bytes) {
+    if (!ws) return LSE_MERGE_ENULL;
+    if (bytes < lsem::kCpHeaderBytes) return LSE_MERGE_EDIMS;
+    cudaError_t e = cudaMemset(ws, 0, (size_t)bytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    return LSE_MERGE_OK;
+}
+
+int lse_merge_cp_workspace_destroy(void* ws) {
+    if (!ws) return LSE_MERGE_ENULL;
+    const cudaError_t e = cudaFree(ws);
+    if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    return LSE_MERGE_OK;
+}
+
+int lse_merge_cp_ipc_handle(void* ws, void* handle) {
+    if (!ws || !handle) return LSE_MERGE_ENULL;
+    cudaIpcMemHandle_t h;
+    const cudaError_t e = cudaIpcGetMemHandle(&h, ws);
+    if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    std::memcpy(handle, &h, sizeof(h));
+    return LSE_MERGE_OK;
+}
+
+int lse_merge_cp_ipc_open(const void* handle, void** peer_ws) {
+    if (!handle || !peer_ws) return LSE_MERGE_ENULL;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    void* p = nullptr;
+    const cudaError_t e = cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    *peer_ws = p;
+    return LSE_MERGE_OK;
+}
+
+int lse_merge_cp_ipc_close(void* peer_ws) {
+    if (!peer_ws) return LSE_MERGE_ENULL;
+    const cudaError_t e = cudaIpcCloseMemHandle(peer_ws);
+    if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    return LSE_MERGE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,179 @@
+// device_common.cuh -- device helpers shared by the kernels of this library:
+// constant division, 16-byte streaming loads, packed fp32 FMA, element
+// conversion, vector stores and programmatic-dependent-launch control.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+namespace lsem {
+namespace {
+
+// Division by a run-time constant d >= 2 of any 32-bit n as the high 64 bits
+// of c * n with c = ceil(2^64 / d) (Lemire, Kaser and Kurz, "Faster remainder
+// by direct computation", 2019, for N = 32 and F = 64 bits).
+__host__ __device__ __forceinline__ uint64_t fastdiv_c(uint32_t d) {
+    return d <= 1 ? 0 : ~0ull / d + 1;
+}
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, uint64_t c, uint32_t d) {
+    return d == 1 ? n : (uint32_t)__umul64hi(c, (uint64_t)n);
+}
+
+// ---------------------------------------------------------------- loads / stores
+
+// 16-byte streaming load: read-only path, no L1 allocation, 256-byte L2 prefetch.
+__device__ __forceinline__ uint4 ld_stream16(const char* p) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+
+// Two fp32 values in one 64-bit register pair, for the packed sm_100 FMA:
+// fma.rn.f32x2 performs two independent IEEE fp32 fused multiply-adds, so
+// every lane of the pair rounds exactly like fmaf.
+__device__ __forceinline__ uint64_t pack2u(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t pack2f(float lo, float hi) {
+    return pack2u(__float_as_uint(lo), __float_as_uint(hi));
+}
+__device__ __forceinline__ void unpack2f(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ void fma2(uint64_t& acc, uint64_t x, uint64_t w) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(x), "l"(w));
+}
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+    static constexpr int kVec = 4;  // elements per 16 bytes
+    __device__ static void unpack(const uint4& v, float* f) {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+    // 16 bytes as fp32 pairs (element 2k in the low half of pair k)
+    __device__ static void unpack2(const uint4& v, uint64_t* x) {
+        x[0] = pack2u(v.x, v.y);
+        x[1] = pack2u(v.z, v.w);
+    }
+    __device__ static float load1(const char* p) { return __ldg(reinterpret_cast<const float*>(p)); }
+    __device__ static void store1(char* p, float x) { *reinterpret_cast<float*>(p) = x; }
+};
+
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float* f) {
+    f[0] = __uint_as_float(w << 16);          // element at the lower address
+    f[1] = __uint_as_float(w & 0xffff0000u);
+}
+
+__device__ __forceinline__ void unpack_f16x2(uint32_t w, float* f) {
+    __half2 h;
+    memcpy(&h, &w, 4);
+    const float2 x = __half22float2(h);
+    f[0] = x.x;
+    f[1] = x.y;
+}
+
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    __device__ static void unpack(const uint4& v, float* f) {
+        unpack_bf16x2(v.x, f + 0);
+        unpack_bf16x2(v.y, f + 2);
+        unpack_bf16x2(v.z, f + 4);
+        unpack_bf16x2(v.w, f + 6);
+    }
+    __device__ static void unpack2(const uint4& v, uint64_t* x) {
+        x[0] = pack2u(v.x << 16, v.x & 0xffff0000u);
+        x[1] = pack2u(v.y << 16, v.y & 0xffff0000u);
+        x[2] = pack2u(v.z << 16, v.z & 0xffff0000u);
+        x[3] = pack2u(v.w << 16, v.w & 0xffff0000u);
+    }
+    __device__ static float widen(unsigned short u) { return __uint_as_float((uint32_t)u << 16); }
+    __device__ static float load1(const char* p) {
+        return widen(__ldg(reinterpret_cast<const unsigned short*>(p)));
+    }
+    __device__ static void store1(char* p, float x) {
+        *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x);
+    }
+    __device__ static uint32_t pack2(float a, float b) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        uint32_t w;
+        memcpy(&w, &h, 4);
+        return w;
+    }
+};
+
+template <>
+struct Elem<__half> {
+    static constexpr int kVec = 8;
+    __device__ static void unpack(const uint4& v, float* f) {
+        unpack_f16x2(v.x, f + 0);
+        unpack_f16x2(v.y, f + 2);
+        unpack_f16x2(v.z, f + 4);
+        unpack_f16x2(v.w, f + 6);
+    }
+    __device__ static void unpack2(const uint4& v, uint64_t* x) {
+        float f[8];
+        unpack(v, f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = pack2f(f[2 * k], f[2 * k + 1]);
+    }
+    __device__ static float widen(unsigned short u) { return __half2float(__ushort_as_half(u)); }
+    __device__ static float load1(const char* p) {
+        return widen(__ldg(reinterpret_cast<const unsigned short*>(p)));
+    }
+    __device__ static void store1(char* p, float x) {
+        *reinterpret_cast<__half*>(p) = __float2half_rn(x);
+    }
+    __device__ static uint32_t pack2(float a, float b) {
+        const __half2 h = __floats2half2_rn(a, b);
+        uint32_t w;
+        memcpy(&w, &h, 4);
+        return w;
+    }
+};
+
+// Store N fp32 values as N elements of TOut at p (aligned to min(16, N*sizeof(TOut))).
+template <typename TOut, int N>
+__device__ __forceinline__ void store_vec(char* p, const float* f) {
+    if constexpr (sizeof(TOut) == 4) {
+#pragma unroll
+        for (int k = 0; k < N; k += 4)
+            *reinterpret_cast<float4*>(p + k * 4) = make_float4(f[k], f[k + 1], f[k + 2], f[k + 3]);
+    } else if constexpr (N == 8) {
+        uint4 w;
+        w.x = Elem<TOut>::pack2(f[0], f[1]);
+        w.y = Elem<TOut>::pack2(f[2], f[3]);
+        w.z = Elem<TOut>::pack2(f[4], f[5]);
+        w.w = Elem<TOut>::pack2(f[6], f[7]);
+        *reinterpret_cast<uint4*>(p) = w;
+    } else {
+        uint2 w;
+        w.x = Elem<TOut>::pack2(f[0], f[1]);
+        w.y = Elem<TOut>::pack2(f[2], f[3]);
+        *reinterpret_cast<uint2*>(p) = w;
+    }
+}
+
+// Programmatic dependent launch: wait for the previous grid in the stream
+// (and its memory) before the first global access, and let the next grid be
+// scheduled as soon as every CTA of this one is running.  Both are no-ops
+// for a launch without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+}  // namespace
+}  // namespace lsem

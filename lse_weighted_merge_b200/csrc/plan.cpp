@@ -313,9 +313,96 @@ int make_state_plan(const void* o_acc, const float* lse_acc, const void* o_new,
     return LSE_MERGE_OK;
 }
 
+int cp_layout(int world, int B, int H, int D, int in_dtype, CpPlan* plan) {
+    const int ib = elem_bytes(in_dtype);
+    if (ib == 0) return LSE_MERGE_EDTYPE;
+    if (world < 1 || world > LSE_MERGE_CP_MAX_WORLD || B < 1 || H < 1 || D < 1 || H % world != 0)
+        return LSE_MERGE_EDIMS;
+    if (((int64_t)D * ib) % 16 != 0) return LSE_MERGE_EALIGN;
+    const i128 lim = (i128)1 << 62;
+    const int Hq = H / world;
+    const i128 slot_o = (i128)B * Hq * D * ib, slot_l = (i128)B * Hq * 4;
+    const i128 n = 2 * (i128)(world - 1);
+    const auto up = [](i128 x) { return (x + 255) / 256 * 256; };
+    const i128 o_off = kCpHeaderBytes;
+    const i128 l_off = up(o_off + n * slot_o);
+    const i128 total = up(l_off + n * slot_l);
+    if ((i128)B * H * D * ib > lim || total > lim) return LSE_MERGE_EDIMS;
+    CpPlan p{};
+    p.world = world;
+    p.Hq = Hq;
+    p.in_bytes = ib;
+    p.dv = (int)((int64_t)D * ib / 16);
+    p.U = (int64_t)B * Hq * p.dv;
+    p.slot_o = (int64_t)slot_o;
+    p.slot_l = (int64_t)slot_l;
+    p.o_off = (int64_t)o_off;
+    p.l_off = (int64_t)l_off;
+    p.ws_bytes = (int64_t)total;
+    *plan = p;
+    return LSE_MERGE_OK;
+}
+
+int make_cp_plan(const lse_merge_cp_args& a, CpPlan* plan) {
+    const int ob = elem_bytes(a.out_dtype);
+    if (elem_bytes(a.in_dtype) == 0 || ob == 0) return LSE_MERGE_EDTYPE;
+    CpPlan p{};
+    int rc = cp_layout(a.world, a.B, a.H, a.D, a.in_dtype, &p);
+    if (rc != LSE_MERGE_OK) return rc;
+    if (a.rank_begin < 0 || a.rank_count < 1 || a.rank_begin + a.rank_count > a.world)
+        return LSE_MERGE_EDIMS;
+    if (a.timeout_ns <= 0 || a.timeout_ns > kCpMaxTimeoutNs) return LSE_MERGE_EDIMS;
+    p.rank_begin = a.rank_begin;
+    p.rank_count = a.rank_count;
+    p.out_bytes = ob;
+    const i128 in_o = (i128)a.B * a.H * a.D * p.in_bytes, in_l = (i128)a.B * a.H * 4;
+    const i128 out_o = (i128)a.B * p.Hq * a.D * ob, out_l = (i128)a.B * p.Hq * 4;
+    // Written spans (workspaces, outputs) may overlap nothing else; inputs
+    // are only read and may overlap one another.
+    Span wr[3 * LSE_MERGE_CP_MAX_WORLD], rd[2 * LSE_MERGE_CP_MAX_WORLD];
+    int nw = 0, nr = 0;
+    for (int q = 0; q < a.world; ++q) {
+        if (!a.ws[q]) return LSE_MERGE_ENULL;
+        if (!aligned(a.ws[q], 256)) return LSE_MERGE_EALIGN;
+        wr[nw++] = Span{(uintptr_t)a.ws[q], (i128)(uintptr_t)a.ws[q] + p.ws_bytes};
+    }
+    for (int i = 0; i < a.rank_count; ++i) {
+        if (!a.local_o[i] || !a.local_lse[i] || !a.out_o[i] || !a.out_lse[i]) return LSE_MERGE_ENULL;
+        if (!aligned(a.local_o[i], 16) || !aligned(a.out_o[i], 16) || !aligned(a.local_lse[i], 4) ||
+            !aligned(a.out_lse[i], 4))
+            return LSE_MERGE_EALIGN;
+        rd[nr++] = Span{(uintptr_t)a.local_o[i], (i128)(uintptr_t)a.local_o[i] + in_o};
+        rd[nr++] = Span{(uintptr_t)a.local_lse[i], (i128)(uintptr_t)a.local_lse[i] + in_l};
+        wr[nw++] = Span{(uintptr_t)a.out_o[i], (i128)(uintptr_t)a.out_o[i] + out_o};
+        wr[nw++] = Span{(uintptr_t)a.out_lse[i], (i128)(uintptr_t)a.out_lse[i] + out_l};
+    }
+    for (int i = 0; i < nw; ++i) {
+        for (int j = i + 1; j < nw; ++j)
+            if (overlap(wr[i], wr[j])) return LSE_MERGE_EALIAS;
+        for (int j = 0; j < nr; ++j)
+            if (overlap(wr[i], rd[j])) return LSE_MERGE_EALIAS;
+    }
+    *plan = p;
+    return LSE_MERGE_OK;
+}
+
 }  // namespace lsem
 
 extern "C" {
+
+int lse_merge_cp_workspace_bytes(int world, int B, int H, int D, int in_dtype, int64_t* bytes) {
+    if (!bytes) return LSE_MERGE_ENULL;
+    lsem::CpPlan p;
+    const int rc = lsem::cp_layout(world, B, H, D, in_dtype, &p);
+    if (rc == LSE_MERGE_OK) *bytes = p.ws_bytes;
+    return rc;
+}
+
+int lse_merge_cp_validate(const lse_merge_cp_args* args) {
+    if (!args) return LSE_MERGE_ENULL;
+    lsem::CpPlan p;
+    return lsem::make_cp_plan(*args, &p);
+}
 
 int lse_merge_plan_query(const void* partial_o, const float* partial_lse, int R, int B, int H,
                          int D, const lse_merge_strides* strides, int in_dtype, int out_dtype,
@@ -339,6 +426,7 @@ const char* lse_merge_strerror(int code) {
         case LSE_MERGE_EALIGN: return "a pointer is not aligned to its element size";
         case LSE_MERGE_EPATH: return "the requested kernel path cannot take these arguments";
         case LSE_MERGE_EUNSUP: return "shape not implemented by the decode-attention kernels (dtype, D, group, R)";
+        case LSE_MERGE_ECUDA: return "a CUDA runtime call of a set-up function failed";
         default: return "unknown lse_merge error code";
     }
 }

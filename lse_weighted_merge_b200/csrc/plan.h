@@ -116,4 +116,31 @@ int make_state_plan(const void* o_acc, const float* lse_acc, const void* o_new,
                     const float* lse_new, int B, int H, int D, const lse_merge_state_strides& st,
                     int acc_dtype, int new_dtype, StatePlan* plan);
 
+// Context-parallel exchange + merge: validated layout of one rank's workspace
+// and of the units each rank sends.  A unit is 16 bytes of one partial row.
+struct CpPlan {
+    int world, rank_begin, rank_count, Hq;
+    int in_bytes, out_bytes;
+    int dv;            // units per row, D * in_bytes / 16
+    int64_t U;         // units one rank sends to one other rank, B * Hq * dv
+    int64_t slot_o;    // bytes of one received partial block [B, Hq, D]
+    int64_t slot_l;    // bytes of one received lse block [B, Hq]
+    int64_t o_off;     // workspace offset of recv_o [2][world-1][B][Hq][D]
+    int64_t l_off;     // workspace offset of recv_lse [2][world-1][B][Hq]
+    int64_t ws_bytes;  // bytes of one workspace
+};
+constexpr int kCpBlock = 256;
+// Workspace header: landed counters (8 x u64) at 0, the status word at
+// LSE_MERGE_CP_STATUS_OFFSET, the rank's completed-call count (u64) and the
+// finished-CTA count of the running call (u32).
+constexpr int64_t kCpHeaderBytes = 256;
+constexpr int64_t kCpEpochOffset = 128;
+constexpr int64_t kCpDoneOffset = 136;
+constexpr int64_t kCpMaxTimeoutNs = 60ll * 1000 * 1000 * 1000;
+
+// Workspace layout for these sizes (no pointer checks).
+int cp_layout(int world, int B, int H, int D, int in_dtype, CpPlan* plan);
+// Full validation of lse_merge_cp_exchange_merge's arguments.
+int make_cp_plan(const lse_merge_cp_args& a, CpPlan* plan);
+
 }  // namespace lsem

@@ -74,6 +74,22 @@ WORKLOADS = {
     ]
 }
 
+# Context-parallel exchange + merge: R = world ranks, layout "rbhd" = rank s's
+# local partials [B, H, D] in block s.  The first two are the shapes of the
+# CP-decode page's result table (batch 1, heads 2, dim 64; batch 1, heads 8,
+# dim 128; the page states no world size, so 2 and 8 ranks are chosen).
+CP_WORKLOADS = {
+    w.name: w for w in [
+        Workload("cp_w2_b1_h2_d64", 2, 1, 2, 64, "bf16", "bf16", "rbhd", 1.0,
+                 "uniform", (-5.0, 5.0), 1100, note="CP decode, 2 ranks, one head each"),
+        Workload("cp_w8_b1_h8_d128", 8, 1, 8, 128, "bf16", "bf16", "rbhd", 1.0,
+                 "uniform", (0.0, 12.0), 1101, note="CP decode, 8 ranks, one head each"),
+        Workload("cp_w8_b64_h32_d128_masked", 8, 64, 32, 128, "bf16", "bf16", "rbhd", 1.0,
+                 "normal", (6.0, 3.0), 1102, empty_shard_p=0.10, empty_row_p=0.01,
+                 note="CP decode, 8 ranks, batch 64, 10% empty shards, 1% empty rows"),
+    ]
+}
+
 SMALL = "r2_b1_h2_d64"
 LARGE = "r16_b512_h16_d512"
 
