@@ -70,6 +70,7 @@ typedef struct {
 #define LSE_MERGE_EPATH (-8)    /* the requested path cannot take these arguments */
 #define LSE_MERGE_EUNSUP (-9)   /* a shape the decode-attention kernels do not implement */
 #define LSE_MERGE_ECUDA (-10)   /* a CUDA runtime call of a set-up function failed */
+#define LSE_MERGE_ESCRATCH (-11) /* the problem needs more than the static scratch holds */
 
 /* Kernel paths.  AUTO picks one from the sizes, dtypes and alignment. */
 #define LSE_MERGE_PATH_AUTO 0
@@ -320,6 +321,41 @@ int lse_merge_cp_workspace_destroy(void* ws);
 int lse_merge_cp_ipc_handle(void* ws, void* handle);
 int lse_merge_cp_ipc_open(const void* handle, void** peer_ws);
 int lse_merge_cp_ipc_close(void* peer_ws);
+
+/* The exchange and merge for callers that cannot allocate device memory.
+ * (No counterpart on the pages; it is a service of this library.)
+ *
+ * Some callers cannot call cudaMalloc at the point where they run this step:
+ * a serving runtime that has handed all spare HBM to its KV-cache pool at
+ * start-up has nothing left to allocate, and cudaMalloc itself may
+ * synchronise the whole device, which a decode step that must keep the
+ * device busy cannot afford.  This entry point therefore allocates nothing:
+ * the workspaces of all ranks are carved out of one array that the library
+ * defines in device memory, LSE_MERGE_CP_NOALLOC_SCRATCH_BYTES (16 MiB) per
+ * GPU, held by every GPU that loads the library until the process exits.
+ * The caller passes inputs and outputs exactly as for
+ * lse_merge_cp_exchange_merge, with these differences:
+ *   - the launch must play every rank (rank_begin = 0, rank_count = world),
+ *     since the array lives on this GPU only and cannot be shared with
+ *     other processes; args->ws is not read;
+ *   - world * lse_merge_cp_workspace_bytes(...) must fit in the array,
+ *     else LSE_MERGE_ESCRATCH is returned and nothing is launched;
+ *   - each call first clears the workspace headers on `stream` (a memset,
+ *     no allocation), so every call starts from zero and a wait that ran out
+ *     in an earlier call needs no restart; the received rows need no
+ *     clearing, every one is written before it is read;
+ *   - all calls on a GPU share the one array: calls whose work overlaps on
+ *     the GPU (different streams, no ordering between them) race and give
+ *     wrong results; order them on one stream;
+ *   - the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make
+ *     that first call before any stream capture begins.
+ * A wait that runs out sets the status word of that rank's workspace inside
+ * the array (not readable through this interface); the kernel still returns.
+ * Returns the codes of lse_merge_cp_exchange_merge, LSE_MERGE_ESCRATCH, and
+ * LSE_MERGE_ECUDA when the address look-up or the header clearing fails. */
+#define LSE_MERGE_CP_NOALLOC_SCRATCH_BYTES (16 << 20)
+int lse_merge_cp_exchange_merge_noalloc(const lse_merge_cp_args* args, lse_merge_stream_t stream);
 
 /* A static, human-readable description of a return code. */
 const char* lse_merge_strerror(int code);

@@ -17,8 +17,8 @@ PATH_AUTO, PATH_VECTOR, PATH_LATENCY, PATH_SCALAR, PATH_STREAM, PATH_WIDE = 0, 1
 PATH_NAMES = {PATH_VECTOR: "vector", PATH_LATENCY: "latency", PATH_SCALAR: "scalar",
               PATH_STREAM: "stream", PATH_WIDE: "wide"}
 
-OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH, EUNSUP, ECUDA = (
-    0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10)
+OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH, EUNSUP, ECUDA, ESCRATCH = (
+    0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10, -11)
 CP_MAX_WORLD = 8
 CP_STATUS_OFFSET = 64
 CP_IPC_HANDLE_BYTES = 64
@@ -29,7 +29,8 @@ EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merg
            "lse_merge_last_cuda_error", "lse_merge_version", "lse_merge_cp_workspace_bytes",
            "lse_merge_cp_validate", "lse_merge_cp_exchange_merge", "lse_merge_cp_workspace_create",
            "lse_merge_cp_workspace_destroy", "lse_merge_cp_ipc_handle", "lse_merge_cp_ipc_open",
-           "lse_merge_cp_ipc_close", "lse_merge_cp_status", "lse_merge_cp_workspace_zero")
+           "lse_merge_cp_ipc_close", "lse_merge_cp_status", "lse_merge_cp_workspace_zero",
+           "lse_merge_cp_exchange_merge_noalloc")
 ABI_VERSION = 3
 
 
@@ -126,6 +127,8 @@ def _load() -> ctypes.CDLL:
     lib.lse_merge_cp_validate.restype = i
     lib.lse_merge_cp_exchange_merge.argtypes = [ctypes.POINTER(CpArgs), vp]
     lib.lse_merge_cp_exchange_merge.restype = i
+    lib.lse_merge_cp_exchange_merge_noalloc.argtypes = [ctypes.POINTER(CpArgs), vp]
+    lib.lse_merge_cp_exchange_merge_noalloc.restype = i
     lib.lse_merge_cp_workspace_create.argtypes = [ctypes.c_int64, ctypes.POINTER(vp)]
     lib.lse_merge_cp_workspace_create.restype = i
     lib.lse_merge_cp_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -248,6 +251,15 @@ def cp_validate(args: CpArgs) -> int:
 
 def cp_exchange_merge_raw(args: CpArgs, stream: int = 0, check: bool = True) -> int:
     rc = lib.lse_merge_cp_exchange_merge(ctypes.byref(args), stream or None)
+    if check and rc != OK:
+        _raise(rc)
+    return rc
+
+
+def cp_exchange_merge_noalloc_raw(args: CpArgs, stream: int = 0, check: bool = True) -> int:
+    """lse_merge_cp_exchange_merge_noalloc: every rank in one launch, the
+    workspaces taken from the library's static device array (args.ws unused)."""
+    rc = lib.lse_merge_cp_exchange_merge_noalloc(ctypes.byref(args), stream or None)
     if check and rc != OK:
         _raise(rc)
     return rc

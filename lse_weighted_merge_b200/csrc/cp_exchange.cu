@@ -479,3 +479,71 @@ int lse_merge_cp_ipc_close(void* peer_ws) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// The entry point that allocates nothing: its workspaces live in this array.
+namespace lsem {
+namespace {
+
+constexpr int64_t kNoAllocBytes = LSE_MERGE_CP_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device.  In host
+// code the array's name is only a stand-in for the symbol, never an address
+// a kernel may be given.
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(void** ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return (int)e;
+    if (dev >= 0 && dev < kMaxDevices) {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (g_noalloc_ptr[dev]) {
+            *ptr = g_noalloc_ptr[dev];
+            return 0;
+        }
+    }
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return (int)e;
+    if (dev >= 0 && dev < kMaxDevices) {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = p;
+    return 0;
+}
+
+}  // namespace
+}  // namespace lsem
+
+extern "C" int lse_merge_cp_exchange_merge_noalloc(const lse_merge_cp_args* args,
+                                                   lse_merge_stream_t stream) {
+    using namespace lsem;
+    if (!args) return LSE_MERGE_ENULL;
+    int64_t ws_bytes = 0;
+    int rc = lse_merge_cp_workspace_bytes(args->world, args->B, args->H, args->D, args->in_dtype,
+                                          &ws_bytes);
+    if (rc != LSE_MERGE_OK) return rc;
+    if (args->rank_begin != 0 || args->rank_count != args->world) return LSE_MERGE_EDIMS;
+    const int64_t pitch = (ws_bytes + 255) / 256 * 256;
+    if ((int64_t)args->world * pitch > kNoAllocBytes) return LSE_MERGE_ESCRATCH;
+    void* base = nullptr;
+    const int se = noalloc_scratch(&base);
+    if (se != 0) return fail_cuda(LSE_MERGE_ECUDA, se);
+    lse_merge_cp_args a = *args;
+    for (int q = 0; q < LSE_MERGE_CP_MAX_WORLD; ++q)
+        a.ws[q] = q < a.world ? static_cast<char*>(base) + (int64_t)q * pitch : nullptr;
+    // Validate before touching the array, so a rejected call changes nothing.
+    rc = lse_merge_cp_validate(&a);
+    if (rc != LSE_MERGE_OK) return rc;
+    // Every call starts from zeroed headers: landed counters, status word,
+    // completed-call count and finished-CTA count of each rank.
+    const cudaError_t e = cudaMemset2DAsync(base, (size_t)pitch, 0, (size_t)kCpHeaderBytes,
+                                            (size_t)a.world, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    return lse_merge_cp_exchange_merge(&a, stream);
+}

@@ -427,6 +427,7 @@ const char* lse_merge_strerror(int code) {
         case LSE_MERGE_EPATH: return "the requested kernel path cannot take these arguments";
         case LSE_MERGE_EUNSUP: return "shape not implemented by the decode-attention kernels (dtype, D, group, R)";
         case LSE_MERGE_ECUDA: return "a CUDA runtime call of a set-up function failed";
+        case LSE_MERGE_ESCRATCH: return "the problem needs more scratch memory than the static array holds (16 MiB)";
         default: return "unknown lse_merge error code";
     }
 }
