@@ -46,6 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FALLBACK = 126 * 1024 * 1024
 BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 KERNEL_SOURCES = ("lse_weighted_merge_b200/csrc/lse_merge.cu",
+                  "lse_weighted_merge_b200/csrc/device_common.cuh",
                   "lse_weighted_merge_b200/csrc/plan.cpp",
                   "lse_weighted_merge_b200/csrc/plan.h")
 
@@ -68,6 +69,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--decode-only", default=None, metavar="SHAPE",
                    help="only time the decode-attention shape SHAPE (for profiling)")
+    p.add_argument("--cp-only", default=None, metavar="WORKLOAD",
+                   help="only time the context-parallel exchange + merge WORKLOAD (for profiling)")
     return p.parse_args(argv)
 
 
@@ -567,7 +570,82 @@ def extra_workloads(device, l2: int, dist) -> dict:
         del sets
         torch.cuda.empty_cache()
     return {"workloads": res, "state_update": time_state_update(device, l2, peak),
-            "decode_attention": time_decode_attention(device, peak)}
+            "decode_attention": time_decode_attention(device, peak),
+            "cp_exchange_merge": time_cp_exchange(device, peak)}
+
+
+def time_cp_exchange(device, peak: float, only: str | None = None) -> dict:
+    """Context-parallel exchange + merge with every rank on this one GPU, all
+    ranks played by one cooperative launch (lse_merge_cp_exchange_merge):
+    us/call eager and graph-replayed.  Bytes per call on one GPU: every
+    rank's partials read once, the (world-1)/world of them owned elsewhere
+    written to and read back from the workspaces, the outputs written.  On
+    world GPUs the same kernel would move the (world-1)/world share over
+    NVLink instead; that cannot be measured here."""
+    import torch
+    from lse_weighted_merge_b200 import cp, synth
+    res = {}
+    for name, w in synth.CP_WORKLOADS.items():
+        if only is not None and name != only:
+            continue
+        inp = synth.make_inputs(w)
+        W, B, H, D = w.R, w.B, w.H, w.D
+        dt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[w.in_dtype]
+        raw = torch.from_numpy(inp["o"].view("int16") if w.in_dtype != "f32" else inp["o"])
+        o = raw.to(device).view(dt).view(W, B, H, D)
+        l = torch.from_numpy(inp["lse"]).to(device).view(W, B, H)
+        lo = [o[r].contiguous() for r in range(W)]
+        ll = [l[r].contiguous() for r in range(W)]
+        ws = [cp.cp_workspace(W, B, H, D, dt, device) for _ in range(W)]
+        outs = cp.cp_exchange_merge(lo, ll, ws)
+        eb = {"bf16": 2, "f16": 2, "f32": 4}[w.in_dtype]
+        part = W * B * H * (D * eb + 4)
+        byts = part + 2 * part * (W - 1) // W + W * B * (H // W) * (D * eb + 4)
+
+        def call():
+            cp.cp_exchange_merge(lo, ll, ws, outs=outs)
+
+        for _ in range(10):
+            call()
+        torch.cuda.synchronize(device)
+        n = 200
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            call()
+        e1.record()
+        torch.cuda.synchronize(device)
+        eager = e0.elapsed_time(e1) * 1e3 / n
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device)
+        side.wait_stream(torch.cuda.current_stream(device))
+        reps = 20
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(reps):
+                    call()
+        torch.cuda.synchronize(device)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize(device)
+        e0.record()
+        for _ in range(10):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize(device)
+        graph = e0.elapsed_time(e1) * 1e3 / (10 * reps)
+        status = [cp.cp_status(x) for x in ws]
+        res[name] = {"shape": f"world={W} B={B} H={H} D={D} {w.in_dtype}, all ranks in one launch",
+                     "eager_us_per_call": eager, "graph_us_per_call": graph,
+                     "bytes_per_call_one_gpu": byts,
+                     "graph_gbs": byts / (graph * 1e-6) / 1e9,
+                     "frac_of_measured_hbm_graph": byts / (graph * 1e-6) / 1e9 / peak,
+                     "nvlink_bytes_per_rank_if_distributed": part // W * (W - 1) // W,
+                     "timeouts": sum(1 for x in status if x)}
+        del g, ws, lo, ll, o, l
+        torch.cuda.empty_cache()
+    return res
 
 
 DECODE_SHAPES = (  # name, B, Hq, Hkv, L, D, R
@@ -678,6 +756,12 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.cp_only:
+        import torch
+        device = torch.device("cuda", 0)
+        peak, _ = hbm_peak()
+        print(json.dumps({"cp_exchange_merge": time_cp_exchange(device, peak, args.cp_only)}))
+        return 0
     if args.decode_only:
         import torch
         device = torch.device("cuda", 0)
