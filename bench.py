@@ -577,7 +577,8 @@ def extra_workloads(device, l2: int, dist) -> dict:
 def time_cp_exchange(device, peak: float, only: str | None = None) -> dict:
     """Context-parallel exchange + merge with every rank on this one GPU, all
     ranks played by one cooperative launch (lse_merge_cp_exchange_merge):
-    us/call eager and graph-replayed.  Bytes per call on one GPU: every
+    us/call eager (a prepared CPMergeCall: one launch per call) and
+    graph-replayed.  Bytes per call on one GPU: every
     rank's partials read once, the (world-1)/world of them owned elsewhere
     written to and read back from the workspaces, the outputs written.  On
     world GPUs the same kernel would move the (world-1)/world share over
@@ -597,13 +598,10 @@ def time_cp_exchange(device, peak: float, only: str | None = None) -> dict:
         lo = [o[r].contiguous() for r in range(W)]
         ll = [l[r].contiguous() for r in range(W)]
         ws = [cp.cp_workspace(W, B, H, D, dt, device) for _ in range(W)]
-        outs = cp.cp_exchange_merge(lo, ll, ws)
+        call = cp.CPMergeCall(lo, ll, ws)
         eb = {"bf16": 2, "f16": 2, "f32": 4}[w.in_dtype]
         part = W * B * H * (D * eb + 4)
         byts = part + 2 * part * (W - 1) // W + W * B * (H // W) * (D * eb + 4)
-
-        def call():
-            cp.cp_exchange_merge(lo, ll, ws, outs=outs)
 
         for _ in range(10):
             call()
@@ -643,7 +641,7 @@ def time_cp_exchange(device, peak: float, only: str | None = None) -> dict:
                      "frac_of_measured_hbm_graph": byts / (graph * 1e-6) / 1e9 / peak,
                      "nvlink_bytes_per_rank_if_distributed": part // W * (W - 1) // W,
                      "timeouts": sum(1 for x in status if x)}
-        del g, ws, lo, ll, o, l
+        del g, call, ws, lo, ll, o, l
         torch.cuda.empty_cache()
     return res
 

@@ -246,7 +246,8 @@ int lse_merge_decode_attention(const void* q, const void* k, const void* v, cons
  *   1. every (b, h) row owned by another rank q is stored into q's workspace
  *      (plain 16-byte stores; ws[q] may be a peer GPU's memory);
  *   2. the rank adds the number of 16-byte units it stored for q to q's
- *      landed counter for this sender (system-scope release);
+ *      landed counter for this sender (a system-scope release; device scope
+ *      when the launch plays every rank);
  *   3. it waits, bounded by timeout_ns of the GPU's global timer, until every
  *      other rank's landed counter in its own workspace reached e * U, e the
  *      number of this call since the workspace was zeroed (U = B*Hq*D*elem/16
@@ -256,9 +257,10 @@ int lse_merge_decode_attention(const void* q, const void* k, const void* v, cons
  *   5. its last CTA to finish records call e as completed in the workspace.
  * The call number lives in the workspace, so every rank must make the same
  * calls since the workspaces were zeroed, each rank's calls ordered on one
- * stream; a captured CUDA graph may replay a call.  Received rows alternate
- * between two slots by the parity of e, so a rank may start call e + 1 while
- * a peer still merges call e.  A wait that runs out ORs bit s (sender s) into
+ * stream; a captured CUDA graph may replay a call.  Across GPUs, received
+ * rows alternate between two slots by the parity of e, so a rank may start
+ * call e + 1 while a peer still merges call e; a launch that plays every rank
+ * uses one slot, since its next call starts after it ends.  A wait that runs out ORs bit s (sender s) into
  * the uint32 status word at byte LSE_MERGE_CP_STATUS_OFFSET of that rank's
  * workspace, leaves that rank's outputs unwritten and returns; the
  * workspaces are then out of step, and every rank must zero its workspace
@@ -285,6 +287,10 @@ int lse_merge_decode_attention(const void* q, const void* k, const void* v, cons
 #define LSE_MERGE_CP_MAX_WORLD 8
 #define LSE_MERGE_CP_STATUS_OFFSET 64     /* uint32 in each workspace; 0 = no wait ran out */
 #define LSE_MERGE_CP_IPC_HANDLE_BYTES 64
+/* Run the cross-GPU protocol (system-scope release and acquire, two receive
+ * slots) even when the launch plays every rank, which otherwise uses device
+ * scope and one slot; this lets one GPU test the multi-GPU protocol. */
+#define LSE_MERGE_CP_FLAG_CROSS_GPU_PROTOCOL 1
 
 typedef struct {
     int world, rank_begin, rank_count;
@@ -295,6 +301,7 @@ typedef struct {
     void* ws[LSE_MERGE_CP_MAX_WORLD];               /* workspace of every rank q < world */
     int B, H, D, in_dtype, out_dtype;
     int64_t timeout_ns;
+    int flags;                                      /* LSE_MERGE_CP_FLAG_*, normally 0 */
 } lse_merge_cp_args;
 
 /* Bytes of one rank's workspace (the same on every rank). */
@@ -366,7 +373,7 @@ int lse_merge_last_cuda_error(void);
 /* ABI version of this header; bumped on any incompatible change. */
 int lse_merge_version(void);
 
-#define LSE_MERGE_ABI_VERSION 3
+#define LSE_MERGE_ABI_VERSION 4
 
 #ifdef __cplusplus
 }

@@ -15,7 +15,7 @@ from __future__ import annotations
 # and the build script import without the compiled library.  Using any of
 # these names without liblse_merge.so raises ImportError: there is no
 # fallback.
-_CP = ("cp_exchange_merge", "cp_workspace", "cp_status", "CPExchangeMerge", "PeerLost")
+_CP = ("cp_exchange_merge", "CPMergeCall", "cp_workspace", "cp_status", "CPExchangeMerge", "PeerLost")
 _API = ("merge", "merge_state_", "merge_host", "release_host_workspace", "merge_raw",
         "state_update_raw", "decode_attention", "decode_raw", "plan_query", "strerror", "LseMergeError", "dtype_code",
         "F32", "F16", "BF16", "PATH_AUTO", "PATH_VECTOR", "PATH_LATENCY", "PATH_SCALAR",

@@ -22,6 +22,7 @@ OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH, EUNSUP, ECUDA
 CP_MAX_WORLD = 8
 CP_STATUS_OFFSET = 64
 CP_IPC_HANDLE_BYTES = 64
+CP_FLAG_CROSS_GPU_PROTOCOL = 1
 
 # Every symbol include/lse_merge.h declares.
 EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merge_state_update",
@@ -31,7 +32,7 @@ EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merg
            "lse_merge_cp_workspace_destroy", "lse_merge_cp_ipc_handle", "lse_merge_cp_ipc_open",
            "lse_merge_cp_ipc_close", "lse_merge_cp_status", "lse_merge_cp_workspace_zero",
            "lse_merge_cp_exchange_merge_noalloc")
-ABI_VERSION = 3
+ABI_VERSION = 4
 
 
 class Strides(ctypes.Structure):
@@ -68,11 +69,12 @@ class CpArgs(ctypes.Structure):
                 ("local_o", _P8), ("local_lse", _P8), ("out_o", _P8), ("out_lse", _P8),
                 ("ws", _P8), ("B", ctypes.c_int), ("H", ctypes.c_int),
                 ("D", ctypes.c_int), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
-                ("timeout_ns", ctypes.c_int64)]
+                ("timeout_ns", ctypes.c_int64), ("flags", ctypes.c_int)]
 
 
 def cp_args(world: int, rank_begin: int, local_o, local_lse, out_o, out_lse, ws,
-            B: int, H: int, D: int, in_dtype: int, out_dtype: int, timeout_ns: int) -> CpArgs:
+            B: int, H: int, D: int, in_dtype: int, out_dtype: int, timeout_ns: int,
+            flags: int = 0) -> CpArgs:
     """Fill lse_merge_cp_args from lists of raw pointers (one per played rank / per rank)."""
     def arr(ptrs):
         if len(ptrs) > CP_MAX_WORLD:
@@ -83,7 +85,7 @@ def cp_args(world: int, rank_begin: int, local_o, local_lse, out_o, out_lse, ws,
         return a
     return CpArgs(int(world), int(rank_begin), len(local_o), arr(local_o), arr(local_lse),
                   arr(out_o), arr(out_lse), arr(ws), int(B), int(H), int(D),
-                  int(in_dtype), int(out_dtype), int(timeout_ns))
+                  int(in_dtype), int(out_dtype), int(timeout_ns), int(flags))
 
 
 class LseMergeError(RuntimeError):

@@ -52,8 +52,61 @@ def _ptr(x) -> int:
     return x if isinstance(x, int) else x.data_ptr()
 
 
+class CPMergeCall:
+    """A prepared exchange + merge over fixed buffers.
+
+    Validates the tensors and builds the C argument block once; each call is
+    then a single launch on the current (or given) stream, which keeps the
+    host cost of an eager step to the launch itself.  Arguments are those of
+    ``cp_exchange_merge``; ``outs`` holds the output pairs it writes.
+    """
+
+    def __init__(self, local_o, local_lse, workspaces, *, rank_begin: int = 0, out_dtype=None,
+                 timeout_s: float = DEFAULT_TIMEOUT_S, outs=None, cross_gpu_protocol: bool = False):
+        import torch
+        world = len(workspaces)
+        n = len(local_o)
+        if n < 1 or len(local_lse) != n:
+            raise ValueError("local_o and local_lse must list the same ranks (at least one)")
+        B, H, D = local_o[0].shape
+        if H % world:
+            raise ValueError(f"H = {H} is not a multiple of world = {world}")
+        Hq = H // world
+        dev = local_o[0].device
+        in_dtype = local_o[0].dtype
+        out_dtype = out_dtype or in_dtype
+        for o, l in zip(local_o, local_lse):
+            if not (o.is_cuda and l.is_cuda) or o.device != dev or l.device != dev:
+                raise ValueError("all tensors must be on one CUDA device (there is no CPU path)")
+            _check_local(o, l, B, H, D, in_dtype)
+        if outs is None:
+            outs = [(torch.empty((B, Hq, D), dtype=out_dtype, device=dev),
+                     torch.empty((B, Hq), dtype=torch.float32, device=dev)) for _ in range(n)]
+        # keep every buffer alive as long as the argument block points at it
+        self._keep = (list(local_o), list(local_lse), list(workspaces))
+        self.outs = outs
+        self.device = dev
+        self.args = _native.cp_args(world, rank_begin, [o.data_ptr() for o in local_o],
+                                    [l.data_ptr() for l in local_lse],
+                                    [o.data_ptr() for o, _ in outs], [l.data_ptr() for _, l in outs],
+                                    [_ptr(w) for w in workspaces], B, H, D, dtype_code(in_dtype),
+                                    dtype_code(out_dtype), int(timeout_s * 1e9),
+                                    _native.CP_FLAG_CROSS_GPU_PROTOCOL if cross_gpu_protocol else 0)
+        rc = _native.cp_validate(self.args)
+        if rc != _native.OK:
+            _native._raise(rc)
+
+    def __call__(self, stream=None):
+        import torch
+        with torch.cuda.device(self.device):
+            s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+            _native.cp_exchange_merge_raw(self.args, s)
+        return self.outs
+
+
 def cp_exchange_merge(local_o, local_lse, workspaces, *, rank_begin: int = 0, out_dtype=None,
-                      timeout_s: float = DEFAULT_TIMEOUT_S, outs=None):
+                      timeout_s: float = DEFAULT_TIMEOUT_S, outs=None,
+                      cross_gpu_protocol: bool = False):
     """Exchange heads between ranks and merge, in one launch on the current stream.
 
     local_o:    list of CUDA tensors [B, H, D] (float32 / float16 / bfloat16,
@@ -66,35 +119,13 @@ def cp_exchange_merge(local_o, local_lse, workspaces, *, rank_begin: int = 0, ou
                 [B, H/world]) pairs.
     Returns one (out, out_lse) pair per played rank.  A rank whose wait runs
     out (timeout_s) leaves its outputs unwritten and sets its workspace's
-    status word (``cp_status``).
+    status word (``cp_status``).  cross_gpu_protocol=True runs the protocol
+    of ranks on different GPUs (system scope, two receive slots) although
+    every rank is on this one, to test it.  For repeated calls over the same
+    buffers, ``CPMergeCall`` prepares the arguments once.
     """
-    import torch
-    world = len(workspaces)
-    n = len(local_o)
-    if n < 1 or len(local_lse) != n:
-        raise ValueError("local_o and local_lse must list the same ranks (at least one)")
-    B, H, D = local_o[0].shape
-    if H % world:
-        raise ValueError(f"H = {H} is not a multiple of world = {world}")
-    Hq = H // world
-    dev = local_o[0].device
-    in_dtype = local_o[0].dtype
-    out_dtype = out_dtype or in_dtype
-    for o, l in zip(local_o, local_lse):
-        if not (o.is_cuda and l.is_cuda) or o.device != dev or l.device != dev:
-            raise ValueError("all tensors must be on one CUDA device (there is no CPU path)")
-        _check_local(o, l, B, H, D, in_dtype)
-    if outs is None:
-        outs = [(torch.empty((B, Hq, D), dtype=out_dtype, device=dev),
-                 torch.empty((B, Hq), dtype=torch.float32, device=dev)) for _ in range(n)]
-    args = _native.cp_args(world, rank_begin, [o.data_ptr() for o in local_o],
-                           [l.data_ptr() for l in local_lse],
-                           [o.data_ptr() for o, _ in outs], [l.data_ptr() for _, l in outs],
-                           [_ptr(w) for w in workspaces], B, H, D, dtype_code(in_dtype),
-                           dtype_code(out_dtype), int(timeout_s * 1e9))
-    with torch.cuda.device(dev):
-        _native.cp_exchange_merge_raw(args, torch.cuda.current_stream(dev).cuda_stream)
-    return outs
+    return CPMergeCall(local_o, local_lse, workspaces, rank_begin=rank_begin, out_dtype=out_dtype,
+                       timeout_s=timeout_s, outs=outs, cross_gpu_protocol=cross_gpu_protocol)()
 
 
 class PeerLost(RuntimeError):
@@ -150,6 +181,8 @@ class CPExchangeMerge:
         self.broken = False
         self.calls = 0
         self._checks = 0
+        self._args_key = None
+        self._args = None
         me = (self.B, self.H, self.D, self.in_dtype, self.out_dtype, self.timeout_ns)
         every = [None] * self.world
         dist.all_gather_object(every, me, group=group)
@@ -178,9 +211,13 @@ class CPExchangeMerge:
             out = torch.empty((self.B, Hq, self.D), dtype=_torch_dtype(self.out_dtype), device=dev)
         if out_lse is None:
             out_lse = torch.empty((self.B, Hq), dtype=torch.float32, device=dev)
-        args = _native.cp_args(self.world, self.rank, [local_o.data_ptr()], [local_lse.data_ptr()],
-                               [out.data_ptr()], [out_lse.data_ptr()], self.peers, self.B, self.H,
-                               self.D, self.in_dtype, self.out_dtype, self.timeout_ns)
+        key = (local_o.data_ptr(), local_lse.data_ptr(), out.data_ptr(), out_lse.data_ptr())
+        if self._args_key != key:      # the argument block is rebuilt only for new buffers
+            self._args = _native.cp_args(self.world, self.rank, [key[0]], [key[1]], [key[2]],
+                                         [key[3]], self.peers, self.B, self.H, self.D,
+                                         self.in_dtype, self.out_dtype, self.timeout_ns)
+            self._args_key = key
+        args = self._args
         if dev.type == "cuda":
             with torch.cuda.device(dev):
                 self.backend.launch(args, stream if stream is not None

@@ -12,25 +12,28 @@
 // plays; blockIdx.x is the CTA within the rank):
 //   1. send: the rank's partial rows of heads owned by rank q != me are
 //      copied, 16 bytes per thread and step, into q's workspace (the slot of
-//      sender me, parity e & 1).  Each CTA owns a contiguous range of the
+//      sender me; parity e & 1 across GPUs, always slot 0 when one launch
+//      plays every rank).  Each CTA owns a contiguous range of the
 //      (q, b, head, 16-byte column) units, so consecutive threads write
 //      consecutive addresses of one receiver;
 //   2. land: after a CTA barrier, one thread makes the CTA's stores visible
-//      system-wide and adds the number of units the CTA sent to q to q's
-//      landed counter of sender me.  The count does not depend on how many
-//      CTAs the sender used, so ranks may launch different grids;
-//   3. wait: one thread per CTA polls the landed counters in me's workspace
-//      (acquire, system scope) until every sender reached e * U units (e: the
-//      number of this call, kept in the workspace header),
-//      bounded by the GPU global timer and by a poll count.  A wait that runs
-//      out sets the sender's bit in me's status word and the CTA returns
-//      without writing its outputs;
+//      (system scope; device scope when every rank is in this launch, so all
+//      readers are on this GPU) and adds the number of units the CTA sent to
+//      q to q's landed counter of sender me.  The count does not depend on
+//      how many CTAs the sender used, so ranks may launch different grids;
+//   3. wait: lane s of warp 0 of every CTA polls sender s's landed counter in
+//      me's workspace (acquire, same scope) until it reached e * U units (e:
+//      the number of this call, kept in the workspace header), all senders
+//      at once, bounded by the GPU global timer and by a poll count.  A wait
+//      that runs out sets the sender's bit in me's status word and the CTA
+//      skips its merge;
 //   4. merge: each thread merges one 16-byte column of one owned row over all
 //      senders: its own partial read in place from local_o, the others from
 //      the workspace (L2-only loads, since other SMs or GPUs wrote them during
 //      this launch), fp32 accumulation, one reciprocal, conversion;
-//   5. the rank's last CTA to finish advances the rank's call count, so the
-//      next call (or the next replay of a captured graph) is call e + 1.
+// The call number e comes from a count of arriving CTAs kept in the rank's
+// workspace, so the next call (or the next replay of a captured graph) is
+// call e + 1 without the host passing anything.
 // All CTAs of the launch are co-resident (cooperative launch), so a CTA that
 // waits never keeps a sending CTA of the same launch from running.
 //
@@ -53,6 +56,26 @@ namespace {
 
 constexpr int kMaxWorld = LSE_MERGE_CP_MAX_WORLD;
 constexpr int kSendUnroll = 4;   // 16-byte units in flight per thread while sending
+// Poll back-off of the landed-counter wait (measured on B200 with every rank
+// in one launch: 32..256 ns gave 4.43 us per call for 2 ranks of one head,
+// 64..2048 ns 4.53 us).
+constexpr unsigned kSleepMinNs = 32;
+constexpr unsigned kSleepMaxNs = 256;
+constexpr unsigned kFullMask = 0xffffffffu;
+// 256 threads per CTA (128: 5.66 vs 4.43 us for 2 ranks of one head; a
+// 64-register cap, 4 CTAs per SM: 6.15 us).
+#ifndef LSEM_CP_THREADS
+#define LSEM_CP_THREADS kCpBlock
+#endif
+constexpr int kThreads = LSEM_CP_THREADS;
+
+// Workspace header (kCpHeaderBytes): at 8*s the landed counter of sender s
+// (u64: 16-byte units received from s over all calls); the status word at
+// LSE_MERGE_CP_STATUS_OFFSET; at kArrivedOffset, on a cache line apart from
+// the landed counters (which take other ranks' atomics and polls), the
+// rank's CTA arrival count: kCallShares per call.
+constexpr int64_t kArrivedOffset = 128;
+constexpr unsigned long long kCallShares = 1ull << 20;   // > any grid: every share >= 1
 
 struct CpParams {
     const char* local_o[kMaxWorld];   // per played rank, dense [B, H, D]
@@ -65,9 +88,11 @@ struct CpParams {
     int64_t U;                        // units per (sender, receiver) pair
     int64_t rowbytes;                 // D * in_bytes
     int64_t slot_o, slot_l, o_off, l_off;
-    int64_t chunk;                    // send units per CTA
     int64_t timeout_ns, max_polls;
+    int64_t chunk;                    // send units per CTA
+    unsigned long long share, share0; // arrival shares: CTA 0 share0, the others share
     int idx32;                        // all unit indices fit in 32 bits
+    int local;                        // every rank is played by this launch (one GPU)
     uint64_t c_U, c_dv, c_Hq;         // fastdiv constants (idx32 only)
 };
 
@@ -80,6 +105,11 @@ __device__ __forceinline__ uint64_t global_ns() {
 __device__ __forceinline__ unsigned long long ld_acquire_sys(const unsigned long long* p) {
     unsigned long long v;
     asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -112,8 +142,60 @@ __device__ __forceinline__ void divmod(const CpParams& p, int64_t n, uint64_t c,
     }
 }
 
+// kSendUnroll units of one sending thread: units u, u + kThreads, ... .
+struct SendBatch {
+    uint4 x[kSendUnroll];
+    float lv[kSendUnroll];
+    int64_t rem[kSendUnroll];   // unit index inside the receiver's block
+    int64_t row[kSendUnroll];   // row (b * Hq + head) inside the receiver's block
+    int q[kSendUnroll];         // receiver, or -1 past the CTA's range
+};
+
+// Load the partial columns (and, for a row's first column, the lse) of the
+// batch at u; nothing here depends on the call number.
+__device__ __forceinline__ void load_batch(const CpParams& p, int me, int64_t u, int64_t u1,
+                                           const char* src_o, const float* src_l, SendBatch& sb) {
+#pragma unroll
+    for (int k = 0; k < kSendUnroll; ++k) {
+        const int64_t uk = u + (int64_t)k * kThreads;
+        sb.q[k] = -1;
+        sb.lv[k] = 0.f;
+        sb.rem[k] = 0;
+        sb.row[k] = 0;
+        sb.x[k] = make_uint4(0u, 0u, 0u, 0u);
+        if (uk < u1) {
+            int64_t qi, rem, row, v, b, hq;
+            divmod(p, uk, p.c_U, p.U, qi, rem);
+            divmod(p, rem, p.c_dv, p.dv, row, v);
+            divmod(p, row, p.c_Hq, p.Hq, b, hq);
+            const int q = (int)qi + ((int)qi >= me ? 1 : 0);   // receiver
+            const int64_t srow = b * p.H + (int64_t)q * p.Hq + hq;
+            sb.x[k] = ld_stream16(src_o + srow * p.rowbytes + v * 16);
+            if (v == 0) sb.lv[k] = __ldg(src_l + srow);
+            sb.q[k] = q;
+            sb.rem[k] = rem;
+            sb.row[k] = v == 0 ? row : -1;
+        }
+    }
+}
+
+// Store the batch into the receivers' slots of sender me, parity par.
+__device__ __forceinline__ void store_batch(const CpParams& p, int me, int w1, int par,
+                                            const SendBatch& sb) {
+#pragma unroll
+    for (int k = 0; k < kSendUnroll; ++k) {
+        const int q = sb.q[k];
+        if (q < 0) continue;
+        const int slot = me - (me > q ? 1 : 0);   // sender slot at q
+        const int64_t blk = (int64_t)par * w1 + slot;
+        *reinterpret_cast<uint4*>(p.ws[q] + p.o_off + blk * p.slot_o + sb.rem[k] * 16) = sb.x[k];
+        if (sb.row[k] >= 0)
+            reinterpret_cast<float*>(p.ws[q] + p.l_off + blk * p.slot_l)[sb.row[k]] = sb.lv[k];
+    }
+}
+
 template <typename TIn, typename TOut>
-__global__ void __launch_bounds__(kCpBlock) cp_exchange_merge_kernel(const __grid_constant__ CpParams p) {
+__global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __grid_constant__ CpParams p) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
     const int pr = blockIdx.y;
@@ -124,88 +206,87 @@ __global__ void __launch_bounds__(kCpBlock) cp_exchange_merge_kernel(const __gri
     const float* src_l = p.local_lse[pr];
     char* const mine = p.ws[me];
     // This call's number e (1 for the first call after the workspace was
-    // zeroed), from the count of calls this rank has completed; the last CTA
-    // of the rank to finish advances the count, after every CTA read it.
-    const unsigned long long e =
-        *reinterpret_cast<volatile const unsigned long long*>(mine + kCpEpochOffset) + 1;
-    const int par = (int)(e & 1);   // receive slot of this call
+    // zeroed): on arrival CTA c adds its share of kCallShares to the rank's
+    // arrival count (shares of one call sum to kCallShares whatever the
+    // grid), and calls of one rank are stream-ordered, so the count a CTA of
+    // call e gets back lies in [(e-1)*kCallShares, e*kCallShares).  The
+    // atomic's round trip overlaps the first partial loads.
+    __shared__ unsigned long long s_e;
+    unsigned long long arrived = 0;
+    if (threadIdx.x == 0)
+        arrived = atomicAdd(reinterpret_cast<unsigned long long*>(mine + kArrivedOffset),
+                            cta == 0 ? p.share0 : p.share);
 
-    // ---- 1. send the rows other ranks own
+    // ---- 1. send the rows other ranks own: CTA c sends units
+    // [c*chunk, (c+1)*chunk) of the rank's total.
     const int64_t total = (int64_t)w1 * p.U;
     const int64_t u0 = min(total, cta * p.chunk);
     const int64_t u1 = min(total, u0 + p.chunk);
-    for (int64_t u = u0 + threadIdx.x; u < u1; u += (int64_t)kCpBlock * kSendUnroll) {
-        uint4 x[kSendUnroll];
-        char* dst[kSendUnroll];
-        float lv[kSendUnroll];
-        float* ldst[kSendUnroll];
-#pragma unroll
-        for (int k = 0; k < kSendUnroll; ++k) {
-            const int64_t uk = u + (int64_t)k * kCpBlock;
-            dst[k] = nullptr;
-            ldst[k] = nullptr;
-            lv[k] = 0.f;
-            x[k] = make_uint4(0u, 0u, 0u, 0u);
-            if (uk < u1) {
-                int64_t qi, rem, row, v, b, hq;
-                divmod(p, uk, p.c_U, p.U, qi, rem);
-                divmod(p, rem, p.c_dv, p.dv, row, v);
-                divmod(p, row, p.c_Hq, p.Hq, b, hq);
-                const int q = (int)qi + ((int)qi >= me ? 1 : 0);   // receiver
-                const int slot = me - (me > q ? 1 : 0);            // sender slot at q
-                const int64_t srow = b * p.H + (int64_t)q * p.Hq + hq;
-                x[k] = ld_stream16(src_o + srow * p.rowbytes + v * 16);
-                const int64_t blk = (int64_t)par * w1 + slot;
-                dst[k] = p.ws[q] + p.o_off + blk * p.slot_o + rem * 16;
-                if (v == 0) {
-                    lv[k] = __ldg(src_l + srow);
-                    ldst[k] = reinterpret_cast<float*>(p.ws[q] + p.l_off + blk * p.slot_l) + row;
-                }
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < kSendUnroll; ++k) {
-            if (dst[k]) *reinterpret_cast<uint4*>(dst[k]) = x[k];
-            if (ldst[k]) *ldst[k] = lv[k];
-        }
+    int64_t u = u0 + threadIdx.x;
+    SendBatch sb;
+    load_batch(p, me, u, u1, src_o, src_l, sb);
+    // Receive slot of this call.  Ranks on different GPUs alternate two slots
+    // by the parity of e, so a rank may start call e + 1 while a peer still
+    // reads call e.  When this launch plays every rank, call e + 1 cannot
+    // start before call e has ended, one slot suffices, and the stores need
+    // not wait for e.
+    int par = 0;
+    if (!p.local) {
+        if (threadIdx.x == 0) s_e = arrived / kCallShares + 1;
+        __syncthreads();
+        par = (int)(s_e & 1);
     }
+    for (;;) {
+        store_batch(p, me, w1, par, sb);
+        u += (int64_t)kThreads * kSendUnroll;
+        if (u >= u1) break;
+        load_batch(p, me, u, u1, src_o, src_l, sb);
+    }
+    if (p.local && threadIdx.x == 0) s_e = arrived / kCallShares + 1;
 
     // ---- 2. land: publish this CTA's units to each receiver
     __syncthreads();
+    const unsigned long long e = s_e;
     if (threadIdx.x == 0 && u1 > u0) {
-        __threadfence_system();
+        // Every rank on this GPU: device scope orders the stores for all
+        // readers; otherwise the readers are other GPUs and need system scope.
+        if (p.local) __threadfence();
+        else __threadfence_system();
         for (int qi = 0; qi < w1; ++qi) {
             const int64_t lo = max(u0, (int64_t)qi * p.U), hi = min(u1, (int64_t)(qi + 1) * p.U);
             if (hi > lo) {
                 const int q = qi + (qi >= me ? 1 : 0);
-                atomicAdd_system(reinterpret_cast<unsigned long long*>(p.ws[q]) + me,
-                                 (unsigned long long)(hi - lo));
+                unsigned long long* c = reinterpret_cast<unsigned long long*>(p.ws[q]) + me;
+                if (p.local) atomicAdd(c, (unsigned long long)(hi - lo));
+                else atomicAdd_system(c, (unsigned long long)(hi - lo));
             }
         }
     }
 
     // ---- 3. wait until every sender's units of calls 1..e have landed here (bounded)
+    // Lane s of warp 0 polls sender s's counter, so the waits for all senders
+    // overlap instead of costing one memory round trip each.
     __shared__ int s_ok;
     const unsigned long long target = e * (unsigned long long)p.U;
-    if (threadIdx.x == 0) {
-        const unsigned long long* landed = reinterpret_cast<const unsigned long long*>(mine);
-        uint32_t missing = 0;
+    if (threadIdx.x < 32) {
+        const int s = threadIdx.x;
+        const unsigned long long* landed = reinterpret_cast<const unsigned long long*>(mine) + s;
+        bool ok = s >= p.world || s == me;
         int64_t polls = 0;
+        unsigned ns = kSleepMinNs;
         const uint64_t t0 = global_ns();
-        for (int s = 0; s < p.world; ++s) {
-            if (s == me) continue;
-            unsigned ns = 64;
-            while (ld_acquire_sys(landed + s) < target) {
-                if (++polls > p.max_polls || global_ns() - t0 > (uint64_t)p.timeout_ns) {
-                    missing |= 1u << s;
-                    break;
-                }
-                __nanosleep(ns);
-                if (ns < 2048) ns <<= 1;
-            }
+        for (;;) {
+            if (!ok) ok = (p.local ? ld_acquire_gpu(landed) : ld_acquire_sys(landed)) >= target;
+            if (__all_sync(kFullMask, ok)) break;
+            if (++polls > p.max_polls || global_ns() - t0 > (uint64_t)p.timeout_ns) break;
+            __nanosleep(ns);
+            if (ns < kSleepMaxNs) ns <<= 1;
         }
-        if (missing) atomicOr(reinterpret_cast<unsigned*>(mine + LSE_MERGE_CP_STATUS_OFFSET), missing);
-        s_ok = missing == 0;
+        const unsigned missing = __ballot_sync(kFullMask, !ok);   // bit s: sender s
+        if (s == 0) {
+            if (missing) atomicOr(reinterpret_cast<unsigned*>(mine + LSE_MERGE_CP_STATUS_OFFSET), missing);
+            s_ok = missing == 0;
+        }
     }
     __syncthreads();
 
@@ -213,7 +294,7 @@ __global__ void __launch_bounds__(kCpBlock) cp_exchange_merge_kernel(const __gri
     char* const dst_o = p.out_o[pr];
     float* const dst_l = p.out_lse[pr];
     const int64_t wend = s_ok ? p.U : 0;
-    for (int64_t w = cta * kCpBlock + threadIdx.x; w < wend; w += (int64_t)gridDim.x * kCpBlock) {
+    for (int64_t w = cta * kThreads + threadIdx.x; w < wend; w += (int64_t)gridDim.x * kThreads) {
         int64_t row, v, b, hq;
         divmod(p, w, p.c_dv, p.dv, row, v);
         divmod(p, row, p.c_Hq, p.Hq, b, hq);
@@ -269,16 +350,6 @@ __global__ void __launch_bounds__(kCpBlock) cp_exchange_merge_kernel(const __gri
         if (v == 0) dst_l[row] = esum > 0.f ? m + logf(esum) : -INFINITY;
     }
 
-    // ---- 5. the last CTA of this rank to finish records call e as completed
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        unsigned* done = reinterpret_cast<unsigned*>(mine + kCpDoneOffset);
-        __threadfence();
-        if (atomicAdd(done, 1u) == gridDim.x - 1) {
-            *done = 0u;
-            *reinterpret_cast<volatile unsigned long long*>(mine + kCpEpochOffset) = e;
-        }
-    }
 }
 
 using CpFn = void (*)(CpParams);
@@ -323,7 +394,7 @@ int co_resident(const void* fn, int64_t* capacity) {
             }
     }
     int per_sm = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kCpBlock, 0);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
     if (e != cudaSuccess) return (int)e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return (int)e;
@@ -379,7 +450,9 @@ int lse_merge_cp_exchange_merge(const lse_merge_cp_args* a, lse_merge_stream_t s
     // sleeps growing to ~2 us, this many polls take several times the timeout.
     kp.max_polls = a->timeout_ns / 256 + 1024;
     const int64_t send_units = (int64_t)(a->world - 1) * pl.U;
+    if (send_units >= ((int64_t)1 << 46)) return LSE_MERGE_EDIMS;   // keeps cta * total in range
     kp.idx32 = (send_units + pl.U) < ((int64_t)1 << 31);
+    kp.local = a->rank_count == a->world && !(a->flags & LSE_MERGE_CP_FLAG_CROSS_GPU_PROTOCOL);
     kp.c_U = fastdiv_c((uint32_t)(kp.idx32 ? pl.U : 1));
     kp.c_dv = fastdiv_c(kp.dv);
     kp.c_Hq = fastdiv_c((uint32_t)pl.Hq);
@@ -390,15 +463,19 @@ int lse_merge_cp_exchange_merge(const lse_merge_cp_args* a, lse_merge_stream_t s
     if (ce != 0) return fail_cuda(LSE_MERGE_ELAUNCH, ce);
     const int64_t cap = capacity / a->rank_count;
     if (cap < 1) return fail_cuda(LSE_MERGE_ELAUNCH, (int)cudaErrorCooperativeLaunchTooLarge);
+    // One CTA per kThreads units of the larger phase, at most what is
+    // co-resident.
     const int64_t work = send_units > pl.U ? send_units : pl.U;
-    int64_t ctas = (work + kCpBlock - 1) / kCpBlock;
+    int64_t ctas = (work + kThreads - 1) / kThreads;
     if (ctas > cap) ctas = cap;
     if (ctas < 1) ctas = 1;
     kp.chunk = (send_units + ctas - 1) / ctas;
+    kp.share = kCallShares / (unsigned long long)ctas;
+    kp.share0 = kCallShares - (unsigned long long)(ctas - 1) * kp.share;
 
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)ctas, (unsigned)a->rank_count, 1);
-    cfg.blockDim = dim3(kCpBlock, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];

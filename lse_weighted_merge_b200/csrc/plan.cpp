@@ -352,6 +352,7 @@ int make_cp_plan(const lse_merge_cp_args& a, CpPlan* plan) {
     if (a.rank_begin < 0 || a.rank_count < 1 || a.rank_begin + a.rank_count > a.world)
         return LSE_MERGE_EDIMS;
     if (a.timeout_ns <= 0 || a.timeout_ns > kCpMaxTimeoutNs) return LSE_MERGE_EDIMS;
+    if (a.flags & ~LSE_MERGE_CP_FLAG_CROSS_GPU_PROTOCOL) return LSE_MERGE_EDIMS;
     p.rank_begin = a.rank_begin;
     p.rank_count = a.rank_count;
     p.out_bytes = ob;

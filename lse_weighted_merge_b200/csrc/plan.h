@@ -130,12 +130,7 @@ struct CpPlan {
     int64_t ws_bytes;  // bytes of one workspace
 };
 constexpr int kCpBlock = 256;
-// Workspace header: landed counters (8 x u64) at 0, the status word at
-// LSE_MERGE_CP_STATUS_OFFSET, the rank's completed-call count (u64) and the
-// finished-CTA count of the running call (u32).
-constexpr int64_t kCpHeaderBytes = 256;
-constexpr int64_t kCpEpochOffset = 128;
-constexpr int64_t kCpDoneOffset = 136;
+constexpr int64_t kCpHeaderBytes = 256;   // counters and status word of a workspace
 constexpr int64_t kCpMaxTimeoutNs = 60ll * 1000 * 1000 * 1000;
 
 // Workspace layout for these sizes (no pointer checks).

@@ -38,8 +38,8 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_strerror():
-    assert nat.lib.lse_merge_version() == nat.ABI_VERSION == 3
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10):
+    assert nat.lib.lse_merge_version() == nat.ABI_VERSION == 4
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10, -11):
         assert nat.strerror(code) and "unknown lse_merge error" not in nat.strerror(code)
     assert "unknown lse_merge error" in nat.strerror(-99)
 

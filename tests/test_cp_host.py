@@ -48,14 +48,14 @@ def test_workspace_bytes_rejects(args, code):
 
 
 def make(world=2, rank_begin=0, rank_count=None, B=2, H=4, D=64, i=nat.BF16, o=nat.BF16,
-         timeout_ns=10**9, lo=None, ll=None, oo=None, ol=None, ws=None):
+         timeout_ns=10**9, lo=None, ll=None, oo=None, ol=None, ws=None, flags=0):
     n = world - rank_begin if rank_count is None else rank_count
     lo = lo if lo is not None else [LO + k * STEP for k in range(n)]
     ll = ll if ll is not None else [LL + k * STEP for k in range(n)]
     oo = oo if oo is not None else [OO + k * STEP for k in range(n)]
     ol = ol if ol is not None else [OL + k * STEP for k in range(n)]
     ws = ws if ws is not None else [WS + q * STEP for q in range(world)]
-    a = nat.cp_args(world, rank_begin, lo, ll, oo, ol, ws, B, H, D, i, o, timeout_ns)
+    a = nat.cp_args(world, rank_begin, lo, ll, oo, ol, ws, B, H, D, i, o, timeout_ns, flags)
     a.rank_count = n
     return a
 
@@ -65,6 +65,7 @@ def test_validate_accepts_good_arguments():
         assert nat.cp_validate(make(world=world, H=8)) == nat.OK
     assert nat.cp_validate(make(world=4, rank_begin=3, rank_count=1, H=8)) == nat.OK
     assert nat.cp_validate(make(i=nat.F32, o=nat.F16, D=4)) == nat.OK
+    assert nat.cp_validate(make(flags=nat.CP_FLAG_CROSS_GPU_PROTOCOL)) == nat.OK
     # inputs are only read: two played ranks may share one input buffer
     assert nat.cp_validate(make(lo=[LO, LO], ll=[LL, LL])) == nat.OK
 
@@ -76,6 +77,7 @@ def test_validate_accepts_good_arguments():
     (dict(rank_begin=1, rank_count=2), nat.EDIMS), (dict(rank_begin=-1, rank_count=1), nat.EDIMS),
     (dict(rank_count=0), nat.EDIMS),
     (dict(timeout_ns=0), nat.EDIMS), (dict(timeout_ns=61 * 10**9), nat.EDIMS),
+    (dict(flags=2), nat.EDIMS),
     (dict(D=4), nat.EALIGN), (dict(i=nat.F32, D=2), nat.EALIGN),
     (dict(ws=[WS, 0]), nat.ENULL), (dict(lo=[LO, 0]), nat.ENULL), (dict(ol=[0, OL]), nat.ENULL),
     (dict(ws=[WS, WS + STEP + 128]), nat.EALIGN), (dict(lo=[LO + 8, LO + STEP]), nat.EALIGN),
@@ -201,9 +203,13 @@ def _group_worker(rank, world, port, q, scenario):
         lse = torch.zeros((2, 4), dtype=torch.float32)
         out, out_lse = g(o, lse)
         res["out_shape"] = (tuple(out.shape), tuple(out_lse.shape), out.dtype == torch.bfloat16)
+        first = g._args
+        g(o, lse, out=out, out_lse=out_lse)
+        res["args_reused"] = g._args is first    # same buffers: the argument block is kept
         with pytest.raises(ValueError):
             g(o[:, :2], lse)                          # wrong shape: rejected on the host
         res["launch"] = [e for e in be.log if e[0] == "launch"]
+        assert len(res["launch"]) == 2
         g.check_peers(timeout_s=20.0)
         be.fake_status = 1 << (1 - rank)
         res["status"] = g.status()
@@ -248,9 +254,10 @@ def test_group_setup_step_status_reset_close():
         assert r["peers"][rank] == r["ws"] == WS + rank * (1 << 36)
         assert r["peers"][other] == ws_other + (1 << 35)
         assert r["out_shape"] == ((2, 2, 64), (2, 2), True)
-        (_, rc, world, begin, count, ws), = r["launch"]
-        assert (rc, world, begin, count) == (nat.OK, 2, rank, 1)
-        assert ws == r["peers"]
+        assert r["args_reused"]
+        for (_, rc, world, begin, count, ws) in r["launch"]:
+            assert (rc, world, begin, count) == (nat.OK, 2, rank, 1)
+            assert ws == r["peers"]
         assert r["status"] == 1 << other and r["raised_when_broken"]
         assert r["zeroed"] and r["zeroed"][0][1] == r["ws"] and r["after_reset"]
         assert r["teardown"] == [("close", ws_other + (1 << 35)), ("destroy", r["ws"])]

@@ -76,38 +76,56 @@ def test_exchange_merge_dtypes(in_dt, out_dt, D):
     compare(outs, inp, f"{in_dt}->{out_dt} D{D}")
 
 
+@pytest.mark.parametrize("cross", [False, True], ids=["one-gpu-protocol", "cross-gpu-protocol"])
 @pytest.mark.parametrize("name", sorted(synth.CP_WORKLOADS))
-def test_exchange_merge_workloads(name):
+def test_exchange_merge_workloads(name, cross):
     inp = inputs(name)
     lo, ll = to_device(inp)
-    outs = cp.cp_exchange_merge(lo, ll, workspaces(inp))
+    outs = cp.cp_exchange_merge(lo, ll, workspaces(inp), cross_gpu_protocol=cross)
     torch.cuda.synchronize()
     compare(outs, inp, name)
 
 
-def test_repeated_calls_alternate_slots_and_count_on_device():
+@pytest.mark.parametrize("cross", [False, True], ids=["one-gpu-protocol", "cross-gpu-protocol"])
+def test_repeated_calls_alternate_slots_and_count_on_device(cross):
     base = inputs(R=4, B=6, H=8, D=128, seed=1)
     ws = workspaces(base)
     U = base["B"] * (base["H"] // 4) * (base["D"] * 2 // 16)
     for call in range(1, 6):
         inp = inputs(R=4, B=6, H=8, D=128, seed=100 + call)
         lo, ll = to_device(inp)
-        outs = cp.cp_exchange_merge(lo, ll, ws)
+        outs = cp.cp_exchange_merge(lo, ll, ws, cross_gpu_protocol=cross)
         torch.cuda.synchronize()
         compare(outs, inp, f"call {call}")
         for q in range(4):
             hdr = ws[q][:256].view(torch.int64).cpu()
-            assert int(hdr[16]) == call                      # completed calls of rank q
             landed = [int(hdr[s]) for s in range(4)]
             assert landed == [0 if s == q else call * U for s in range(4)], (q, landed)
+            assert int(hdr[16]) == call << 20                 # rank q's arrival count
             assert cp.cp_status(ws[q]) == 0
 
 
-def test_graph_replays_are_new_calls():
+def test_prepared_call_reused_over_updated_buffers():
+    inp = inputs(R=4, B=5, H=8, D=64, seed=60)
+    lo, ll = to_device(inp)
+    call = cp.CPMergeCall(lo, ll, workspaces(inp))
+    for k in range(3):
+        nxt = inputs(R=4, B=5, H=8, D=64, seed=61 + k)
+        nlo, nll = to_device(nxt)
+        for s_ in range(4):
+            lo[s_].copy_(nlo[s_])
+            ll[s_].copy_(nll[s_])
+        outs = call()
+        torch.cuda.synchronize()
+        compare(outs, nxt, f"prepared call {k}")
+
+
+@pytest.mark.parametrize("cross", [False, True], ids=["one-gpu-protocol", "cross-gpu-protocol"])
+def test_graph_replays_are_new_calls(cross):
     inp = inputs(R=8, B=2, H=16, D=128, seed=3)
     lo, ll = to_device(inp)
     ws = workspaces(inp)
-    outs = cp.cp_exchange_merge(lo, ll, ws)                 # eager call 1
+    outs = cp.cp_exchange_merge(lo, ll, ws, cross_gpu_protocol=cross)    # eager call 1
     torch.cuda.synchronize()
     compare(outs, inp, "eager")
     g = torch.cuda.CUDAGraph()
@@ -115,7 +133,7 @@ def test_graph_replays_are_new_calls():
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
-            outs = cp.cp_exchange_merge(lo, ll, ws)
+            outs = cp.cp_exchange_merge(lo, ll, ws, cross_gpu_protocol=cross)
     torch.cuda.synchronize()
     for rep in range(3):
         nxt = inputs(R=8, B=2, H=16, D=128, seed=50 + rep)
@@ -126,7 +144,7 @@ def test_graph_replays_are_new_calls():
         g.replay()
         torch.cuda.synchronize()
         compare(outs, nxt, f"replay {rep}")
-    assert int(ws[0][:256].view(torch.int64)[16].item()) == 4
+    assert int(ws[0][:256].view(torch.int64)[16].item()) == 4 << 20     # 4 calls arrived
 
 
 def test_a_sender_that_never_sends_times_out():
@@ -145,7 +163,7 @@ def test_a_sender_that_never_sends_times_out():
     assert bool((out == 7.0).all()) and bool((out_lse == 7.0).all())
     U = 4 * 2 * (128 * 2 // 16)
     assert int(ws[1][:8].view(torch.int64).item()) == U    # rank 0's units landed at rank 1
-    assert int(ws[0][:256].view(torch.int64)[16].item()) == 1
+    assert int(ws[0][:256].view(torch.int64)[16].item()) == 1 << 20    # one call arrived
     # restart: zero every workspace, then a full call is correct again
     for w in ws:
         w.zero_()
