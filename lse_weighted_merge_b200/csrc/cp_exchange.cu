@@ -30,7 +30,7 @@
 //   4. merge: each thread merges one 16-byte column of one owned row over all
 //      senders: its own partial read in place from local_o, the others from
 //      the workspace (L2-only loads, since other SMs or GPUs wrote them during
-//      this launch), fp32 accumulation, one reciprocal, conversion;
+//      this launch), fp32 accumulation, one reciprocal, conversion.
 // The call number e comes from a count of arriving CTAs kept in the rank's
 // workspace, so the next call (or the next replay of a captured graph) is
 // call e + 1 without the host passing anything.
@@ -62,12 +62,10 @@ constexpr int kSendUnroll = 4;   // 16-byte units in flight per thread while sen
 constexpr unsigned kSleepMinNs = 32;
 constexpr unsigned kSleepMaxNs = 256;
 constexpr unsigned kFullMask = 0xffffffffu;
-// 256 threads per CTA (128: 5.66 vs 4.43 us for 2 ranks of one head; a
-// 64-register cap, 4 CTAs per SM: 6.15 us).
-#ifndef LSEM_CP_THREADS
-#define LSEM_CP_THREADS kCpBlock
-#endif
-constexpr int kThreads = LSEM_CP_THREADS;
+// Threads per CTA: kCpBlock = 256 (measured on B200 for 2 ranks of one head:
+// 128 threads 5.66 us against 4.43 us; a 64-register cap, 4 CTAs per SM,
+// 6.15 us).
+constexpr int kThreads = kCpBlock;
 
 // Workspace header (kCpHeaderBytes): at 8*s the landed counter of sender s
 // (u64: 16-byte units received from s over all calls); the status word at
