@@ -154,8 +154,9 @@ int lse_merge_plan_query(const void* partial_o, const float* partial_lse,
  *     o_acc   = (e_a * o_acc + e_n * o_new) / (e_a + e_n)
  *     lse_acc = m + log(e_a + e_n)
  *
- * and 0, -inf when both sides are empty.  An empty side is never read, so an
- * accumulator can start as lse_acc = -inf with o_acc uninitialised.  The pages
+ * and 0, -inf when both sides are empty.  The values of an empty side never
+ * reach the result (NaN there does not leak), so an accumulator can start as
+ * lse_acc = -inf with o_acc uninitialised.  The pages
  * describe the R-way merge only; this entry point is derived from it.
  *
  *   o_acc, lse_acc  device pointers, dense [B,H,D] of acc_dtype and [B,H] fp32;

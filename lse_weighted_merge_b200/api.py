@@ -196,8 +196,8 @@ def merge_state_(o_acc, lse_acc, o_new, lse_new):
     o_acc [B, H, D] (contiguous; float32 / float16 / bfloat16) and lse_acc
     [B, H] (contiguous float32) are read and overwritten with the merge of
     themselves and (o_new [B, H, D], any strides with stride 1 along D;
-    lse_new [B, H] float32).  An accumulator with lse_acc = -inf is empty: its
-    o_acc is never read.  Returns (o_acc, lse_acc).
+    lse_new [B, H] float32).  An accumulator with lse_acc = -inf is empty: the
+    values in its o_acc never reach the result.  Returns (o_acc, lse_acc).
     """
     import torch
     for t in (o_acc, lse_acc, o_new, lse_new):

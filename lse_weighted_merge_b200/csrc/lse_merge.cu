@@ -634,9 +634,20 @@ __device__ __forceinline__ void store8(char* p, int n, const float* f) {
     }
 }
 
+// 8-element chunks a lane loads before it needs any weight: both sides of
+// kStateChunks chunks are in flight while the two lse values arrive.
+// Measured on B200 (B=512 H=16 D=512, fp32 accumulator, bf16 partial): one
+// chunk 8.93 us (40 registers); two 10.11 us and four 11.03 us (more
+// registers, fewer resident warps); loads issued only after the weights
+// 10.04 us.
+constexpr int kStateChunks = 1;
+
 // A group of p.lanes lanes per row.  Lane 0 of the group reads both lse values
 // and hands them to the group by shuffle, so no lane reads lse_acc after lane
 // 0 has overwritten it; each element of o_acc is read and written by one lane.
+// The data loads do not wait for the weights: a side of weight 0 is loaded
+// but replaced by 0 before the FMA, so NaN stored there cannot reach the
+// result.
 template <typename TA, typename TN, bool VEC>
 __global__ void __launch_bounds__(kBlock) state_update_kernel(const SParams p) {
     pdl_wait();
@@ -647,6 +658,26 @@ __global__ void __launch_bounds__(kBlock) state_update_kernel(const SParams p) {
     const bool live = row < p.rows;
     const int64_t r = live ? row : 0;
     const int64_t b = r / p.H, h = r - b * p.H;
+    char* arow = p.acc + r * p.D * (int64_t)sizeof(TA);
+    const char* nrow = p.nw + b * p.n_b + h * p.n_h;
+
+    float fa[kStateChunks][8], fn[kStateChunks][8];
+    auto load_batch = [&](int c0) {
+#pragma unroll
+        for (int i = 0; i < kStateChunks; ++i) {
+            const int c = c0 + i * p.lanes;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) fa[i][k] = fn[i][k] = 0.f;
+            if (live && c < p.chunks) {
+                const int d0 = c * 8;
+                const int n = min(8, p.D - d0);
+                load8<TA, VEC, false>(arow + (int64_t)d0 * sizeof(TA), n, fa[i]);
+                load8<TN, VEC, true>(nrow + (int64_t)d0 * sizeof(TN), n, fn[i]);
+            }
+        }
+    };
+    load_batch(j);
+
     float la = -INFINITY, ln = -INFINITY;
     if (live && j == 0) {
         la = p.lse_acc[r];
@@ -660,19 +691,25 @@ __global__ void __launch_bounds__(kBlock) state_update_kernel(const SParams p) {
     const float esum = ea + en;
     const float inv = esum > 0.f ? 1.f / esum : 0.f;
     if (!live) return;
-    char* arow = p.acc + r * p.D * (int64_t)sizeof(TA);
-    const char* nrow = p.nw + b * p.n_b + h * p.n_h;
-    for (int c = j; c < p.chunks; c += p.lanes) {
-        const int d0 = c * 8;
-        const int n = min(8, p.D - d0);
-        float fa[8], fn[8], o[8];
+    for (int c0 = j;;) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) fa[k] = fn[k] = 0.f;
-        if (ea != 0.f) load8<TA, VEC, false>(arow + (int64_t)d0 * sizeof(TA), n, fa);
-        if (en != 0.f) load8<TN, VEC, true>(nrow + (int64_t)d0 * sizeof(TN), n, fn);
+        for (int i = 0; i < kStateChunks; ++i) {
+            const int c = c0 + i * p.lanes;
+            if (c < p.chunks) {
+                const int d0 = c * 8;
+                float o[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] = fmaf(ea, fa[k], en * fn[k]) * inv;
-        store8<TA, VEC>(arow + (int64_t)d0 * sizeof(TA), n, o);
+                for (int k = 0; k < 8; ++k) {
+                    const float xa = ea != 0.f ? fa[i][k] : 0.f;
+                    const float xn = en != 0.f ? fn[i][k] : 0.f;
+                    o[k] = fmaf(ea, xa, en * xn) * inv;
+                }
+                store8<TA, VEC>(arow + (int64_t)d0 * sizeof(TA), min(8, p.D - d0), o);
+            }
+        }
+        c0 += p.lanes * kStateChunks;
+        if (c0 >= p.chunks) break;
+        load_batch(c0);
     }
     if (j == 0) p.lse_acc[r] = esum > 0.f ? m + logf(esum) : -INFINITY;
 }
