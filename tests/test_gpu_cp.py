@@ -173,6 +173,40 @@ def test_a_sender_that_never_sends_times_out():
     assert cp.cp_status(ws[0]) == 0 and cp.cp_status(ws[1]) == 0
 
 
+@pytest.mark.parametrize("cross", [False, True], ids=["one-gpu-protocol", "cross-gpu-protocol"])
+@pytest.mark.parametrize("world,B,Hq,D", [(2, 3, 1, 64), (8, 5, 3, 128), (4, 2, 2, 8)])
+def test_writes_stay_inside_outputs_and_workspaces(world, B, Hq, D, cross):
+    """Outputs and workspaces are carved out of larger buffers whose guard
+    bytes hold a canary pattern; after two calls no guard byte has changed
+    (the only writes are inside the documented extents)."""
+    G = 4096                                        # guard bytes on each side
+    inp = inputs(R=world, B=B, H=world * Hq, D=D, seed=500 + world + D)
+    lo, ll = to_device(inp)
+    nbytes = nat.cp_workspace_bytes(world, B, world * Hq, D, nat.BF16)
+    canary = 0xA5
+    ws_buf = [torch.full((G + nbytes + G,), canary, dtype=torch.uint8, device="cuda")
+              for _ in range(world)]
+    for w in ws_buf:
+        w[G:G + nbytes].zero_()
+    o_bytes, l_bytes = B * Hq * D * 2, B * Hq * 4
+    out_buf = [torch.full((G + o_bytes + G,), canary, dtype=torch.uint8, device="cuda")
+               for _ in range(world)]
+    lse_buf = [torch.full((G + l_bytes + G,), canary, dtype=torch.uint8, device="cuda")
+               for _ in range(world)]
+    outs = [(o[G:G + o_bytes].view(torch.bfloat16).view(B, Hq, D),
+             l[G:G + l_bytes].view(torch.float32).view(B, Hq)) for o, l in zip(out_buf, lse_buf)]
+    for _ in range(2):
+        cp.cp_exchange_merge(lo, ll, [w[G:G + nbytes] for w in ws_buf], outs=outs,
+                             cross_gpu_protocol=cross)
+    torch.cuda.synchronize()
+    compare(outs, inp, "guarded")
+    for name, bufs, n in (("workspace", ws_buf, nbytes), ("out", out_buf, o_bytes),
+                          ("out_lse", lse_buf, l_bytes)):
+        for q, buf in enumerate(bufs):
+            assert bool((buf[:G] == canary).all()), f"{name} {q}: write before the buffer"
+            assert bool((buf[G + n:] == canary).all()), f"{name} {q}: write past the buffer"
+
+
 def test_rejected_arguments_raise():
     inp = inputs(R=2, B=1, H=2, D=64, seed=0)
     lo, ll = to_device(inp)

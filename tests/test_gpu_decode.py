@@ -235,3 +235,34 @@ def test_automatic_splits_and_fusion(B, Hq, Hkv, L):
     torch.cuda.synchronize()
     want, want_lse, vmax = reference(q, k, v, 1 / math.sqrt(D), [L] * B)
     check_rows(out.cpu(), lse.cpu(), want, want_lse, vmax, "bf16", "bf16", "auto")
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "partials"])
+def test_outputs_written_exactly_in_bounds(fused):
+    """Outputs carved out of larger buffers with canary guard bytes: after a
+    call no guard byte has changed and q, k, v are left as they were."""
+    B, Hq, Hkv, L, D, R = 2, 8, 2, 300, 128, 4
+    q, k, v = make(B, Hq, Hkv, L, D, seed=77)
+    scale = 1 / math.sqrt(D)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    q0, k0, v0 = qd.clone(), kd.clone(), vd.clone()
+    G, canary = 4096, 0x3C
+    o_bytes = B * Hq * D * 2 if fused else B * Hq * R * D * 4
+    l_bytes = B * Hq * 4 if fused else B * Hq * R * 4
+    o_buf = torch.full((G + o_bytes + G,), canary, dtype=torch.uint8, device="cuda")
+    l_buf = torch.full((G + l_bytes + G,), canary, dtype=torch.uint8, device="cuda")
+    st = (qd.stride(0), qd.stride(1), kd.stride(0), kd.stride(1), kd.stride(2),
+          vd.stride(0), vd.stride(1), vd.stride(2))
+    nat.decode_raw(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), 0, B, Hq, Hkv, L, D, R, scale, st,
+                   nat.BF16, o_buf.data_ptr() + G, l_buf.data_ptr() + G,
+                   torch.cuda.current_stream().cuda_stream, fused=fused,
+                   **({"out_dtype": nat.BF16} if fused else {}))
+    torch.cuda.synchronize()
+    for buf, n in ((o_buf, o_bytes), (l_buf, l_bytes)):
+        assert bool((buf[:G] == canary).all()) and bool((buf[G + n:] == canary).all())
+    assert torch.equal(qd, q0) and torch.equal(kd, k0) and torch.equal(vd, v0)
+    if fused:
+        out = o_buf[G:G + o_bytes].view(torch.bfloat16).view(B, Hq, D).cpu()
+        lse = l_buf[G:G + l_bytes].view(torch.float32).view(B, Hq).cpu()
+        want, want_lse, vmax = reference(q, k, v, scale, [L] * B)
+        check_rows(out, lse, want, want_lse, vmax, "bf16", "bf16", "guarded fused")

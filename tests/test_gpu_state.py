@@ -110,3 +110,35 @@ def test_large_state_update_full_parity():
     want, want_lse = oracle.state_update(acc, la, oracle.F32, new, ln, oracle.BF16, B, H, D)
     got, got_lse = run(acc, la, new, ln, B, H, D, "f32", "bf16")
     check(got, got_lse, want, want_lse, "f32", "large")
+
+
+@pytest.mark.parametrize("acc_dt,D", [("f32", 96), ("bf16", 100), ("f16", 8)])
+def test_writes_stay_inside_the_accumulator(acc_dt, D):
+    """The accumulator and its lse are carved out of larger buffers whose
+    guard bytes hold a canary pattern: after a fold no guard byte has
+    changed, and the new partial and its lse are left as they were."""
+    B, H, G = 5, 3, 4096
+    acc, la, new, ln = make(B, H, D, acc_dt, "bf16", seed=D)
+    want, want_lse = oracle.state_update(acc, la, synth.DTYPES[acc_dt], new, ln, synth.DTYPES["bf16"],
+                                         B, H, D)
+    raw = torch.from_numpy(acc.view(np.uint8).copy())
+    canary = 0x5A
+    a_buf = torch.full((G + raw.numel() + G,), canary, dtype=torch.uint8)
+    a_buf[G:G + raw.numel()] = raw
+    l_raw = torch.from_numpy(la.view(np.uint8).copy())
+    l_buf = torch.full((G + l_raw.numel() + G,), canary, dtype=torch.uint8)
+    l_buf[G:G + l_raw.numel()] = l_raw
+    a_buf, l_buf = a_buf.cuda(), l_buf.cuda()
+    d_new, d_ln = dev(new), dev(ln)
+    new0, ln0 = d_new.clone(), d_ln.clone()
+    nat.state_update_raw(a_buf.data_ptr() + G, l_buf.data_ptr() + G, d_new.data_ptr(), d_ln.data_ptr(),
+                         B, H, D, None, synth.DTYPES[acc_dt], synth.DTYPES["bf16"],
+                         torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    n = raw.numel()
+    assert bool((a_buf[:G] == canary).all()) and bool((a_buf[G + n:] == canary).all())
+    assert bool((l_buf[:G] == canary).all()) and bool((l_buf[G + l_raw.numel():] == canary).all())
+    assert torch.equal(d_new, new0) and torch.equal(d_ln, ln0)
+    got = a_buf[G:G + n].view(TORCH_DT[acc_dt]).double().cpu().numpy().reshape(B, H, D)
+    got_lse = l_buf[G:G + l_raw.numel()].view(torch.float32).double().cpu().numpy().reshape(B, H)
+    check(got, got_lse, want, want_lse, acc_dt, f"guarded {acc_dt} D{D}")
