@@ -144,6 +144,11 @@ class NativeBackend:
     close = staticmethod(_native.cp_ipc_close)
 
     @staticmethod
+    def device():
+        import torch
+        return torch.cuda.current_device()
+
+    @staticmethod
     def launch(args, stream: int) -> None:
         _native.cp_exchange_merge_raw(args, stream)
 
@@ -154,10 +159,14 @@ class CPExchangeMerge:
     Construction is collective: every rank allocates its workspace on its
     current CUDA device, the ranks check that they agree on (B, H, D, dtypes)
     and exchange CUDA IPC handles, and each maps its peers' workspaces.  Each
-    call then launches one kernel on the rank's current stream that stores
-    the rows other ranks own into their workspaces over NVLink and merges the
-    rows this rank owns.  The group itself is only used on the host (set-up,
-    ``check_peers``, ``reset``, ``close``); no collective runs per step.
+    step of the set-up shares its local outcome with the other ranks, so a
+    failure on one rank (a bad shape, an allocation, an IPC mapping) makes
+    every rank raise, after releasing what it had set up, instead of leaving
+    the others waiting in the next collective.  Each call then launches one
+    kernel on the rank's current stream that stores the rows other ranks own
+    into their workspaces over NVLink and merges the rows this rank owns.
+    The group itself is only used on the host (set-up, ``check_peers``,
+    ``reset``, ``close``); no collective runs per step.
 
     A peer that never sends makes this rank's kernel give up after
     ``timeout_s`` (its outputs stay unwritten); ``status()`` then reads
@@ -171,32 +180,78 @@ class CPExchangeMerge:
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
-        if not 1 <= self.world <= _native.CP_MAX_WORLD:
-            raise ValueError(f"world size {self.world} outside 1..{_native.CP_MAX_WORLD}")
         self.B, self.H, self.D = int(B), int(H), int(D)
         self.in_dtype = dtype_code(dtype)
         self.out_dtype = dtype_code(out_dtype or dtype)
         self.timeout_ns = int(timeout_s * 1e9)
         self.backend = backend or NativeBackend()
+        self.device = self.backend.device()
         self.broken = False
         self.calls = 0
         self._checks = 0
         self._args_key = None
         self._args = None
+        self.ws = None
+        self.peers = []
+
+        # 1. the same problem on every rank, and one this library can run
+        err = None
+        try:
+            if not 1 <= self.world <= _native.CP_MAX_WORLD:
+                raise ValueError(f"world size {self.world} outside 1..{_native.CP_MAX_WORLD}")
+            if self.H % self.world:
+                raise ValueError(f"H = {self.H} is not a multiple of world = {self.world}")
+            self.nbytes = self.backend.workspace_bytes(self.world, self.B, self.H, self.D,
+                                                       self.in_dtype)
+        except Exception as exc:   # shared with the other ranks below, then raised everywhere
+            err = f"rank {self.rank}: {exc}"
         me = (self.B, self.H, self.D, self.in_dtype, self.out_dtype, self.timeout_ns)
-        every = [None] * self.world
-        dist.all_gather_object(every, me, group=group)
-        if any(x != me for x in every):
-            raise ValueError(f"ranks disagree on (B, H, D, dtypes, timeout): {every}")
-        if self.H % self.world:
-            raise ValueError(f"H = {self.H} is not a multiple of world = {self.world}")
-        self.nbytes = self.backend.workspace_bytes(self.world, self.B, self.H, self.D, self.in_dtype)
-        self.ws = self.backend.create(self.nbytes)
-        handles = [None] * self.world
-        dist.all_gather_object(handles, self.backend.handle(self.ws), group=group)
-        self.peers = [self.ws if q == self.rank else self.backend.open(handles[q])
-                      for q in range(self.world)]
-        dist.barrier(group=group)
+        every = self._gather((me, err))
+        errors = [e for _, e in every if e]
+        if errors:
+            raise ValueError("; ".join(errors))
+        if any(x != me for x, _ in every):
+            raise ValueError(f"ranks disagree on (B, H, D, dtypes, timeout): {[x for x, _ in every]}")
+
+        # 2. this rank's workspace and its IPC handle
+        handle, err = None, None
+        try:
+            self.ws = self.backend.create(self.nbytes)
+            handle = self.backend.handle(self.ws)
+        except Exception as exc:
+            err = f"rank {self.rank}: workspace: {exc}"
+        every = self._gather((handle, err))
+        errors = [e for _, e in every if e]
+        if errors:
+            self._release()
+            raise RuntimeError("; ".join(errors))
+
+        # 3. the peers' workspaces mapped here
+        err = None
+        try:
+            for q in range(self.world):
+                self.peers.append(self.ws if q == self.rank else self.backend.open(every[q][0]))
+        except Exception as exc:
+            err = f"rank {self.rank}: mapping a peer's workspace: {exc}"
+        errors = [e for e in self._gather(err) if e]
+        if errors:
+            self._release()
+            raise RuntimeError("; ".join(errors))
+
+    def _gather(self, obj) -> list:
+        out = [None] * self.world
+        self.dist.all_gather_object(out, obj, group=self.group)
+        return out
+
+    def _release(self) -> None:
+        """Unmap the peers' workspaces and free this rank's (local, no collective)."""
+        for q, p in enumerate(self.peers):
+            if q != self.rank:
+                self.backend.close(p)
+        self.peers = []
+        if self.ws is not None:
+            self.backend.destroy(self.ws)
+            self.ws = None
 
     def __call__(self, local_o, local_lse, out=None, out_lse=None, stream: int | None = None):
         """Send this rank's partials (local_o [B, H, D], local_lse [B, H]) and
@@ -204,9 +259,13 @@ class CPExchangeMerge:
         import torch
         if self.broken:
             raise RuntimeError("a wait ran out in an earlier call: call reset() on every rank")
+        if self.ws is None:
+            raise RuntimeError("this exchange has been closed")
         Hq = self.H // self.world
         dev = local_o.device
         _check_local(local_o, local_lse, self.B, self.H, self.D, _torch_dtype(self.in_dtype))
+        if self.device is not None and dev.index != self.device:
+            raise ValueError(f"local_o is on {dev}, the workspace on cuda:{self.device}")
         if out is None:
             out = torch.empty((self.B, Hq, self.D), dtype=_torch_dtype(self.out_dtype), device=dev)
         if out_lse is None:
@@ -258,12 +317,14 @@ class CPExchangeMerge:
         self.calls = 0
 
     def close(self) -> None:
-        """Collective: unmap the peers' workspaces, then free this rank's."""
+        """Collective: every rank unmaps its peers' workspaces, then, once all
+        have, frees its own."""
         if self.ws is None:
             return
         for q, p in enumerate(self.peers):
             if q != self.rank:
                 self.backend.close(p)
+        self.peers = [self.ws]
         self.dist.barrier(group=self.group)
         self.backend.destroy(self.ws)
         self.ws = None

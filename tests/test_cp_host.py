@@ -128,11 +128,18 @@ class FakeBackend:
         self.base = WS + rank * (1 << 36)
         self.log = []
         self.fake_status = 0
+        self.fail_create = False
+        self.fail_open = False
 
     def workspace_bytes(self, *a):
         return nat.cp_workspace_bytes(*a)
 
+    def device(self):
+        return None     # CPU tensors: no device to match
+
     def create(self, nbytes):
+        if self.fail_create:
+            raise MemoryError("no device memory left")
         self.log.append(("create", nbytes))
         return self.base
 
@@ -140,6 +147,8 @@ class FakeBackend:
         return ptr.to_bytes(8, "little") + bytes(nat.CP_IPC_HANDLE_BYTES - 8)
 
     def open(self, handle):
+        if self.fail_open:
+            raise OSError("cannot map the peer's memory")
         assert len(handle) == nat.CP_IPC_HANDLE_BYTES
         ptr = int.from_bytes(handle[:8], "little") + (1 << 35)   # mapped at another address
         self.log.append(("open", ptr))
@@ -183,10 +192,14 @@ def _group_worker(rank, world, port, q, scenario):
     try:
         be = FakeBackend(rank)
         H = 8 if (scenario == "mismatch" and rank == 1) else 4
+        D = 4 if (scenario == "bad_shape" and rank == 0) else 64
+        be.fail_create = scenario == "create_fails" and rank == 1
+        be.fail_open = scenario == "open_fails" and rank == 0
         try:
-            g = cp.CPExchangeMerge(2, H, 64, torch.bfloat16, backend=be)
-        except ValueError as exc:
-            res["error"] = str(exc)
+            g = cp.CPExchangeMerge(2, H, D, torch.bfloat16, backend=be)
+        except (ValueError, RuntimeError) as exc:
+            res["error"] = f"{type(exc).__name__}: {exc}"
+            res["log"] = list(be.log)
             q.put(res)
             return
         res["peers"] = list(g.peers)
@@ -267,6 +280,26 @@ def test_group_rejects_disagreeing_shapes_on_every_rank():
     res, codes = _run_group("mismatch")
     assert codes == [0, 0]
     assert all("disagree" in r.get("error", "") for r in res), res
+
+
+@pytest.mark.parametrize("scenario,kind,words", [
+    ("bad_shape", "ValueError", "rank 0"),
+    ("create_fails", "RuntimeError", "rank 1: workspace"),
+    ("open_fails", "RuntimeError", "rank 0: mapping"),
+])
+def test_a_set_up_failure_on_one_rank_raises_on_every_rank(scenario, kind, words):
+    """No rank is left waiting in a collective: every rank raises the same
+    error, and a rank that had created its workspace frees it again."""
+    res, codes = _run_group(scenario)
+    assert codes == [0, 0]
+    for r in res:
+        assert r.get("error", "").startswith(kind) and words in r["error"], r
+        created = [e for e in r["log"] if e[0] == "create"]
+        freed = [e for e in r["log"] if e[0] == "destroy"]
+        assert len(created) == len(freed), r["log"]
+        opened = [e for e in r["log"] if e[0] == "open"]
+        closed = [e for e in r["log"] if e[0] == "close"]
+        assert len(opened) == len(closed), r["log"]
 
 
 def test_group_reports_a_lost_peer():
