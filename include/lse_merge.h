@@ -275,7 +275,8 @@ int lse_merge_decode_attention(const void* q, const void* k, const void* v, cons
  * peers' workspaces (lse_merge_cp_ipc_open).
  *
  * Requirements: 1 <= world <= LSE_MERGE_CP_MAX_WORLD; H % world == 0;
- * D * elem(in_dtype) a multiple of 16 bytes; 0 <= rank_begin and
+ * D * elem(in_dtype) a multiple of 16 bytes; B*H*D*elem(in_dtype) below
+ * 32 GiB (2^31 units of 16 bytes); 0 <= rank_begin and
  * rank_begin + rank_count <= world; local_o and out_o 16-byte aligned, lse
  * pointers 4-byte aligned, workspaces 256-byte aligned and
  * lse_merge_cp_workspace_bytes() long (zeroed before the first call);

@@ -89,9 +89,8 @@ struct CpParams {
     int64_t timeout_ns, max_polls;
     int64_t chunk;                    // send units per CTA
     unsigned long long share, share0; // arrival shares: CTA 0 share0, the others share
-    int idx32;                        // all unit indices fit in 32 bits
     int local;                        // every rank is played by this launch (one GPU)
-    uint64_t c_U, c_dv, c_Hq;         // fastdiv constants (idx32 only)
+    uint64_t c_U, c_dv, c_Hq;         // fastdiv constants of U, dv and Hq
 };
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -127,17 +126,12 @@ __device__ __forceinline__ float ld_cg_f32(const float* p) {
     return v;
 }
 
-// n / d and n % d, through the 32-bit constant division when idx32.
-__device__ __forceinline__ void divmod(const CpParams& p, int64_t n, uint64_t c, int64_t d,
-                                       int64_t& q, int64_t& r) {
-    if (p.idx32) {
-        const uint32_t qq = fastdiv((uint32_t)n, c, (uint32_t)d);
-        q = qq;
-        r = (int64_t)((uint32_t)n - qq * (uint32_t)d);
-    } else {
-        q = n / d;
-        r = n - q * d;
-    }
+// n / d and n % d by the 32-bit constant division: the planner keeps every
+// unit index below 2^31.
+__device__ __forceinline__ void divmod(int64_t n, uint64_t c, int64_t d, int64_t& q, int64_t& r) {
+    const uint32_t qq = fastdiv((uint32_t)n, c, (uint32_t)d);
+    q = qq;
+    r = (int64_t)((uint32_t)n - qq * (uint32_t)d);
 }
 
 // kSendUnroll units of one sending thread: units u, u + kThreads, ... .
@@ -163,9 +157,9 @@ __device__ __forceinline__ void load_batch(const CpParams& p, int me, int64_t u,
         sb.x[k] = make_uint4(0u, 0u, 0u, 0u);
         if (uk < u1) {
             int64_t qi, rem, row, v, b, hq;
-            divmod(p, uk, p.c_U, p.U, qi, rem);
-            divmod(p, rem, p.c_dv, p.dv, row, v);
-            divmod(p, row, p.c_Hq, p.Hq, b, hq);
+            divmod(uk, p.c_U, p.U, qi, rem);
+            divmod(rem, p.c_dv, p.dv, row, v);
+            divmod(row, p.c_Hq, p.Hq, b, hq);
             const int q = (int)qi + ((int)qi >= me ? 1 : 0);   // receiver
             const int64_t srow = b * p.H + (int64_t)q * p.Hq + hq;
             sb.x[k] = ld_stream16(src_o + srow * p.rowbytes + v * 16);
@@ -294,8 +288,8 @@ __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __gri
     const int64_t wend = s_ok ? p.U : 0;
     for (int64_t w = cta * kThreads + threadIdx.x; w < wend; w += (int64_t)gridDim.x * kThreads) {
         int64_t row, v, b, hq;
-        divmod(p, w, p.c_dv, p.dv, row, v);
-        divmod(p, row, p.c_Hq, p.Hq, b, hq);
+        divmod(w, p.c_dv, p.dv, row, v);
+        divmod(row, p.c_Hq, p.Hq, b, hq);
         const int64_t srow = b * p.H + (int64_t)me * p.Hq + hq;
         uint4 x[kMaxWorld];
         float l[kMaxWorld];
@@ -448,10 +442,8 @@ int lse_merge_cp_exchange_merge(const lse_merge_cp_args* a, lse_merge_stream_t s
     // sleeps growing to ~2 us, this many polls take several times the timeout.
     kp.max_polls = a->timeout_ns / 256 + 1024;
     const int64_t send_units = (int64_t)(a->world - 1) * pl.U;
-    if (send_units >= ((int64_t)1 << 46)) return LSE_MERGE_EDIMS;   // keeps cta * total in range
-    kp.idx32 = (send_units + pl.U) < ((int64_t)1 << 31);
     kp.local = a->rank_count == a->world && !(a->flags & LSE_MERGE_CP_FLAG_CROSS_GPU_PROTOCOL);
-    kp.c_U = fastdiv_c((uint32_t)(kp.idx32 ? pl.U : 1));
+    kp.c_U = fastdiv_c((uint32_t)pl.U);
     kp.c_dv = fastdiv_c(kp.dv);
     kp.c_Hq = fastdiv_c((uint32_t)pl.Hq);
 

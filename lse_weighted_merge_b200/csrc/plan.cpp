@@ -328,6 +328,9 @@ int cp_layout(int world, int B, int H, int D, int in_dtype, CpPlan* plan) {
     const i128 l_off = up(o_off + n * slot_o);
     const i128 total = up(l_off + n * slot_l);
     if ((i128)B * H * D * ib > lim || total > lim) return LSE_MERGE_EDIMS;
+    // every 16-byte unit index of the kernel fits in 31 bits (32 GiB of
+    // partials per rank)
+    if ((i128)world * B * (H / world) * (D * ib / 16) >= ((i128)1 << 31)) return LSE_MERGE_EDIMS;
     CpPlan p{};
     p.world = world;
     p.Hq = Hq;
