@@ -321,9 +321,12 @@ int lse_merge_cp_exchange_merge(const lse_merge_cp_args* args, lse_merge_stream_
  * and create is the one place the library allocates.  They return
  * LSE_MERGE_ECUDA when the CUDA call fails (lse_merge_last_cuda_error). */
 int lse_merge_cp_workspace_create(int64_t bytes, void** ws);
-/* The status word of a workspace (a synchronous copy; 0 = no wait ran out,
- * bit s = sender s never landed) and the restart after a wait ran out:
- * zero `bytes` of the workspace, synchronously. */
+/* The status word of a workspace (0 = no wait ran out, bit s = sender s never
+ * landed) and the restart after a wait ran out: zero `bytes` of the
+ * workspace.  Both first wait for all work on the current device, on every
+ * stream, then copy or zero synchronously.  Before zeroing, every rank must
+ * also know that no peer's kernel still writes into this workspace (the
+ * Python group synchronises every device, then passes a barrier). */
 int lse_merge_cp_status(const void* ws, uint32_t* status);
 int lse_merge_cp_workspace_zero(void* ws, int64_t bytes);
 int lse_merge_cp_workspace_destroy(void* ws);

@@ -149,6 +149,11 @@ class NativeBackend:
         return torch.cuda.current_device()
 
     @staticmethod
+    def sync() -> None:
+        import torch
+        torch.cuda.synchronize()
+
+    @staticmethod
     def launch(args, stream: int) -> None:
         _native.cp_exchange_merge_raw(args, stream)
 
@@ -309,7 +314,11 @@ class CPExchangeMerge:
             raise PeerLost(f"ranks {missing} did not check in within {timeout_s} s") from exc
 
     def reset(self) -> None:
-        """Collective restart after a wait ran out: zero every workspace."""
+        """Collective restart after a wait ran out: once no rank's kernel
+        runs any more (each synchronises its device, then all pass a
+        barrier), every rank zeroes its workspace; a second barrier keeps any
+        rank from sending into a workspace not yet zeroed."""
+        self.backend.sync()
         self.dist.barrier(group=self.group)
         self.backend.zero(self.ws, self.nbytes)
         self.dist.barrier(group=self.group)
@@ -321,6 +330,7 @@ class CPExchangeMerge:
         have, frees its own."""
         if self.ws is None:
             return
+        self.backend.sync()            # none of this rank's kernels still writes to a peer
         for q, p in enumerate(self.peers):
             if q != self.rank:
                 self.backend.close(p)

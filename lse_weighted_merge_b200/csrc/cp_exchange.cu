@@ -496,8 +496,11 @@ int lse_merge_cp_workspace_create(int64_t bytes, void** ws) {
 
 int lse_merge_cp_status(const void* ws, uint32_t* status) {
     if (!ws || !status) return LSE_MERGE_ENULL;
-    const cudaError_t e = cudaMemcpy(status, static_cast<const char*>(ws) + LSE_MERGE_CP_STATUS_OFFSET,
-                                     sizeof(uint32_t), cudaMemcpyDeviceToHost);
+    // every call already enqueued on the device, on any stream, first
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(status, static_cast<const char*>(ws) + LSE_MERGE_CP_STATUS_OFFSET,
+                       sizeof(uint32_t), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
     return LSE_MERGE_OK;
 }
@@ -505,7 +508,8 @@ int lse_merge_cp_status(const void* ws, uint32_t* status) {
 int lse_merge_cp_workspace_zero(void* ws, int64_t bytes) {
     if (!ws) return LSE_MERGE_ENULL;
     if (bytes < lsem::kCpHeaderBytes) return LSE_MERGE_EDIMS;
-    cudaError_t e = cudaMemset(ws, 0, (size_t)bytes);
+    cudaError_t e = cudaDeviceSynchronize();   // no call of this device still uses it
+    if (e == cudaSuccess) e = cudaMemset(ws, 0, (size_t)bytes);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return lsem::fail_cuda(LSE_MERGE_ECUDA, (int)e);
     return LSE_MERGE_OK;

@@ -168,6 +168,9 @@ class FakeBackend:
     def zero(self, ptr, nbytes):
         self.log.append(("zero", ptr, nbytes))
 
+    def sync(self):
+        self.log.append(("sync",))
+
     def status(self, ptr):
         return self.fake_status
 
@@ -239,6 +242,8 @@ def _group_worker(rank, world, port, q, scenario):
         g.reset()
         be.fake_status = 0
         res["zeroed"] = [e for e in be.log if e[0] == "zero"]
+        res["synced_before_zero"] = [e[0] for e in be.log].index("sync") < \
+            [e[0] for e in be.log].index("zero")
         res["after_reset"] = g.status() == 0 and not g.broken
         g(o, lse)
         g.close()
@@ -278,6 +283,7 @@ def test_group_setup_step_status_reset_close():
             assert ws == r["peers"]
         assert r["status"] == 1 << other and r["raised_when_broken"]
         assert r["zeroed"] and r["zeroed"][0][1] == r["ws"] and r["after_reset"]
+        assert r["synced_before_zero"]
         assert r["teardown"] == [("close", ws_other + (1 << 35)), ("destroy", r["ws"])]
 
 
