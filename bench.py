@@ -221,6 +221,18 @@ def profiled_traffic(workload: str):
         return None, "summary has no dram_bytes_per_launch"
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -433,7 +445,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(w, args.gpus, "no GPU (host cores)"),
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         "cpu": cpu_model(), "host_cores": os.cpu_count()},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -520,7 +533,8 @@ def run_ours(args):
         bps, passes, secs = oracle_seconds(smp, args.cpu_seconds)
         cpu = {"value": bps / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": (f"first {batches} of {w.B} batches ({batches * w.H} of {w.rows} rows), "
-                          f"{passes} passes in {secs:.1f} s, fp64 C oracle, single thread")}
+                          f"{passes} passes in {secs:.1f} s, fp64 C oracle, single thread"),
+               "cpu": cpu_model(), "host_cores": os.cpu_count()}
 
     if dist is not None:
         barrier(dist, device)
