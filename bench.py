@@ -261,7 +261,7 @@ class DeviceSets:
         self.lse = [host_l.to(device) for _ in range(n)]
         self.out = [torch.empty((self.B, self.H, self.D), dtype=out_dt, device=device) for _ in range(n)]
         self.out_lse = [torch.empty((self.B, self.H), dtype=torch.float32, device=device) for _ in range(n)]
-        self.strides = nat.Strides(*inp["o_strides"], *inp["lse_strides"])
+        self.strides = (*inp["o_strides"], *inp["lse_strides"])
         self.ind = synth.DTYPES[inp["in_dtype"]]
         self.outd = synth.DTYPES[inp["out_dtype"]]
         self.n = n
@@ -271,8 +271,8 @@ class DeviceSets:
     def launch(self, i: int, stream_handle: int):
         from lse_weighted_merge_b200 import _native as nat
         o, l, out, ol = self.args[i % self.n]
-        rc = nat.lib.lse_merge(o, l, self.R, self.B, self.H, self.D, self.strides, self.ind,
-                               self.outd, out, ol, stream_handle or None)
+        rc = nat.merge_raw(o, l, self.R, self.B, self.H, self.D, self.strides, self.ind,
+                           self.outd, out, ol, stream_handle, check=False)
         if rc != 0:
             raise RuntimeError(f"lse_merge returned {rc}: {nat.strerror(rc)}")
 

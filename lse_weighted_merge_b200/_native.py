@@ -152,6 +152,14 @@ def _load() -> ctypes.CDLL:
 
 lib = _load()
 
+# Vectorcall forwarding of the per-call entry points (csrc/pyfast.c), built
+# next to the library; it calls the same C functions for a fraction of
+# ctypes' marshalling cost.  Without it the ctypes calls below are used.
+try:
+    from . import _fast
+except ImportError:
+    _fast = None
+
 
 def strerror(code: int) -> str:
     return lib.lse_merge_strerror(int(code)).decode()
@@ -162,16 +170,31 @@ def _strides(s) -> ctypes.POINTER(Strides) | None:
         return None
     if isinstance(s, Strides):
         return ctypes.pointer(s)
+    return ctypes.pointer(Strides(*[int(x) for x in _stride_tuple(s)]))
+
+
+def _stride_tuple(s):
+    """Strides as the flat (o_r, o_b, o_h, lse_r, lse_b, lse_h) tuple, or None."""
+    if s is None:
+        return None
+    if isinstance(s, Strides):
+        return (s.o_r, s.o_b, s.o_h, s.lse_r, s.lse_b, s.lse_h)
+    if len(s) == 6:
+        return tuple(s)
     o, l = s
-    return ctypes.pointer(Strides(*[int(x) for x in o], *[int(x) for x in l]))
+    return (*[int(x) for x in o], *[int(x) for x in l])
 
 
 def merge_raw(o_ptr: int, lse_ptr: int, R: int, B: int, H: int, D: int, strides,
               in_dtype: int, out_dtype: int, out_ptr: int, out_lse_ptr: int, stream: int = 0,
               path: int = PATH_AUTO, check: bool = True) -> int:
     """Call lse_merge_with_path on raw device pointers; raises on error if ``check``."""
-    rc = lib.lse_merge_with_path(o_ptr, lse_ptr, R, B, H, D, _strides(strides), in_dtype,
-                                 out_dtype, out_ptr, out_lse_ptr, stream or None, path)
+    if _fast is not None:
+        rc = _fast.merge(o_ptr, lse_ptr, R, B, H, D, _stride_tuple(strides), in_dtype, out_dtype,
+                         out_ptr, out_lse_ptr, stream or 0, path)
+    else:
+        rc = lib.lse_merge_with_path(o_ptr, lse_ptr, R, B, H, D, _strides(strides), in_dtype,
+                                     out_dtype, out_ptr, out_lse_ptr, stream or None, path)
     if check and rc != OK:
         extra = ""
         if rc == ELAUNCH:
@@ -194,9 +217,14 @@ def state_update_raw(acc_ptr: int, lse_acc_ptr: int, new_ptr: int, lse_new_ptr: 
                      H: int, D: int, new_strides, acc_dtype: int, new_dtype: int,
                      stream: int = 0, check: bool = True) -> int:
     """Call lse_merge_state_update; ``new_strides`` = (o_b, o_h, lse_b, lse_h) or None."""
-    st = None if new_strides is None else ctypes.pointer(StateStrides(*[int(x) for x in new_strides]))
-    rc = lib.lse_merge_state_update(acc_ptr, lse_acc_ptr, new_ptr, lse_new_ptr, B, H, D, st,
-                                    acc_dtype, new_dtype, stream or None)
+    if _fast is not None:
+        st = None if new_strides is None else tuple(int(x) for x in new_strides)
+        rc = _fast.state_update(acc_ptr, lse_acc_ptr, new_ptr, lse_new_ptr, B, H, D, st,
+                                acc_dtype, new_dtype, stream or 0)
+    else:
+        st = None if new_strides is None else ctypes.pointer(StateStrides(*[int(x) for x in new_strides]))
+        rc = lib.lse_merge_state_update(acc_ptr, lse_acc_ptr, new_ptr, lse_new_ptr, B, H, D, st,
+                                        acc_dtype, new_dtype, stream or None)
     if check and rc != OK:
         extra = ""
         if rc == ELAUNCH:
@@ -252,7 +280,10 @@ def cp_validate(args: CpArgs) -> int:
 
 
 def cp_exchange_merge_raw(args: CpArgs, stream: int = 0, check: bool = True) -> int:
-    rc = lib.lse_merge_cp_exchange_merge(ctypes.byref(args), stream or None)
+    if _fast is not None:
+        rc = _fast.cp_exchange_merge(ctypes.addressof(args), stream or 0)
+    else:
+        rc = lib.lse_merge_cp_exchange_merge(ctypes.byref(args), stream or None)
     if check and rc != OK:
         _raise(rc)
     return rc

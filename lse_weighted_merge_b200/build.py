@@ -1,4 +1,5 @@
-"""Build the C-ABI shared library (liblse_merge.so) in-tree with nvcc for sm_100a.
+"""Build the C-ABI shared library (liblse_merge.so) in-tree with nvcc for sm_100a,
+and the small CPython extension (_fast) that forwards its per-call entry points.
 
     python -m lse_weighted_merge_b200.build [--verbose]
 """
@@ -36,6 +37,27 @@ def stale(out: str = LIB) -> bool:
     return any(os.path.getmtime(s) > t for s in SOURCES + HEADERS)
 
 
+FAST_SRC = os.path.join(CSRC, "pyfast.c")
+
+
+def fast_path() -> str:
+    """In-tree path of the CPython extension that forwards the per-call entry points."""
+    import sysconfig
+    return os.path.join(PKG, "_fast" + sysconfig.get_config_var("EXT_SUFFIX"))
+
+
+def build_fast(lib: str = LIB) -> str:
+    """Compile pyfast.c (gcc, CPython headers) against liblse_merge.so, found at
+    run time next to the extension ($ORIGIN)."""
+    import sysconfig
+    out = fast_path()
+    cmd = ["gcc", "-O2", "-shared", "-fPIC", "-std=c11", "-I", INCLUDE,
+           "-I", sysconfig.get_paths()["include"], FAST_SRC, "-L", os.path.dirname(lib),
+           "-l:" + os.path.basename(lib), "-Wl,-rpath,$ORIGIN", "-o", out]
+    subprocess.run(cmd, check=True)
+    return out
+
+
 def build(out: str = LIB, verbose: bool = False, extra: list[str] | None = None) -> str:
     cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *SOURCES, "-o", out]
     if verbose:
@@ -43,9 +65,12 @@ def build(out: str = LIB, verbose: bool = False, extra: list[str] | None = None)
     if extra:
         cmd[1:1] = extra
     subprocess.run(cmd, check=True)
+    if out == LIB:
+        build_fast(out)
     return out
 
 
 if __name__ == "__main__":
     build(verbose="--verbose" in sys.argv)
     print(LIB)
+    print(fast_path())

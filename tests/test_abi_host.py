@@ -236,3 +236,27 @@ def test_decode_valid_arguments_pass_validation():
     # valid arguments get past validation (here, without a GPU, the launch itself fails)
     for kw in (dict(), dict(R=3, fused=False), dict(R=64, fused=False), dict(D=64, Hq=16, Hkv=1)):
         assert dq(**kw) in (nat.OK, nat.ELAUNCH), kw
+
+
+def test_fast_forwarding_extension_is_built_and_checks_its_arguments():
+    """The vectorcall extension forwards to the same C entry points: a call
+    the library rejects returns the library's code (no CUDA call is made),
+    and Python-level mistakes raise before C is reached."""
+    from lse_weighted_merge_b200 import _fast
+    st = (64, 256, 128, 1, 4, 2)
+    assert _fast.merge(PO, PL, 2, 1, 0, 64, st, nat.BF16, nat.BF16, OUT, OUTL, 0, 0) == nat.EDIMS
+    assert _fast.merge(PO, PL, 2, 1, 2, 64, None, 7, nat.BF16, OUT, OUTL, 0, 0) == nat.EDTYPE
+    assert _fast.merge(0, PL, 2, 1, 2, 64, None, nat.BF16, nat.BF16, OUT, OUTL, 0, 0) == nat.ENULL
+    assert _fast.state_update(PO, PL, OUT, OUTL, 0, 2, 64, None, nat.F32, nat.BF16, 0) == nat.EDIMS
+    with pytest.raises(TypeError):
+        _fast.merge(PO, PL, 2, 1, 2, 64)                       # too few arguments
+    with pytest.raises(TypeError):
+        _fast.merge(PO, PL, 2, 1, 2, 64, (1, 2), 2, 2, OUT, OUTL, 0, 0)   # strides tuple of 2
+    with pytest.raises(OverflowError):
+        _fast.merge(PO, PL, 2**40, 1, 2, 64, None, 2, 2, OUT, OUTL, 0, 0)
+    with pytest.raises(OverflowError):
+        _fast.merge(-5, PL, 2, 1, 2, 64, None, 2, 2, OUT, OUTL, 0, 0)     # a negative pointer
+    # merge_raw takes every strides form it documents and routes through the extension
+    for s in (st, ((64, 256, 128), (1, 4, 2)), nat.Strides(*st)):
+        assert nat.merge_raw(PO, PL, 2, 1, 0, 64, s, nat.BF16, nat.BF16, OUT, OUTL, 0,
+                             check=False) == nat.EDIMS
