@@ -67,12 +67,13 @@ def merge(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, out=N
         raise ValueError("out_lse must be a contiguous float32 [B, H] tensor")
     if partial_lse.device != dev or out.device != dev or out_lse.device != dev:
         raise ValueError("all tensors must be on the same CUDA device")
-    # The library launches on the current device: make it the tensors' one.
-    with torch.cuda.device(dev):
-        stream = torch.cuda.current_stream(dev).cuda_stream
-        merge_raw(partial_o.data_ptr(), partial_lse.data_ptr(), R, B, H, D, st,
-                  dtype_code(partial_o.dtype), dtype_code(out_dtype), out.data_ptr(),
-                  out_lse.data_ptr(), stream, path)
+    args = (partial_o.data_ptr(), partial_lse.data_ptr(), R, B, H, D, (*st[0], *st[1]),
+            dtype_code(partial_o.dtype), dtype_code(out_dtype), out.data_ptr(), out_lse.data_ptr())
+    if torch.cuda.current_device() == dev.index:
+        merge_raw(*args, torch.cuda.current_stream().cuda_stream, path)
+    else:   # the library launches on the current device: make it the tensors' one
+        with torch.cuda.device(dev):
+            merge_raw(*args, torch.cuda.current_stream().cuda_stream, path)
     return out, out_lse
 
 

@@ -98,9 +98,13 @@ class CPMergeCall:
 
     def __call__(self, stream=None):
         import torch
-        with torch.cuda.device(self.device):
-            s = stream if stream is not None else torch.cuda.current_stream(self.device).cuda_stream
+        if torch.cuda.current_device() == self.device.index:
+            s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
             _native.cp_exchange_merge_raw(self.args, s)
+        else:   # the library launches on the current device: make it the tensors' one
+            with torch.cuda.device(self.device):
+                s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+                _native.cp_exchange_merge_raw(self.args, s)
         return self.outs
 
 
