@@ -18,11 +18,13 @@ Two ways in:
 from __future__ import annotations
 
 import datetime
+import itertools
 
 from . import _native
 from .api import dtype_code
 
 DEFAULT_TIMEOUT_S = 2.0
+_INSTANCES = itertools.count()
 
 
 def cp_workspace(world: int, B: int, H: int, D: int, dtype, device):
@@ -200,6 +202,8 @@ class CPExchangeMerge:
         self._checks = 0
         self._args_key = None
         self._args = None
+        # instances are numbered in construction order, the same on every rank
+        self._uid = next(_INSTANCES)
         self.ws = None
         self.peers = []
 
@@ -264,7 +268,9 @@ class CPExchangeMerge:
 
     def __call__(self, local_o, local_lse, out=None, out_lse=None, stream: int | None = None):
         """Send this rank's partials (local_o [B, H, D], local_lse [B, H]) and
-        merge the heads it owns: returns (out [B, H/world, D], out_lse [B, H/world])."""
+        merge the heads it owns: returns (out [B, H/world, D], out_lse [B, H/world]).
+        Passing the same out / out_lse (and inputs) on every step keeps the
+        prepared argument block; new buffers rebuild it."""
         import torch
         if self.broken:
             raise RuntimeError("a wait ran out in an earlier call: call reset() on every rank")
@@ -307,7 +313,7 @@ class CPExchangeMerge:
         the group's store and waits for all the others'.  Raises PeerLost
         naming the ranks that did not post in time."""
         store = self.dist.distributed_c10d._get_default_store()
-        prefix = f"lse_cp/alive/{self._checks}/"
+        prefix = f"lse_cp/{self._uid}/alive/{self._checks}/"
         self._checks += 1
         store.set(prefix + str(self.rank), b"1")
         keys = [prefix + str(q) for q in range(self.world)]
