@@ -87,6 +87,17 @@ def test_exchange_merge_workloads(name, cross):
 
 
 @pytest.mark.parametrize("cross", [False, True], ids=["one-gpu-protocol", "cross-gpu-protocol"])
+def test_exchange_merge_large(cross):
+    """8 ranks of B=256 H=64 D=128 (34 MB of partials): many CTAs per rank, so
+    every receiver collects counts from many sending CTAs of each sender."""
+    inp = inputs(R=8, B=256, H=64, D=128, seed=900)
+    lo, ll = to_device(inp)
+    outs = cp.cp_exchange_merge(lo, ll, workspaces(inp), cross_gpu_protocol=cross)
+    torch.cuda.synchronize()
+    compare(outs, inp, "large")
+
+
+@pytest.mark.parametrize("cross", [False, True], ids=["one-gpu-protocol", "cross-gpu-protocol"])
 def test_repeated_calls_alternate_slots_and_count_on_device(cross):
     base = inputs(R=4, B=6, H=8, D=128, seed=1)
     ws = workspaces(base)
