@@ -19,7 +19,7 @@
  *     and divides by denom; the fused kernel's steps 2 and 3 are "LSE-based
  *     softmax weights" and "accumulate in FP32, then convert to FP16/BF16".
  *
- * Readings where the page is silent (each also listed in the design doc):
+ * Readings where the page is silent:
  *   - lse is a natural logarithm;
  *   - weights = exp(lse_r - m) with m = max_r lse_r, denom = sum of weights
  *     (the plainest reading of the snippet's `weights` and `denom`);
