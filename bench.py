@@ -408,6 +408,61 @@ def oracle_seconds(inp: dict, budget_s: float):
     return byts * passes / dt, passes, dt
 
 
+def _timed(fn, budget_s: float):
+    """Call fn() repeatedly for at least budget_s; returns (calls, seconds)."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            return n, dt
+
+
+def next_rows_cpu_baselines(extra: dict, budget_s: float = 1.0) -> None:
+    """The fp64 oracle timed beside the state update, the decode attention and
+    the exchange lines, on a bounded sample of each (single thread): adds a
+    `cpu_baseline` entry to each row of `extra`."""
+    import math
+    import numpy as np
+    import oracle
+    from lse_weighted_merge_b200 import synth
+    lib = oracle.load()
+    rng = np.random.Generator(np.random.PCG64(7))
+    if "state_update" in extra:
+        # 8 of the 512 batches of the B=512 H=16 D=512 fold, fp32 accumulator, bf16 partial
+        B, H, D = 8, 16, 512
+        acc = rng.standard_normal(B * H * D, dtype=np.float32)
+        new = synth.pack(rng.standard_normal(B * H * D, dtype=np.float32), "bf16")
+        la = rng.uniform(0, 8, B * H).astype(np.float32)
+        byts = B * H * (D * 10 + 12)
+        n, dt = _timed(lambda: oracle.state_update(acc, la, oracle.F32, new, la, oracle.BF16,
+                                                   B, H, D, lib=lib), budget_s)
+        extra["state_update"]["cpu_baseline"] = {
+            "value": byts * n / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"8 of 512 batches, {n} passes in {dt:.1f} s, fp64 C oracle, single thread"}
+    for name, row in extra.get("decode_attention", {}).items():
+        # one (b, query head) row of the shape: attention over all L keys, fp64
+        L, D = (4096, 128) if "l4096" in name else (32768, 128)
+        q = rng.standard_normal(D)
+        k = rng.standard_normal((L, D))
+        v = rng.standard_normal((L, D))
+        n, dt = _timed(lambda: oracle.attention_shard(q, k, v, 1 / math.sqrt(D), 0, L, lib=lib),
+                       budget_s)
+        per_row = L * D * 2 * 2 // (4 if "hq32_hkv8" in name else 1)   # K and V bytes per query head
+        row["cpu_baseline"] = {
+            "value": per_row * n / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"one query head over all {L} keys, {n} passes in {dt:.1f} s, fp64 C oracle",
+            "us_per_query_head": dt / n * 1e6}
+    for name, row in extra.get("cp_exchange_merge", {}).items():
+        w = synth.CP_WORKLOADS[name]
+        inp = synth.make_inputs(w)
+        n, dt = _timed(lambda: oracle.cp_exchange_merge(inp["o"], inp["lse"], w.R, w.B, w.H, w.D,
+                                                        synth.DTYPES[w.in_dtype], lib=lib), budget_s)
+        row["cpu_baseline"] = {"value": dt / n * 1e6, "unit": "us/call", "cores": 1, "kind": "oracle",
+                               "sample": f"the whole workload, {n} calls in {dt:.1f} s, fp64 C oracle"}
+
+
 # ------------------------------------------------------------------------- arms
 
 def run_reference(args):
@@ -525,6 +580,8 @@ def run_ours(args):
     if not args.no_extra:
         extra = extra_workloads(device, l2, dist)
     clock.stop()
+    if extra and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        next_rows_cpu_baselines(extra)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

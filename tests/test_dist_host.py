@@ -70,3 +70,18 @@ def test_reference_arm_prints_on_rank0_only():
     line = json.loads(p.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_next_rows_get_an_oracle_baseline():
+    """bench.py times the fp64 oracle beside the state-update, decode-attention
+    and exchange lines (bounded samples, one thread)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    extra = {"state_update": {}, "decode_attention": {"b64_hq32_hkv8_l4096_d128_r4": {}},
+             "cp_exchange_merge": {"cp_w2_b1_h2_d64": {}}}
+    bench.next_rows_cpu_baselines(extra, budget_s=0.02)
+    rows = [extra["state_update"], extra["decode_attention"]["b64_hq32_hkv8_l4096_d128_r4"],
+            extra["cp_exchange_merge"]["cp_w2_b1_h2_d64"]]
+    for row in rows:
+        cb = row["cpu_baseline"]
+        assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0 and cb["sample"]
