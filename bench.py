@@ -71,6 +71,8 @@ def parse_args(argv=None):
                    help="only time the decode-attention shape SHAPE (for profiling)")
     p.add_argument("--cp-only", default=None, metavar="WORKLOAD",
                    help="only time the context-parallel exchange + merge WORKLOAD (for profiling)")
+    p.add_argument("--state-only", action="store_true",
+                   help="only time the in-place state update (for profiling)")
     return p.parse_args(argv)
 
 
@@ -825,6 +827,14 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.state_only:
+        import torch
+        device = torch.device("cuda", 0)
+        peak, _ = hbm_peak()
+        props = torch.cuda.get_device_properties(device)
+        l2 = getattr(props, "L2_cache_size", 0) or L2_FALLBACK
+        print(json.dumps({"state_update": time_state_update(device, l2, peak)}))
+        return 0
     if args.cp_only:
         import torch
         device = torch.device("cuda", 0)
