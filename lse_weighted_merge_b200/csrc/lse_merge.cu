@@ -409,13 +409,15 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const 
 
 // ------------------------------------------------------------------ wide kernel
 
-// For R > 16: one CTA of up to kWideWarps warps per row slice, so that every
-// partial of the row can be in flight at once.  The CTA's lane groups (of
-// p.lanes lanes, one 16-byte column each) are S sub-groups; sub-group s takes
-// the partials s, s + S, s + 2S, ... in batches of RC and keeps an online
-// state (running max m, weight sum, fp32 accumulator), rescaled when a batch
-// raises the max.  The S states are then merged -- the same LSE combine --
-// by shuffles inside each warp and through shared memory across warps.
+// For R > 16, and for a handful of rows of any R (at most kWideMaxSlices row
+// slices, where more threads per row beat more loads per thread): one CTA of
+// up to kWideWarps warps per row slice, so that every partial of the row can
+// be in flight at once.  The CTA's lane groups (of p.lanes lanes, one 16-byte
+// column each) are S sub-groups; sub-group s takes the partials s, s + S,
+// s + 2S, ... in batches of RC and keeps an online state (running max m,
+// weight sum, fp32 accumulator), rescaled when a batch raises the max.  The S
+// states are then merged -- the same LSE combine -- by shuffles inside each
+// warp and through shared memory across warps.
 constexpr int kWideWarps = 4;
 
 __device__ __forceinline__ void combine_state(float& m, float& es, float* acc, float m2, float es2,

@@ -46,7 +46,7 @@ constexpr long long kStreamMinBytes = 8ll << 20;
 // R <= 16: a handful of rows is latency-bound, and more threads per row beat
 // more loads per thread (8 rows of R=8: 2.03 us WIDE, 2.23 us VECTOR).
 constexpr long long kWideMaxSlices = 128;
-// Threads per CTA of the wide kernel (R > 16: one CTA per row slice).
+// Most threads per CTA of the wide kernel (one CTA per row slice).
 constexpr int kWideBlock = 128;
 // Upper bound on the 16-byte columns per lane (1, 2 or 4).
 #ifndef LSEM_MAX_NV
