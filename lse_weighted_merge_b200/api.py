@@ -1,6 +1,8 @@
 """The torch-facing call: tensors in, one C-ABI launch, tensors out."""
 from __future__ import annotations
 
+import threading
+
 from ._native import (BF16, F16, F32, PATH_AUTO, PATH_LATENCY, PATH_SCALAR, PATH_STREAM,
                       PATH_VECTOR,
                       LseMergeError, decode_raw, merge_raw, plan_query, state_update_raw,
@@ -79,11 +81,15 @@ def merge(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, out=N
 
 _STREAMS: dict = {}
 _WORKSPACE: dict = {}
+# merge_host's caches are shared by every thread; one call at a time per
+# process uses them (the copies and merges it enqueues still overlap).
+_HOST_LOCK = threading.Lock()
 
 
 def release_host_workspace() -> None:
     """Free the device staging buffers merge_host keeps between calls."""
-    _WORKSPACE.clear()
+    with _HOST_LOCK:
+        _WORKSPACE.clear()
 
 
 def _workspace(device, o_shape, o_dtype, l_shape, B, H, D, out_dtype):
@@ -149,6 +155,14 @@ def merge_host(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, 
         out = torch.empty((B, H, D), dtype=out_dtype).pin_memory()
     if out_lse is None:
         out_lse = torch.empty((B, H), dtype=torch.float32).pin_memory()
+    with _HOST_LOCK:
+        return _merge_host_locked(partial_o, partial_lse, layout, out_dtype, chunks, device, out,
+                                  out_lse, sync, R, B, H, D)
+
+
+def _merge_host_locked(partial_o, partial_lse, layout, out_dtype, chunks, device, out, out_lse,
+                       sync, R, B, H, D):
+    import torch
     ws = _workspace(device, tuple(partial_o.shape), partial_o.dtype, tuple(partial_lse.shape),
                     B, H, D, out_dtype)
     d_o, d_l, d_out, d_out_lse = ws["bufs"]

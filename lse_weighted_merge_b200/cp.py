@@ -312,6 +312,8 @@ class CPExchangeMerge:
         """Host-side liveness check between steps: every rank posts a key in
         the group's store and waits for all the others'.  Raises PeerLost
         naming the ranks that did not post in time."""
+        # the default process group's key-value store: torch offers no public
+        # accessor for it, and it works with every backend (NCCL included)
         store = self.dist.distributed_c10d._get_default_store()
         prefix = f"lse_cp/{self._uid}/alive/{self._checks}/"
         self._checks += 1
