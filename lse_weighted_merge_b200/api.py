@@ -123,7 +123,7 @@ def _side_streams(device):
 
 
 def merge_host(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, chunks: int = 8,
-               device=None, out=None, out_lse=None, sync: bool = True):
+               device=None, out=None, out_lse=None, sync: bool = True, pipeline: bool = False):
     """Merge partials that live in (pinned) host memory; results land in host memory.
 
     The batch is cut into ``chunks`` slices along B.  Slice i is copied to the
@@ -140,6 +140,16 @@ def merge_host(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, 
     ``sync=False`` the call returns once everything is enqueued; the current
     stream of ``device`` is made to wait for the last copy, so synchronising
     that stream (or the device) makes the results valid.
+
+    ``pipeline=True`` (with ``sync=False``, for a stream of batches) lets this
+    call's uploads start as soon as the previous call's uploads end, instead
+    of after the previous call's last copy back: the staging buffers are
+    reused chunk by chunk once the previous call has merged that chunk and
+    copied its result back.  The uploads then no longer wait for the current
+    stream, so the host inputs must not be written by device work still
+    pending there (inputs filled by the CPU, the usual case, are fine); give
+    consecutive pipelined calls distinct host outputs, or read each call's
+    outputs before the next call's copies back can overwrite them.
     """
     import torch
     if partial_o.is_cuda or partial_lse.is_cuda:
@@ -157,26 +167,54 @@ def merge_host(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, 
         out_lse = torch.empty((B, H), dtype=torch.float32).pin_memory()
     with _HOST_LOCK:
         return _merge_host_locked(partial_o, partial_lse, layout, out_dtype, chunks, device, out,
-                                  out_lse, sync, R, B, H, D)
+                                  out_lse, sync, pipeline, R, B, H, D)
+
+
+def _chunk_events(ws: dict, parity: int, n: int) -> list:
+    """The (landed, merged, copied-back) events of n chunks, in one of two sets
+    that alternate between calls: a call records into one set while the next
+    call waits on it and records into the other."""
+    import torch
+    sets = ws.setdefault("event_sets", [[], []])
+    evs = sets[parity]
+    while len(evs) < n:
+        evs.append((torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()))
+    return evs
 
 
 def _merge_host_locked(partial_o, partial_lse, layout, out_dtype, chunks, device, out, out_lse,
-                       sync, R, B, H, D):
+                       sync, pipeline, R, B, H, D):
     import torch
     ws = _workspace(device, tuple(partial_o.shape), partial_o.dtype, tuple(partial_lse.shape),
                     B, H, D, out_dtype)
     d_o, d_l, d_out, d_out_lse = ws["bufs"]
     cur = torch.cuda.current_stream(device)
     s_in, s_merge, s_back = _side_streams(device)
-    # The staging buffers are free once the previous call's last copy is done
-    # (its `done` event); the host outputs may be in use on the current stream.
-    for s_ in (s_in, s_back):
-        s_.wait_event(ws["done"])
-        s_.wait_stream(cur)
     nb = max(1, -(-B // max(1, int(chunks))))
-    for b0 in range(0, B, nb):
+    n = -(-B // nb)
+    # The previous call's chunk events, if it cut the batch the same way.
+    prev = ws.get("chunks")
+    prev = prev[1] if (pipeline and prev is not None and prev[0] == nb) else None
+    if prev is None:
+        # The staging buffers are free once the previous call's last copy is
+        # done (its `done` event); the host inputs and outputs may be in use
+        # on the current stream.
+        for s_ in (s_in, s_back):
+            s_.wait_event(ws["done"])
+            s_.wait_stream(cur)
+    else:
+        # Pipelined: chunk i's staging buffers are free once the previous call
+        # merged chunk i and copied its result back, so this call's uploads
+        # follow the previous call's without waiting for its last copy back.
+        s_back.wait_stream(cur)      # the host outputs may be in use on the current stream
+    parity = ws.get("parity", 0) ^ 1
+    evs = _chunk_events(ws, parity, n)
+    for i, b0 in enumerate(range(0, B, nb)):
         b1 = min(B, b0 + nb)
+        landed, merged, copied = evs[i]
         with torch.cuda.stream(s_in):
+            if prev is not None:
+                s_in.wait_event(prev[i][1])
             if layout == "bhrd":
                 d_o[b0:b1].copy_(partial_o[b0:b1], non_blocking=True)
                 d_l[b0:b1].copy_(partial_lse[b0:b1], non_blocking=True)
@@ -186,18 +224,21 @@ def _merge_host_locked(partial_o, partial_lse, layout, out_dtype, chunks, device
                     d_o[r, b0:b1].copy_(partial_o[r, b0:b1], non_blocking=True)
                     d_l[r, b0:b1].copy_(partial_lse[r, b0:b1], non_blocking=True)
                 vo, vl = d_o[:, b0:b1], d_l[:, b0:b1]
-            landed = torch.cuda.Event()
             landed.record(s_in)
         s_merge.wait_event(landed)
+        if prev is not None:
+            s_merge.wait_event(prev[i][2])
         with torch.cuda.stream(s_merge):
             merge(vo, vl, layout=layout, out_dtype=out_dtype, out=d_out[b0:b1],
                   out_lse=d_out_lse[b0:b1])
-            merged = torch.cuda.Event()
             merged.record(s_merge)
         s_back.wait_event(merged)
         with torch.cuda.stream(s_back):
             out[b0:b1].copy_(d_out[b0:b1], non_blocking=True)
             out_lse[b0:b1].copy_(d_out_lse[b0:b1], non_blocking=True)
+            copied.record(s_back)
+    ws["chunks"] = (nb, evs[:n])
+    ws["parity"] = parity
     ws["done"].record(s_back)
     cur.wait_stream(s_back)
     if sync:

@@ -267,6 +267,31 @@ def test_merge_host_pipelined(name, chunks):
     check(out.double().numpy(), out_lse.double().numpy(), want, want_lse, inp["out_dtype"], name)
 
 
+@pytest.mark.parametrize("layout", ["bhrd", "rbhd"])
+def test_merge_host_pipelined_calls_in_a_row(layout):
+    """Consecutive pipelined calls (each call's uploads start before the
+    previous call's copies back end), a default call and a call with another
+    chunk count among them, each with its own inputs and host outputs: after
+    one synchronisation every result matches the oracle."""
+    from lse_weighted_merge_b200 import merge_host
+    w = W["r4_b64_h32_d128_masked"]
+    plan = [(8, True), (8, True), (8, False), (8, True), (3, True), (3, True)]
+    results = []
+    for k, (chunks, pipe) in enumerate(plan):
+        inp = synth.make_inputs(w, seed=700 + k, poison_empty=True, layout=layout)
+        R, B, H, D = inp["R"], inp["B"], inp["H"], inp["D"]
+        shape_o = (B, H, R, D) if layout == "bhrd" else (R, B, H, D)
+        h_o = torch.from_numpy(inp["o"].view(np.int16)).view(torch.bfloat16).reshape(shape_o).pin_memory()
+        h_l = torch.from_numpy(inp["lse"]).reshape(shape_o[:3]).pin_memory()
+        out, out_lse = merge_host(h_o, h_l, layout=layout, chunks=chunks, sync=False, pipeline=pipe)
+        results.append((inp, out, out_lse, h_o, h_l))
+    torch.cuda.synchronize()
+    for k, (inp, out, out_lse, _, _) in enumerate(results):
+        want, want_lse = run_oracle(inp)
+        check(out.double().numpy(), out_lse.double().numpy(), want, want_lse, inp["out_dtype"],
+              f"call {k} {plan[k]}")
+
+
 @pytest.mark.parametrize("R,B,H,D", [(64, 1, 8, 128), (64, 64, 32, 128), (128, 4, 8, 512),
                                      (48, 2, 3, 64)])
 def test_many_partials_wide_path(R, B, H, D):
