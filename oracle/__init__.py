@@ -26,12 +26,11 @@ LIB = os.path.join(HERE, "liboracle.so")
 F32, F16, BF16 = 0, 1, 2
 
 
-def build(out_path: str = LIB, mutant: int = 0) -> str:
-    """Compile the oracle with gcc (optionally with one planted mistake)."""
+def build(out_path: str = LIB, src: str = SRC) -> str:
+    """Compile the oracle with gcc (``src``: another copy of the source, as the
+    tests that plant a mistake in one use)."""
     cmd = ["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-fno-fast-math",
-           SRC, "-o", out_path, "-lm"]
-    if mutant:
-        cmd.insert(1, f"-DORACLE_MUTANT={int(mutant)}")
+           src, "-o", out_path, "-lm"]
     subprocess.run(cmd, check=True)
     return out_path
 
@@ -49,7 +48,6 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_attention_shard.argtypes = [
         dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
         ctypes.c_int, dp, dp]
-    lib.oracle_mutant.restype = ctypes.c_int
     lib.oracle_state_update.restype = ctypes.c_int
     lib.oracle_state_update.argtypes = [
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,

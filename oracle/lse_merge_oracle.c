@@ -30,24 +30,15 @@
  *     fp64 arithmetic below gives (NaN propagates), nothing is special-cased.
  *
  * The result stays in fp64; rounding to the output dtype is not modelled.
- *
- * ORACLE_MUTANT: when compiled with -DORACLE_MUTANT=k (k >= 1) one plausible
- * mistake is planted on purpose, so the pin tests can show that each such
- * mistake is caught.  The normal build defines no mutant.
  */
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
 
-#ifndef ORACLE_MUTANT
-#define ORACLE_MUTANT 0
-#endif
-
 /* Element types, numbered like the public C-ABI but defined here on their own. */
 enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2 };
 
 int oracle_version(void) { return 1; }
-int oracle_mutant(void) { return ORACLE_MUTANT; }
 
 /* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
 static double widen_f16(uint16_t bits) {
@@ -128,14 +119,8 @@ int oracle_lse_merge(const void* partial_o, const float* partial_lse,
         return -2;
     for (int b = 0; b < B; ++b) {
         for (int h = 0; h < H; ++h) {
-#if ORACLE_MUTANT == 3
-            /* planted mistake: batch and head strides swapped */
-            const int64_t o_row = (int64_t)b * os[2] + (int64_t)h * os[1];
-            const int64_t l_row = (int64_t)b * ls[2] + (int64_t)h * ls[1];
-#else
             const int64_t o_row = (int64_t)b * os[1] + (int64_t)h * os[2];
             const int64_t l_row = (int64_t)b * ls[1] + (int64_t)h * ls[2];
-#endif
             double* out = out_o + ((int64_t)b * H + h) * D;
             double* olse = out_lse + (int64_t)b * H + h;
 
@@ -152,37 +137,17 @@ int oracle_lse_merge(const void* partial_o, const float* partial_lse,
 
             for (int d = 0; d < D; ++d) out[d] = 0.0;
             double denom = 0.0;
-#if ORACLE_MUTANT == 6
-            for (int r = 1; r < R; ++r) {               /* planted mistake: first shard dropped */
-#else
             for (int r = 0; r < R; ++r) {
-#endif
                 double l = (double)partial_lse[l_row + (int64_t)r * ls[0]];
-#if ORACLE_MUTANT != 4
                 if (l == -INFINITY) continue;           /* empty shard: weight 0, o_r not read */
-#endif
-#if ORACLE_MUTANT == 2
-                double e = exp(m - l);                  /* planted mistake: sign flipped */
-#else
                 double e = exp(l - m);
-#endif
                 denom += e;
                 const int64_t o_sh = o_row + (int64_t)r * os[0];
                 for (int d = 0; d < D; ++d)
                     out[d] += e * load_elem(partial_o, o_sh + d, in_dtype);
             }
-            for (int d = 0; d < D; ++d) {
-#if ORACLE_MUTANT == 5
-                out[d] /= (double)R;                    /* planted mistake: plain mean */
-#else
-                out[d] /= denom;
-#endif
-            }
-#if ORACLE_MUTANT == 1
-            *olse = log(denom);                         /* planted mistake: max term dropped */
-#else
+            for (int d = 0; d < D; ++d) out[d] /= denom;
             *olse = m + log(denom);
-#endif
         }
     }
     return 0;
@@ -260,14 +225,8 @@ int oracle_state_update(const void* acc, const float* lse_acc, int acc_dtype,
                 out_lse[row] = -INFINITY;
                 continue;
             }
-#if ORACLE_MUTANT == 7
-            /* planted mistake: the two weights swapped */
-            const double en = (la == -INFINITY) ? 0.0 : exp(la - m);
-            const double ea = (ln == -INFINITY) ? 0.0 : exp(ln - m);
-#else
             const double ea = (la == -INFINITY) ? 0.0 : exp(la - m);
             const double en = (ln == -INFINITY) ? 0.0 : exp(ln - m);
-#endif
             const double denom = ea + en;
             for (int d = 0; d < D; ++d) {
                 double s = 0.0;
@@ -307,11 +266,7 @@ int oracle_cp_exchange_merge(const void* local_o, const float* local_lse, int wo
     const int64_t os[3] = {(int64_t)B * H * D, (int64_t)H * D, D};
     const int64_t ls[3] = {(int64_t)B * H, H, 1};
     for (int q = 0; q < world; ++q) {
-#if ORACLE_MUTANT == 8
-        const int64_t h0 = 0;                           /* planted mistake: owner's head offset dropped */
-#else
         const int64_t h0 = (int64_t)q * Hq;             /* first head rank q owns */
-#endif
         const char* o = (const char*)local_o + h0 * D * esize;
         const float* l = local_lse + h0;
         int rc = oracle_lse_merge(o, l, world, B, Hq, D, os, ls, in_dtype,
