@@ -20,6 +20,8 @@ import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "lse_merge_oracle.c")
+# Runs the unchanged merge on several host threads (CPU-baseline timing only).
+THREADS_SRC = os.path.join(HERE, "oracle_threads.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 # Element types, numbered like the public C-ABI (defined again here on purpose).
@@ -29,8 +31,8 @@ F32, F16, BF16 = 0, 1, 2
 def build(out_path: str = LIB, src: str = SRC) -> str:
     """Compile the oracle with gcc (``src``: another copy of the source, as the
     tests that plant a mistake in one use)."""
-    cmd = ["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-fno-fast-math",
-           src, "-o", out_path, "-lm"]
+    cmd = ["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-fno-fast-math", "-pthread",
+           src, THREADS_SRC, "-o", out_path, "-lm"]
     subprocess.run(cmd, check=True)
     return out_path
 
@@ -53,6 +55,12 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
         ctypes.c_int64, ctypes.c_int64, dp, dp]
+    lib.oracle_lse_merge_threads.restype = ctypes.c_int
+    lib.oracle_lse_merge_threads.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, i64p, i64p, ctypes.c_int, dp, dp, ctypes.c_int,
+        ctypes.POINTER(ctypes.c_int)]
+    lib.oracle_host_threads.restype = ctypes.c_int
     lib.oracle_cp_exchange_merge.restype = ctypes.c_int
     lib.oracle_cp_exchange_merge.argtypes = [
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -69,7 +77,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     if path in _cached:
         return _cached[path]
     if path == LIB and (not os.path.exists(LIB)
-                        or os.path.getmtime(LIB) < os.path.getmtime(SRC)):
+                        or os.path.getmtime(LIB) < max(os.path.getmtime(SRC),
+                                                       os.path.getmtime(THREADS_SRC))):
         build(LIB)
     lib = _bind(ctypes.CDLL(path))
     _cached[path] = lib
@@ -82,12 +91,15 @@ def widen(bits: int, dtype: int, lib: ctypes.CDLL | None = None) -> float:
 
 def merge(partial_o: np.ndarray, partial_lse: np.ndarray, R: int, B: int, H: int,
           D: int, o_strides, lse_strides, in_dtype: int,
-          lib: ctypes.CDLL | None = None):
+          lib: ctypes.CDLL | None = None, threads: int = 1, stats: dict | None = None):
     """Run the fp64 merge.
 
     partial_o: a flat numpy buffer holding the raw elements (uint16 bit
     patterns for F16/BF16, float32 for F32); partial_lse: flat float32.
     Strides are (r, b, h) in elements; the d stride is 1.
+    threads: 1 runs oracle_lse_merge on the calling thread; any other value
+    splits the batches over that many host threads (0: one per core), each
+    running the same function; ``stats["threads"]`` receives the count used.
     Returns (out [B, H, D] float64, out_lse [B, H] float64).
     """
     lib = lib or load()
@@ -100,10 +112,20 @@ def merge(partial_o: np.ndarray, partial_lse: np.ndarray, R: int, B: int, H: int
     ls_ = (ctypes.c_int64 * 3)(*[int(s) for s in lse_strides])
     out = np.empty((B, H, D), dtype=np.float64)
     out_lse = np.empty((B, H), dtype=np.float64)
-    rc = lib.oracle_lse_merge(
-        po.ctypes.data, pl.ctypes.data, R, B, H, D, os_, ls_, in_dtype,
-        out.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
-        out_lse.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
+    dp = ctypes.POINTER(ctypes.c_double)
+    if threads == 1:
+        rc = lib.oracle_lse_merge(po.ctypes.data, pl.ctypes.data, R, B, H, D, os_, ls_, in_dtype,
+                                  out.ctypes.data_as(dp), out_lse.ctypes.data_as(dp))
+        used = 1
+    else:
+        n = ctypes.c_int(0)
+        rc = lib.oracle_lse_merge_threads(po.ctypes.data, pl.ctypes.data, R, B, H, D, os_, ls_,
+                                          in_dtype, out.ctypes.data_as(dp),
+                                          out_lse.ctypes.data_as(dp), int(threads),
+                                          ctypes.byref(n))
+        used = n.value
+    if stats is not None:
+        stats["threads"] = used
     if rc != 0:
         raise ValueError(f"oracle_lse_merge returned {rc}")
     return out, out_lse
