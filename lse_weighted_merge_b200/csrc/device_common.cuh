@@ -175,5 +175,15 @@ __device__ __forceinline__ void store_vec(char* p, const float* f) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
+// Ask L2 to fetch the line holding p.  L2 is the device's point of coherence,
+// so a line fetched here before the previous grid has finished writing it
+// still reads that grid's data afterwards: the prefetch may be issued before
+// pdl_wait(), where it overlaps this grid's first DRAM round with the drain
+// of the previous one.  It returns no data and never faults on the addresses
+// the kernel would load anyway.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 }  // namespace
 }  // namespace lsem

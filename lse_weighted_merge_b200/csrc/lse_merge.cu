@@ -139,11 +139,9 @@ __device__ __forceinline__ void store_cols(const KParams& p, int64_t row, int v0
 // This is the form with one 16-byte column per lane (NV = 1), used whenever
 // the planner gives a lane a single column.
 template <typename TIn, typename TOut, int RC>
-__global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec1_kernel(const KParams p) {
+__global__ void __launch_bounds__(kBlock, kMinBlocksVec1) merge_vec1_kernel(const KParams p) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
-    pdl_wait();
-    pdl_release();
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t grp = t >> p.lg;
     const int j = (int)(t & (p.lanes - 1));
@@ -153,6 +151,14 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec1_kernel(const KP
     const bool vlive = live && v < p.dv;
     const char* orow = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)v * 16;
     const float* lrow = p.lse + ri.b * p.l_b + ri.h * p.l_h;
+    if (kPrefetch) {   // the first RC partial rows, while the previous grid drains
+#pragma unroll
+        for (int i = 0; i < RC; ++i)
+            if (vlive && i < p.R) prefetch_l2(orow + (int64_t)i * p.o_r);
+        if (live && j < p.R) prefetch_l2(lrow + (int64_t)j * p.l_r);
+    }
+    pdl_wait();
+    pdl_release();
 
     // Partial rows 0..RC-1 go in flight first; nothing here waits on lse.
     uint4 x[RC];
@@ -238,8 +244,6 @@ template <typename TIn, typename TOut, int RC, int NV>
 __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KParams p) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
-    pdl_wait();
-    pdl_release();
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t grp = t >> p.lg;
     const int j = (int)(t & (p.lanes - 1));
@@ -251,6 +255,16 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KPa
     bool cl[NV];   // column k of this lane lies inside the row
 #pragma unroll
     for (int k = 0; k < NV; ++k) cl[k] = live && v0 + k * p.lanes < p.dv;
+    if (kPrefetch) {   // the first RC partial rows, while the previous grid drains
+#pragma unroll
+        for (int i = 0; i < RC; ++i)
+#pragma unroll
+            for (int k = 0; k < NV; ++k)
+                if (cl[k] && i < p.R) prefetch_l2(orow + (int64_t)i * p.o_r + k * p.lanes * 16);
+        if (live && j < p.R) prefetch_l2(lrow + (int64_t)j * p.l_r);
+    }
+    pdl_wait();
+    pdl_release();
 
     // Partial rows 0..RC-1 go in flight first; nothing here waits on lse.
     uint4 x[RC][NV];
@@ -326,11 +340,9 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KPa
 // keeps up to R*NV 16-byte loads in flight across slice boundaries and no
 // warp ever waits for a CTA to retire or launch.
 template <typename TIn, typename TOut, int RC, int NV>
-__global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const KParams p, const int64_t G) {
+__global__ void __launch_bounds__(kBlock, kMinBlocksStream) merge_stream_kernel(const KParams p, const int64_t G) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
-    pdl_wait();
-    pdl_release();
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int j = (int)(t & (p.lanes - 1));
     // The first group of a warp has the most slices: a warp-uniform trip count
@@ -362,6 +374,18 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_stream_kernel(const 
     };
 
     Slice cur = locate(grp0);
+    // The first kPrefetch slices' lines, while the previous grid drains.
+    for (int64_t it = 0; it < kPrefetch && it < trips; ++it) {
+        const Slice s = it == 0 ? cur : locate(grp0 + it * G);
+#pragma unroll
+        for (int i = 0; i < RC; ++i)
+#pragma unroll
+            for (int k = 0; k < NV; ++k)
+                if (s.cl[k] && i < p.R) prefetch_l2(s.o + (int64_t)i * p.o_r + k * p.lanes * 16);
+        if (s.live && j < p.R) prefetch_l2(s.l + (int64_t)j * p.l_r);
+    }
+    pdl_wait();
+    pdl_release();
     uint4 x[RC][NV];
 #pragma unroll
     for (int i = 0; i < RC; ++i)
@@ -436,8 +460,6 @@ __global__ void __launch_bounds__(kWideWarps * 32) merge_wide_kernel(const KPara
     constexpr int N2 = N / 2;
     __shared__ float sh_acc[kWideWarps][32][N];
     __shared__ float sh_m[kWideWarps], sh_es[kWideWarps];
-    pdl_wait();
-    pdl_release();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = blockDim.x >> 5;                    // warps of this CTA (<= kWideWarps)
     const int j = lane & (p.lanes - 1);
@@ -452,6 +474,14 @@ __global__ void __launch_bounds__(kWideWarps * 32) merge_wide_kernel(const KPara
     const float* lrow = p.lse + ri.b * p.l_b + ri.h * p.l_h;
     const int n_w = p.R > s_w ? (p.R - s_w + S - 1) / S : 0;   // partials of sub-group s_w
     const int batches = (n_w + RC - 1) / RC;                    // warp-uniform
+    if (kPrefetch) {   // the first batch, while the previous grid drains
+#pragma unroll
+        for (int i = 0; i < RC; ++i)
+            if (vlive && s + S * i < p.R) prefetch_l2(orow + (int64_t)(s + S * i) * p.o_r);
+        if (j < RC && s + S * j < p.R) prefetch_l2(lrow + (int64_t)(s + S * j) * p.l_r);
+    }
+    pdl_wait();
+    pdl_release();
 
     float m = -INFINITY, es = 0.f;
     uint64_t acc[N2];
@@ -643,6 +673,11 @@ __device__ __forceinline__ void store8(char* p, int n, const float* f) {
 // registers, fewer resident warps); loads issued only after the weights
 // 10.04 us.
 constexpr int kStateChunks = 1;
+// Chunks per lane whose lines are prefetched into L2 before pdl_wait().
+#ifndef LSEM_STATE_PREFETCH
+#define LSEM_STATE_PREFETCH 4
+#endif
+constexpr int kStatePrefetch = LSEM_STATE_PREFETCH;
 
 // A group of p.lanes lanes per row.  Lane 0 of the group reads both lse values
 // and hands them to the group by shuffle, so no lane reads lse_acc after lane
@@ -652,8 +687,6 @@ constexpr int kStateChunks = 1;
 // result.
 template <typename TA, typename TN, bool VEC>
 __global__ void __launch_bounds__(kBlock) state_update_kernel(const SParams p) {
-    pdl_wait();
-    pdl_release();
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t row = t >> p.lg;
     const int j = (int)(t & (p.lanes - 1));
@@ -662,6 +695,18 @@ __global__ void __launch_bounds__(kBlock) state_update_kernel(const SParams p) {
     const int64_t b = r / p.H, h = r - b * p.H;
     char* arow = p.acc + r * p.D * (int64_t)sizeof(TA);
     const char* nrow = p.nw + b * p.n_b + h * p.n_h;
+    if (kPrefetch && live) {   // this lane's first kStatePrefetch chunks of both sides
+        for (int i = 0, c = j; i < kStatePrefetch && c < p.chunks; ++i, c += p.lanes) {
+            prefetch_l2(arow + (int64_t)c * 8 * sizeof(TA));
+            prefetch_l2(nrow + (int64_t)c * 8 * sizeof(TN));
+        }
+        if (j == 0) {
+            prefetch_l2(p.lse_acc + r);
+            prefetch_l2(p.lse_new + b * p.l_b + h * p.l_h);
+        }
+    }
+    pdl_wait();
+    pdl_release();
 
     float fa[kStateChunks][8], fn[kStateChunks][8];
     auto load_batch = [&](int c0) {
