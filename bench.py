@@ -9,18 +9,25 @@ A step is one merge of one batch of the large decode-merge workload
 R*B*H*(D*2+4) + B*H*(D*4+4).  Rank 0 prints one JSON line.
 
   value     device throughput (GB/s of algorithmic bytes, all ranks) with the
-            inputs resident in HBM; K eager launches timed with CUDA events on
-            the launch stream, inputs and outputs rotated over enough buffer
-            sets that each step misses L2 (max over ranks for N > 1).
-  e2e       the same metric through the public host-buffer call merge_host:
-            each step copies its partials from pinned host memory to the GPU
-            and the result back, in 8 batch slices overlapped with the merge.
+            inputs resident in HBM: W untimed launches, then 5 trials of K
+            back-to-back launches, each timed with CUDA events on the launch
+            stream; the median trial is reported (max over ranks for N > 1).
+            Inputs and outputs rotate over enough buffer sets that each step
+            misses L2.
+  e2e       the same metric through the host-buffer call of the C ABI,
+            lse_merge_host (via merge_host): each step copies its partials
+            from pinned host memory to the GPU and the result back, in 8
+            batch slices overlapped with the merge.
   roofline  the kernel's achieved GB/s against the measured HBM copy peak,
             and its DRAM traffic from the committed ncu summary.
-  workloads eager and CUDA-graph-replayed us/call, GB/s and fraction of
-            peak of every workload.
-  state_update  the in-place fold of one partial into an accumulator.
-  cpu_baseline  the fp64 CPU oracle on a bounded sample (rank 0, N = 1).
+  cpu_baseline  the fp64 CPU oracle on a bounded sample (rank 0, N = 1), on
+            every host core and on one.
+  state_update, decode_attention, cp_exchange_merge
+            the rows built beside the merge.
+  workloads (last key) every merge workload: eager and CUDA-graph-replayed
+            us/call (median of 5 trials; eager 200 calls, graph 100 calls x
+            50 replays), GB/s and fraction of peak from the graph time, and
+            the largest error against the fp64 oracle over every output.
 
 With --gpus N under torchrun every rank merges its own batch (the rows are
 independent; no collective touches the data, NCCL only times the job).
@@ -58,14 +65,15 @@ def log(*a):
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=5000)
+    p.add_argument("--steps", type=int, default=1000)
     p.add_argument("--warmup", type=int, default=50)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default=None, help="workload name (default: the large merge)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-extra", action="store_true", help="skip latency / per-workload lines")
-    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--cpu-seconds", type=float, default=8.0)
+    p.add_argument("--trials", type=int, default=5, help="timed trials per loop (median reported)")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--decode-only", default=None, metavar="SHAPE",
                    help="only time the decode-attention shape SHAPE (for profiling)")
@@ -283,31 +291,40 @@ def n_sets(bytes_per_set: int, l2_bytes: int) -> int:
     return int(min(256, max(2, math.ceil(2 * l2_bytes / max(bytes_per_set, 1)) + 1)))
 
 
-def time_eager(sets: DeviceSets, steps: int, warmup: int, device):
-    """Run `warmup` then `steps` back-to-back launches on the current stream;
-    returns (region_ms, t0, t1).  One kernel launch per step, so region/steps
-    is the kernel's average launch duration; no event sits between launches
-    (an event record between two launches would serialise them)."""
+def time_eager(sets: DeviceSets, steps: int, warmup: int, device, trials: int = 1):
+    """Run `warmup` launches, then `trials` times `steps` back-to-back launches
+    on the current stream, each trial between two CUDA events; returns
+    (list of region ms per trial, t0, t1) with t0/t1 the host times around all
+    trials.  One kernel launch per step, so region/steps is the kernel's
+    average launch duration; no event sits between launches (an event record
+    between two launches would serialise them)."""
     import torch
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
     for i in range(warmup):
         sets.launch(i, sh)
     torch.cuda.synchronize(device)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    regions = []
     t0 = time.perf_counter()
-    e0.record(stream)
-    for i in range(steps):
-        sets.launch(warmup + i, sh)
-    e1.record(stream)
-    torch.cuda.synchronize(device)
+    k = warmup
+    for _ in range(trials):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            sets.launch(k, sh)
+            k += 1
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        regions.append(e0.elapsed_time(e1))
     t1 = time.perf_counter()
-    return e0.elapsed_time(e1), t0, t1
+    return regions, t0, t1
 
 
-def time_graph(sets: DeviceSets, calls: int, replays: int, device) -> float:
-    """us per call of `calls` merges captured in one CUDA graph, replayed."""
+def time_graph(sets: DeviceSets, calls: int, replays: int, device, trials: int = 5):
+    """us per call of `calls` merges captured in one CUDA graph and replayed
+    `replays` times, median over `trials` timed rounds; returns
+    (median us, host t0, host t1)."""
     import torch
     s = torch.cuda.Stream(device)
     s.wait_stream(torch.cuda.current_stream(device))
@@ -323,16 +340,20 @@ def time_graph(sets: DeviceSets, calls: int, replays: int, device) -> float:
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize(device)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(replays):
-        g.replay()
-    e1.record()
-    torch.cuda.synchronize(device)
-    us = e0.elapsed_time(e1) * 1000.0 / (calls * replays)
+    us = []
+    t0 = time.perf_counter()
+    for _ in range(trials):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(replays):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize(device)
+        us.append(e0.elapsed_time(e1) * 1000.0 / (calls * replays))
+    t1 = time.perf_counter()
     del g
-    return us
+    return statistics.median(us), t0, t1
 
 
 def time_e2e(inp: dict, steps: int, device, chunks: int = 8) -> dict:
@@ -364,22 +385,26 @@ def time_e2e(inp: dict, steps: int, device, chunks: int = 8) -> dict:
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
     e0.record()
     for _ in range(steps):
         step()
     e1.record()
     torch.cuda.synchronize(device)
+    t1 = time.perf_counter()
     ms = e0.elapsed_time(e1) / steps
     w = inp["workload"]
     return {"ms_per_step": ms, "gbs": w.bytes_total() / (ms * 1e-3) / 1e9,
             "h2d_bytes_per_step": int(h_o.numel() * h_o.element_size() + h_l.numel() * 4),
             "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size() + h_out_lse.numel() * 4),
-            "steps": steps, "chunks": chunks}
+            "steps": steps, "chunks": chunks, "t0": t0, "t1": t1}
 
 
 def sample_inputs(inp: dict, batches: int) -> dict:
     """The first `batches` batches of a [B,H,R,D] workload (a contiguous prefix)."""
     w = inp["workload"]
+    if batches >= w.B:
+        return inp
     assert w.layout == "bhrd"
     per_b_o = w.H * w.R * w.D
     per_b_l = w.H * w.R
@@ -390,9 +415,10 @@ def sample_inputs(inp: dict, batches: int) -> dict:
     return s
 
 
-def oracle_seconds(inp: dict, budget_s: float):
-    """Run the fp64 oracle over `inp` repeatedly for at least budget_s; returns
-    (bytes/s, passes, seconds)."""
+def oracle_seconds(inp: dict, budget_s: float, threads: int = 1):
+    """Run the fp64 oracle over `inp` repeatedly for at least budget_s, on
+    `threads` host threads (0: one per core); returns (bytes/s, passes,
+    seconds, threads used)."""
     import oracle
     from lse_weighted_merge_b200 import synth
     w = inp["workload"]
@@ -400,15 +426,64 @@ def oracle_seconds(inp: dict, budget_s: float):
         inp["B"] * inp["H"] * (inp["D"] * synth.ELEM_BYTES[w.out_dtype] + 4)
     lib = oracle.load()
     passes = 0
+    st = {}
     t0 = time.perf_counter()
     while True:
         oracle.merge(inp["o"], inp["lse"], inp["R"], inp["B"], inp["H"], inp["D"], inp["o_strides"],
-                     inp["lse_strides"], synth.DTYPES[w.in_dtype], lib=lib)
+                     inp["lse_strides"], synth.DTYPES[w.in_dtype], lib=lib, threads=threads, stats=st)
         passes += 1
         dt = time.perf_counter() - t0
         if dt >= budget_s:
             break
-    return byts * passes / dt, passes, dt
+    return byts * passes / dt, passes, dt, st.get("threads", 1)
+
+
+def cpu_baselines(inp: dict, batches: int, seconds: float) -> dict:
+    """The oracle on the first `batches` batches of the workload, on every
+    host core (the reported value) and on one core; each leg runs for about
+    `seconds`."""
+    w = inp["workload"]
+    smp = sample_inputs(inp, batches)
+    what = f"first {batches} of {w.B} batches ({batches * w.H} of {w.rows} rows)"
+    bps_n, passes_n, secs_n, used = oracle_seconds(smp, seconds, threads=0)
+    bps_1, passes_1, secs_1, _ = oracle_seconds(smp, seconds, threads=1)
+    return {"value": bps_n / 1e9, "unit": "GB/s", "cores": used, "kind": "oracle",
+            "sample": (f"{what}, {passes_n} passes in {secs_n:.1f} s, fp64 C oracle, batches split "
+                       f"over {used} host threads"),
+            "single_thread": {"value": bps_1 / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                              "sample": f"{what}, {passes_1} passes in {secs_1:.1f} s, one thread"},
+            "cpu": cpu_model(), "host_cores": os.cpu_count()}
+
+
+def oracle_errors(captured: dict) -> dict:
+    """Largest error of each workload's GPU output (captured after its timing)
+    against the fp64 oracle over every output element: |gpu - oracle| /
+    (1 + |oracle|) and the merged-lse error over its bound max(1e-5, 2^-22
+    |lse|); empty rows must give exactly 0 and -inf.  The oracle runs on every
+    host core (the batches split over threads, each calling the unchanged
+    oracle)."""
+    import numpy as np
+    import oracle
+    from lse_weighted_merge_b200 import synth
+    lib = oracle.load()
+    tol = {"bf16": 4e-3, "f16": 4e-3, "f32": 1e-5}
+    res = {}
+    for name, (inp, got, got_lse) in captured.items():
+        want, want_lse = oracle.merge(inp["o"], inp["lse"], inp["R"], inp["B"], inp["H"], inp["D"],
+                                      inp["o_strides"], inp["lse_strides"],
+                                      synth.DTYPES[inp["in_dtype"]], lib=lib, threads=0)
+        err = float(np.max(np.abs(got - want) / (1.0 + np.abs(want))))
+        empty = want_lse == -np.inf
+        wl = want_lse[~empty]
+        lerr = float(np.max(np.abs(got_lse[~empty] - wl) / np.maximum(1e-5, 2.0 ** -22 * np.abs(wl)))) \
+            if wl.size else 0.0
+        empty_ok = bool(np.array_equal(got_lse == -np.inf, empty) and np.all(got[empty] == 0.0))
+        t = tol[inp["out_dtype"]]
+        res[name] = {"max_scaled_err": err, "tol": t, "lse_err_over_bound": lerr,
+                     "empty_rows": int(empty.sum()), "empty_rows_ok": empty_ok,
+                     "nan": bool(np.isnan(got).any() or np.isnan(got_lse).any()),
+                     "ok": bool(err <= t and lerr <= 1.0 and empty_ok)}
+    return res
 
 
 def _timed(fn, budget_s: float):
@@ -477,16 +552,18 @@ def run_reference(args):
     name = args.workload or synth.LARGE
     w = synth.WORKLOADS[name]
     inp = synth.make_inputs(w)
-    batches = max(1, w.B // 16)
+    batches = w.B   # the whole workload: one step of the oracle is one merge of the batch
     smp = sample_inputs(inp, batches)
     import oracle
     lib = oracle.load()
     sbytes = w.R * batches * w.H * (w.D * synth.ELEM_BYTES[w.in_dtype] + 4) + \
         batches * w.H * (w.D * synth.ELEM_BYTES[w.out_dtype] + 4)
 
+    st = {}
+
     def one():
         oracle.merge(smp["o"], smp["lse"], w.R, batches, w.H, w.D, smp["o_strides"],
-                     smp["lse_strides"], synth.DTYPES[w.in_dtype], lib=lib)
+                     smp["lse_strides"], synth.DTYPES[w.in_dtype], lib=lib, threads=0, stats=st)
 
     for _ in range(args.warmup):
         one()
@@ -496,15 +573,16 @@ def run_reference(args):
     dt = time.perf_counter() - t0
     ms = dt * 1e3 / args.steps
     gbs = sbytes * args.steps / dt / 1e9
-    sample = (f"first {batches} of {w.B} batches ({batches * w.H} of {w.rows} rows) per step, "
-              "fp64 C oracle, single thread")
+    used = st.get("threads", 1)
+    sample = (f"all {w.B} batches ({w.rows} rows) per step, fp64 C oracle, batches split over "
+              f"{used} host threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(w, args.gpus, "no GPU (host cores)"),
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
-                         "cpu": cpu_model(), "host_cores": os.cpu_count()},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle",
+                         "sample": sample, "cpu": cpu_model(), "host_cores": os.cpu_count()},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -543,20 +621,23 @@ def run_ours(args):
     clock = ClockSampler(device)
     clock.start()
     attempts = []
+    trials = max(1, args.trials)
     for attempt in range(2):
         barrier(dist, device)
         torch.cuda.synchronize(device)
-        region_ms, t0, t1 = time_eager(sets, args.steps, args.warmup, device)
+        regions, t0, t1 = time_eager(sets, args.steps, args.warmup, device, trials)
         barrier(dist, device)
-        region_ms = max_over_ranks(region_ms, dist, device)
+        # every rank takes the same collective steps: one max per trial
+        regions = [max_over_ranks(r, dist, device) for r in regions]
         clk = clock.summary(t0, t1)
-        attempts.append((region_ms, clk))
+        attempts.append((regions, clk))
         bad = [r for r in clk.get("reasons", []) if r in BAD_REASONS]
         bad_flag = max_over_ranks(1.0 if bad else 0.0, dist, device)
         if bad_flag == 0.0:
             break
         log(f"clock reasons {bad} during the timed region: measuring once more")
-    region_ms, clk = attempts[-1]
+    regions, clk = attempts[-1]
+    region_ms = statistics.median(regions)
     launch_ms = region_ms / args.steps
     if len(attempts) > 1:
         clk["remeasured"] = True
@@ -577,24 +658,31 @@ def run_ours(args):
                "h2d_bytes_per_step": r["h2d_bytes_per_step"],
                "d2h_bytes_per_step": r["d2h_bytes_per_step"], "ms_per_step": ms_e2e,
                "steps": r["steps"], "chunks": r["chunks"],
-               "api": "lse_weighted_merge_b200.merge_host(pipeline=True) (pinned host tensors in and out)"}
+               "api": ("lse_merge_host (C ABI: chunked uploads, merges and copies back on its own "
+                       "streams) through lse_weighted_merge_b200.merge_host(pipeline=True), pinned "
+                       "host tensors in and out"),
+               "clocks": clock.summary(r["t0"], r["t1"])}
 
-    extra = {}
+    extra, captured = {}, {}
     if not args.no_extra:
-        extra = extra_workloads(device, l2, dist)
+        extra, captured = extra_workloads(device, l2, dist, clock, trials)
     clock.stop()
-    if extra and rank == 0 and world == 1 and not args.no_cpu_baseline:
-        next_rows_cpu_baselines(extra)
+    del sets
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        batches = max(1, w.B // 8)
-        smp = sample_inputs(inp, batches)
-        bps, passes, secs = oracle_seconds(smp, args.cpu_seconds)
-        cpu = {"value": bps / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": (f"first {batches} of {w.B} batches ({batches * w.H} of {w.rows} rows), "
-                          f"{passes} passes in {secs:.1f} s, fp64 C oracle, single thread"),
-               "cpu": cpu_model(), "host_cores": os.cpu_count()}
+        if extra:
+            next_rows_cpu_baselines(extra)
+            errs = oracle_errors(captured)
+            for wname, row in extra["workload_detail"].items():
+                row["oracle"] = errs.get(wname)
+            for wname, row in extra["workloads"].items():
+                e = errs.get(wname)
+                if e:
+                    row.update({"err": _r(e["max_scaled_err"], 3), "tol": e["tol"],
+                                "lse_err": _r(e["lse_err_over_bound"], 3), "ok": e["ok"]})
+        cpu = cpu_baselines(inp, max(1, w.B // 8), args.cpu_seconds)
 
     if dist is not None:
         barrier(dist, device)
@@ -606,6 +694,8 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": config_block(w, world, l2_note),
+        "trials": {"count": trials, "steps_each": args.steps, "reported": "median",
+                   "region_ms": regions},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                      "traffic_source": traffic_src, "kernel_us": launch_ms * 1e3,
@@ -614,49 +704,76 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps,
+        "gpu_launches_note": "one merge kernel per step; each of the trials times exactly `steps` launches",
         "clocks": clk,
+        "gpu": torch.cuda.get_device_name(device),
         **extra,
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def extra_workloads(device, l2: int, dist) -> dict:
-    """us/call of the two tiny decode shapes (eager and graph replay) and GB/s of
-    the mid-size shapes (eager, L2 rotated)."""
+def _r(x, digits: int = 4):
+    """x rounded to `digits` significant digits (None stays None)."""
+    return None if x is None else float(f"{x:.{digits}g}")
+
+
+def extra_workloads(device, l2: int, dist, clock, trials: int = 5):
+    """Every merge workload: eager us/call (200 back-to-back calls) and
+    CUDA-graph-replayed us/call (100 calls x 50 replays), each the median of
+    `trials` rounds, inputs rotated past L2 except for the two latency shapes
+    (L2-resident, as a decode step's merge would be).  Returns (extra keys of
+    the JSON line, {workload: (inputs, output, merged lse)} of one call for the
+    oracle comparison).  The compact `workloads` block is placed last."""
+    import numpy as np
     import torch
     from lse_weighted_merge_b200 import synth
-    res = {}
+    detail, compact, captured = {}, {}, {}
     peak, _ = hbm_peak()
     for name, w in synth.WORKLOADS.items():
         inp = synth.make_inputs(w)
         tiny = w.bytes_total() < 1 << 20
         nset = 4 if tiny else n_sets(w.bytes_total(), l2)
         sets = DeviceSets(inp, nset, device)
-        region, _, _ = time_eager(sets, 400 if tiny else 200, 20, device)
-        eager_us = region * 1e3 / (400 if tiny else 200)
-        row = {"eager_us_per_call": eager_us, "gbs": w.bytes_total() / (eager_us * 1e-6) / 1e9,
-               "l2": "resident (latency shape)" if tiny else f"rotating {nset} sets"}
-        row["frac_of_measured_hbm"] = row["gbs"] / peak
-        row["graph_us_per_call"] = time_graph(sets, 100, 20 if tiny else 5, device)
-        row["graph_gbs"] = w.bytes_total() / (row["graph_us_per_call"] * 1e-6) / 1e9
-        res[name] = row
+        # one call on set 0 for the comparison with the oracle
+        sets.launch(0, torch.cuda.current_stream(device).cuda_stream)
+        torch.cuda.synchronize(device)
+        captured[name] = (inp, sets.out[0].double().cpu().numpy(),
+                          sets.out_lse[0].double().cpu().numpy())
+        regions, e_t0, e_t1 = time_eager(sets, 200, 20, device, trials)
+        eager_us = statistics.median(regions) * 1e3 / 200
+        graph_us, g_t0, g_t1 = time_graph(sets, 100, 50, device, trials)
+        mhz = clock.summary(g_t0, g_t1).get("sm_mhz")
+        gbs = w.bytes_total() / (graph_us * 1e-6) / 1e9
+        detail[name] = {
+            "eager_us_per_call": eager_us, "eager_trials_us": [r * 1e3 / 200 for r in regions],
+            "graph_us_per_call": graph_us, "graph": "100 calls captured, 50 replays, median of trials",
+            "gbs_graph": gbs, "gbs_eager": w.bytes_total() / (eager_us * 1e-6) / 1e9,
+            "frac_of_measured_hbm_graph": gbs / peak, "bytes_per_call": w.bytes_total(),
+            "sm_mhz_graph": mhz, "graph_kcycles": graph_us * mhz / 1e3 if mhz else None,
+            "l2": "resident (latency shape)" if tiny else f"rotating {nset} sets"}
+        compact[name] = {"eager_us": _r(eager_us), "graph_us": _r(graph_us), "gbs": _r(gbs),
+                         "frac": _r(gbs / peak, 3), "mhz": mhz}
         del sets
         torch.cuda.empty_cache()
-    return {"workloads": res, "state_update": time_state_update(device, l2, peak),
-            "decode_attention": time_decode_attention(device, peak),
-            "cp_exchange_merge": time_cp_exchange(device, peak)}
+    extra = {"state_update": time_state_update(device, l2, peak, trials=trials),
+             "decode_attention": time_decode_attention(device, peak, trials=trials),
+             "cp_exchange_merge": time_cp_exchange(device, peak, trials=trials),
+             "workload_detail": detail,
+             "workloads": compact}
+    return extra, captured
 
 
-def time_cp_exchange(device, peak: float, only: str | None = None) -> dict:
+def time_cp_exchange(device, peak: float, only: str | None = None, trials: int = 5) -> dict:
     """Context-parallel exchange + merge with every rank on this one GPU, all
     ranks played by one cooperative launch (lse_merge_cp_exchange_merge):
-    us/call eager (a prepared CPMergeCall: one launch per call) and
-    graph-replayed.  Bytes per call on one GPU: every
-    rank's partials read once, the (world-1)/world of them owned elsewhere
-    written to and read back from the workspaces, the outputs written.  On
-    world GPUs the same kernel would move the (world-1)/world share over
-    NVLink instead; that cannot be measured here."""
+    us/call eager (a prepared CPMergeCall: one launch per call, 200 calls)
+    and graph-replayed (20 calls captured, 50 replays), each the median of
+    `trials` rounds.  Bytes per call on one GPU: every rank's partials read
+    once, the (world-1)/world of them owned elsewhere written to and read back
+    from the workspaces, the outputs written.  On world GPUs the same kernel
+    would move the (world-1)/world share over NVLink instead; that cannot be
+    measured here."""
     import torch
     from lse_weighted_merge_b200 import cp, synth
     res = {}
@@ -681,14 +798,16 @@ def time_cp_exchange(device, peak: float, only: str | None = None) -> dict:
             call()
         torch.cuda.synchronize(device)
         n = 200
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(n):
-            call()
-        e1.record()
-        torch.cuda.synchronize(device)
-        eager = e0.elapsed_time(e1) * 1e3 / n
+        eager = []
+        for _ in range(trials):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                call()
+            e1.record()
+            torch.cuda.synchronize(device)
+            eager.append(e0.elapsed_time(e1) * 1e3 / n)
         g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(device)
         side.wait_stream(torch.cuda.current_stream(device))
@@ -701,18 +820,23 @@ def time_cp_exchange(device, peak: float, only: str | None = None) -> dict:
         for _ in range(3):
             g.replay()
         torch.cuda.synchronize(device)
-        e0.record()
-        for _ in range(10):
-            g.replay()
-        e1.record()
-        torch.cuda.synchronize(device)
-        graph = e0.elapsed_time(e1) * 1e3 / (10 * reps)
+        graph = []
+        for _ in range(trials):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(50):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize(device)
+            graph.append(e0.elapsed_time(e1) * 1e3 / (50 * reps))
         status = [cp.cp_status(x) for x in ws]
+        gu = statistics.median(graph)
         res[name] = {"shape": f"world={W} B={B} H={H} D={D} {w.in_dtype}, all ranks in one launch",
-                     "eager_us_per_call": eager, "graph_us_per_call": graph,
+                     "eager_us_per_call": statistics.median(eager), "graph_us_per_call": gu,
                      "bytes_per_call_one_gpu": byts,
-                     "graph_gbs": byts / (graph * 1e-6) / 1e9,
-                     "frac_of_measured_hbm_graph": byts / (graph * 1e-6) / 1e9 / peak,
+                     "graph_gbs": byts / (gu * 1e-6) / 1e9,
+                     "frac_of_measured_hbm_graph": byts / (gu * 1e-6) / 1e9 / peak,
                      "nvlink_bytes_per_rank_if_distributed": part // W * (W - 1) // W,
                      "timeouts": sum(1 for x in status if x)}
         del g, call, ws, lo, ll, o, l
@@ -726,70 +850,96 @@ DECODE_SHAPES = (  # name, B, Hq, Hkv, L, D, R
 )
 
 
-def time_decode_attention(device, peak: float, only: str | None = None) -> dict:
-    """Split-KV decode attention producing and merging the partials: fused
-    (one cluster kernel, the merge in distributed shared memory) against
+def time_decode_attention(device, peak: float, only: str | None = None, trials: int = 5) -> dict:
+    """Split-KV decode attention producing and merging the partials, three
+    ways: fused (one launch; each split's partial goes to a workspace and the
+    last split of each (b, KV head) merges them), cluster (one launch; the
+    splits form a cluster and merge in distributed shared memory) and
     unfused (the partials kernel, then lse_merge).  Algorithmic bytes per call:
-    K and V once (B*Hkv*L*D*2*2), q and the output once; the caches exceed L2,
-    so no rotation is needed."""
+    K and V once (B*Hkv*L*D*2*2), q and the output once.  Two input/output
+    sets alternate from call to call, so every call reads its 1.07 GB of K/V
+    from HBM (the other set's 1.07 GB has passed through the 126 MB L2 in
+    between).  50 calls per trial, median of `trials`."""
     import torch
     from lse_weighted_merge_b200 import _native as nat
     res = {}
+    nsets = 2
     for name, B, Hq, Hkv, L, D, R in DECODE_SHAPES:
         if only is not None and name != only:
             continue
         gen = torch.Generator(device=device).manual_seed(7)
-        q = torch.randn((B, Hq, D), generator=gen, device=device).to(torch.bfloat16)
-        k = torch.randn((B, Hkv, L, D), generator=gen, device=device).to(torch.bfloat16)
-        v = torch.randn((B, Hkv, L, D), generator=gen, device=device).to(torch.bfloat16)
-        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=device)
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
-        po = torch.empty((B, Hq, R, D), dtype=torch.float32, device=device)
-        pl = torch.empty((B, Hq, R), dtype=torch.float32, device=device)
+        sets = []
+        for _ in range(nsets):
+            q = torch.randn((B, Hq, D), generator=gen, device=device).to(torch.bfloat16)
+            k = torch.randn((B, Hkv, L, D), generator=gen, device=device).to(torch.bfloat16)
+            v = torch.randn((B, Hkv, L, D), generator=gen, device=device).to(torch.bfloat16)
+            out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=device)
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
+            po = torch.empty((B, Hq, R, D), dtype=torch.float32, device=device)
+            pl = torch.empty((B, Hq, R), dtype=torch.float32, device=device)
+            ws = torch.zeros(nat.decode_workspace_bytes(B, Hq, Hkv, R, D), dtype=torch.uint8,
+                             device=device)
+            sets.append((q, k, v, out, lse, po, pl, ws))
         s = torch.cuda.current_stream(device).cuda_stream
         scale = 1.0 / math.sqrt(D)
         byts = B * Hkv * L * D * 2 * 2 + B * Hq * D * 2 * 2 + B * Hq * 4
 
-        def fused():
+        def fused(i):
+            q, k, v, out, lse, _, _, ws = sets[i % nsets]
+            nat.decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), 0, B, Hq, Hkv, L, D, R,
+                           scale, None, nat.BF16, out.data_ptr(), lse.data_ptr(), s, fused=True,
+                           out_dtype=nat.BF16, workspace=ws.data_ptr(), workspace_bytes=ws.numel())
+
+        def cluster(i):
+            q, k, v, out, lse, _, _, _ = sets[i % nsets]
             nat.decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), 0, B, Hq, Hkv, L, D, R,
                            scale, None, nat.BF16, out.data_ptr(), lse.data_ptr(), s, fused=True,
                            out_dtype=nat.BF16)
 
-        def unfused():
+        def unfused(i):
+            q, k, v, out, lse, po, pl, _ = sets[i % nsets]
             nat.decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), 0, B, Hq, Hkv, L, D, R,
                            scale, None, nat.BF16, po.data_ptr(), pl.data_ptr(), s, fused=False)
             nat.merge_raw(po.data_ptr(), pl.data_ptr(), R, B, Hq, D, None, nat.F32, nat.BF16,
                           out.data_ptr(), lse.data_ptr(), s)
 
         row = {"shape": f"B={B} Hq={Hq} Hkv={Hkv} L={L} D={D} splits={R}, bf16",
-               "bytes_per_call": byts}
-        for tag, fn, n in (("fused", fused, 50), ("unfused", unfused, 50)):
-            for _ in range(5):
-                fn()
+               "bytes_per_call": byts, "l2": f"{nsets} input sets alternating (K/V past L2)"}
+        n = 50
+        for tag, fn in (("fused", fused), ("cluster", cluster), ("unfused", unfused)):
+            for i in range(4):
+                fn(i)
             torch.cuda.synchronize(device)
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(n):
-                fn()
-            e1.record()
-            torch.cuda.synchronize(device)
-            us = e0.elapsed_time(e1) * 1e3 / n
-            row[tag] = {"us_per_call": us, "gbs": byts / (us * 1e-6) / 1e9,
-                        "frac_of_measured_hbm": byts / (us * 1e-6) / 1e9 / peak,
-                        "launches_per_call": 1 if tag == "fused" else 2}
+            us = []
+            for _ in range(trials):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for i in range(n):
+                    fn(i)
+                e1.record()
+                torch.cuda.synchronize(device)
+                us.append(e0.elapsed_time(e1) * 1e3 / n)
+            u = statistics.median(us)
+            row[tag] = {"us_per_call": u, "gbs": byts / (u * 1e-6) / 1e9,
+                        "frac_of_measured_hbm": byts / (u * 1e-6) / 1e9 / peak,
+                        "launches_per_call": 2 if tag == "unfused" else 1}
+        row["fused_over_unfused"] = row["fused"]["us_per_call"] / row["unfused"]["us_per_call"]
+        row["cluster_over_unfused"] = row["cluster"]["us_per_call"] / row["unfused"]["us_per_call"]
         res[name] = row
-        del q, k, v
+        del sets
         torch.cuda.empty_cache()
     return res
 
 
-def time_state_update(device, l2: int, peak: float, B: int = 512, H: int = 16, D: int = 512) -> dict:
+def time_state_update(device, l2: int, peak: float, B: int = 512, H: int = 16, D: int = 512,
+                      trials: int = 5) -> dict:
     """In-place fold of one bf16 partial into an fp32 accumulator of B*H rows
-    (lse_merge_state_update), eager, inputs rotated past L2.  Algorithmic bytes
-    per call: B*H*(D*(4+2+4) + 12) (accumulator read and written, partial
-    read, three lse values).  lse_new starts equal to lse_acc, so the new
-    partial keeps a weight of about 1/k after k folds and is always read."""
+    (lse_merge_state_update), eager, inputs rotated past L2, 200 calls per
+    trial, median of `trials`.  Algorithmic bytes per call:
+    B*H*(D*(4+2+4) + 12) (accumulator read and written, partial read, three
+    lse values).  lse_new starts equal to lse_acc, so the new partial keeps a
+    weight of about 1/k after k folds and is always read."""
     import torch
     from lse_weighted_merge_b200 import _native as nat
     per = B * H * (D * 10 + 12)
@@ -809,18 +959,23 @@ def time_state_update(device, l2: int, peak: float, B: int = 512, H: int = 16, D
     for i in range(20):
         launch(i)
     torch.cuda.synchronize(device)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     n = 200
-    e0.record()
-    for i in range(n):
-        launch(i)
-    e1.record()
-    torch.cuda.synchronize(device)
-    us = e0.elapsed_time(e1) * 1e3 / n
-    gbs = per / (us * 1e-6) / 1e9
+    us = []
+    k = 20
+    for _ in range(trials):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            launch(k)
+            k += 1
+        e1.record()
+        torch.cuda.synchronize(device)
+        us.append(e0.elapsed_time(e1) * 1e3 / n)
+    u = statistics.median(us)
+    gbs = per / (u * 1e-6) / 1e9
     return {"shape": f"B={B} H={H} D={D}, fp32 accumulator, bf16 partial",
-            "eager_us_per_call": us, "gbs": gbs, "frac_of_measured_hbm": gbs / peak,
+            "eager_us_per_call": u, "gbs": gbs, "frac_of_measured_hbm": gbs / peak,
             "bytes_per_call": per, "l2": f"rotating {nset} sets"}
 
 

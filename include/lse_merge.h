@@ -25,7 +25,8 @@
  * allocates nothing, keeps no pointer after returning, never synchronises
  * the host, and only enqueues work on `stream`, so a call can be captured in
  * a CUDA graph.  The exceptions are the set-up calls of the context-parallel
- * exchange (lse_merge_cp_workspace_create and the IPC calls), which say so.
+ * exchange (lse_merge_cp_workspace_create and the IPC calls) and of the
+ * host-buffer merge (lse_merge_host_create / _destroy), which say so.
  */
 #ifndef LSE_MERGE_H
 #define LSE_MERGE_H
@@ -71,6 +72,7 @@ typedef struct {
 #define LSE_MERGE_EUNSUP (-9)   /* a shape the decode-attention kernels do not implement */
 #define LSE_MERGE_ECUDA (-10)   /* a CUDA runtime call of a set-up function failed */
 #define LSE_MERGE_ESCRATCH (-11) /* the problem needs more than the static scratch holds */
+#define LSE_MERGE_EDEVICE (-12)  /* the current device is not the one the context was made on */
 
 /* Kernel paths.  AUTO picks one from the sizes, dtypes and alignment. */
 #define LSE_MERGE_PATH_AUTO 0
@@ -204,15 +206,29 @@ int lse_merge_state_update(void* o_acc, float* lse_acc, const void* o_new, const
  * default), for a separate merge.
  *
  * lse_merge_decode_attention also merges them, inside the same kernel: the
- * R CTAs of one (b, KV head) form a thread-block cluster, each holds its
- * split's partial in shared memory, and after a cluster barrier every CTA
- * merges a slice of D from all R partials through distributed shared memory,
- * so the partials never reach HBM.  R must be 1, 2, 4 or 8.  Output out_o
- * dense [B, Hq, D] of out_dtype and out_lse dense [B, Hq] fp32: attention over
- * keys [0, len_b).
+ * R CTAs of one (b, KV head) form a thread-block cluster; CTAs 1..R-1 store
+ * their split's partial into CTA 0's shared memory (distributed shared
+ * memory) and exit, and CTA 0 merges the R partials, so the partials never
+ * reach HBM.  R must be 1, 2, 4 or 8.  Output out_o dense [B, Hq, D] of
+ * out_dtype and out_lse dense [B, Hq] fp32: attention over keys [0, len_b).
+ * CTA 0's wait for the other partials is bounded (2 s); should it ever run
+ * out, that row's outputs are NaN instead of the kernel hanging.
  *
- * Both return the codes of lse_merge, and LSE_MERGE_EUNSUP for a D, group
- * size, dtype or R outside the above.
+ * lse_merge_decode_attention_ws merges them in the same kernel without a
+ * cluster, through a caller workspace of lse_merge_decode_workspace_bytes()
+ * bytes (16-byte aligned, overlapping no other argument): each split CTA
+ * stores its fp32 partial there and counts itself in a per-(b, KV head)
+ * counter; the CTA that completes the count merges the R partials (still in
+ * L2) and resets the counter.  No CTA waits for another, and any R >= 1 is
+ * accepted.  The workspace must be zeroed once before its first use; every
+ * call leaves it ready for the next one (counters back at 0).  Calls that
+ * may run at the same time on the GPU need workspaces of their own, and a
+ * call that did not complete (a launch error) requires zeroing it again.
+ * Output as for lse_merge_decode_attention.
+ *
+ * All return the codes of lse_merge, and LSE_MERGE_EUNSUP for a D, group
+ * size, dtype or R outside the above; the workspace form also EDIMS for a
+ * workspace shorter than lse_merge_decode_workspace_bytes().
  */
 typedef struct {
     int64_t q_b, q_h;
@@ -229,6 +245,17 @@ int lse_merge_decode_attention(const void* q, const void* k, const void* v, cons
                                int B, int Hq, int Hkv, int L, int D, int R, float scale,
                                const lse_merge_attn_strides* strides, int dtype, int out_dtype,
                                void* out_o, float* out_lse, lse_merge_stream_t stream);
+
+/* Bytes of the workspace of lse_merge_decode_attention_ws: counters [B, Hkv]
+ * (uint32), then the split lse [B, Hq, R] and o [B, Hq, R, D] (fp32). */
+int lse_merge_decode_workspace_bytes(int B, int Hq, int Hkv, int R, int D, int64_t* bytes);
+
+int lse_merge_decode_attention_ws(const void* q, const void* k, const void* v,
+                                  const int32_t* kv_len, int B, int Hq, int Hkv, int L, int D,
+                                  int R, float scale, const lse_merge_attn_strides* strides,
+                                  int dtype, int out_dtype, void* workspace,
+                                  int64_t workspace_bytes, void* out_o, float* out_lse,
+                                  lse_merge_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Context-parallel exchange and merge in one kernel.
@@ -293,6 +320,11 @@ int lse_merge_decode_attention(const void* q, const void* k, const void* v, cons
  * slots) even when the launch plays every rank, which otherwise uses device
  * scope and one slot; this lets one GPU test the multi-GPU protocol. */
 #define LSE_MERGE_CP_FLAG_CROSS_GPU_PROTOCOL 1
+/* For tests of the failure path only: the highest-numbered rank of the call
+ * sends nothing, so every other rank's bounded wait for it runs out after
+ * timeout_ns, sets that sender's bit in the rank's status word and skips
+ * the rank's merge.  The kernel still ends on its own; nothing faults. */
+#define LSE_MERGE_CP_FLAG_TEST_SILENT_LAST_RANK 2
 
 typedef struct {
     int world, rank_begin, rank_count;
@@ -360,14 +392,77 @@ int lse_merge_cp_ipc_close(void* peer_ws);
  *     the GPU (different streams, no ordering between them) race and give
  *     wrong results; order them on one stream;
  *   - the first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and keeps it; make
- *     that first call before any stream capture begins.
+ *     (cudaGetSymbolAddress, with that device current) and keeps it for
+ *     that device's current context (a new context, e.g. after
+ *     cudaDeviceReset, looks it up again); make that first call before any
+ *     stream capture begins.
  * A wait that runs out sets the status word of that rank's workspace inside
- * the array (not readable through this interface); the kernel still returns.
+ * the array and the rank's outputs are left unwritten; the kernel still
+ * returns.  Read the status words with lse_merge_cp_noalloc_status.
  * Returns the codes of lse_merge_cp_exchange_merge, LSE_MERGE_ESCRATCH, and
  * LSE_MERGE_ECUDA when the address look-up or the header clearing fails. */
 #define LSE_MERGE_CP_NOALLOC_SCRATCH_BYTES (16 << 20)
 int lse_merge_cp_exchange_merge_noalloc(const lse_merge_cp_args* args, lse_merge_stream_t stream);
+
+/* The status words of the last lse_merge_cp_exchange_merge_noalloc call on
+ * the current device: status[q], for every rank q < args->world, is 0 when
+ * all of rank q's waits completed (its outputs were written), else bit s is
+ * set for each sender s whose rows never landed (rank q's outputs were not
+ * written).  `args` must describe that call (world, B, H, D and in_dtype
+ * fix where each rank's workspace lies in the array; the pointers are not
+ * read).  Like lse_merge_cp_status it first waits for all work on the
+ * current device, on every stream, then copies the words to the host; it
+ * allocates nothing.  Returns LSE_MERGE_ENULL, the size codes of
+ * lse_merge_cp_exchange_merge_noalloc (EDIMS, EALIGN, ESCRATCH), or
+ * LSE_MERGE_ECUDA when a CUDA call fails.  No counterpart on the pages. */
+int lse_merge_cp_noalloc_status(const lse_merge_cp_args* args, uint32_t* status);
+
+/* ---------------------------------------------------------------------------
+ * The merge of partials that live in host memory.  (No counterpart on the
+ * pages, whose merge reads device memory; it serves callers whose partials
+ * arrive in host memory, and it is what an end-to-end measurement times.)
+ *
+ * A host context, made on the current device by lse_merge_host_create, owns
+ * a device staging area of `stage_bytes` (cudaMalloc), three streams and
+ * their events; lse_merge_host_destroy waits for its last call and frees it
+ * all.  These two are set-up calls: they allocate and synchronise.
+ *
+ * lse_merge_host merges h_partial_o / h_partial_lse, in host memory (pinned,
+ * e.g. cudaMallocHost, for full copy speed; pageable memory works but the
+ * copies then stall the host), into h_out_o [B,H,D] of out_dtype and
+ * h_out_lse [B,H] fp32 in host memory.  The partials are dense in one of two
+ * layouts: LSE_MERGE_LAYOUT_BHRD (o [B,H,R,D], lse [B,H,R]) or
+ * LSE_MERGE_LAYOUT_RBHD (o [R,B,H,D], lse [R,B,H]).  The batch is cut into
+ * `chunks` slices along B (at most LSE_MERGE_HOST_MAX_CHUNKS); slice i is
+ * copied to the staging area while slice i-1 is merged (lse_merge, one
+ * kernel launch) and slice i-2's results are copied back, so the upload of
+ * the partials bounds the call.  The call only enqueues: `stream` is made to
+ * wait for the last copy back, so synchronising `stream` makes the host
+ * outputs valid.  Unless flags has LSE_MERGE_HOST_PIPELINE, the uploads first
+ * wait for the work already on `stream` and for the context's previous call
+ * to finish; with it, when the previous call had the same sizes, slice i
+ * waits only until the previous call has merged slice i (for a stream of
+ * batches: the uploads then follow each other back to back), so the host
+ * inputs must not be written by device work still pending on `stream`.  One
+ * thread at a time per context; not for stream capture.
+ *
+ * lse_merge_host_stage_bytes gives the staging bytes a call of these sizes
+ * needs.  Returns the codes of lse_merge, LSE_MERGE_ESCRATCH when the
+ * context's staging area is too small, LSE_MERGE_EDEVICE when another device
+ * is current, and LSE_MERGE_ECUDA when a CUDA call fails. */
+#define LSE_MERGE_LAYOUT_BHRD 0
+#define LSE_MERGE_LAYOUT_RBHD 1
+#define LSE_MERGE_HOST_MAX_CHUNKS 64
+#define LSE_MERGE_HOST_PIPELINE 1
+typedef struct lse_merge_host_ctx lse_merge_host_ctx;
+int lse_merge_host_stage_bytes(int R, int B, int H, int D, int in_dtype, int out_dtype,
+                               int64_t* bytes);
+int lse_merge_host_create(int64_t stage_bytes, lse_merge_host_ctx** ctx);
+int lse_merge_host_destroy(lse_merge_host_ctx* ctx);
+int lse_merge_host(lse_merge_host_ctx* ctx, const void* h_partial_o, const float* h_partial_lse,
+                   int R, int B, int H, int D, int layout, int in_dtype, int out_dtype,
+                   void* h_out_o, float* h_out_lse, int chunks, int flags,
+                   lse_merge_stream_t stream);
 
 /* A static, human-readable description of a return code. */
 const char* lse_merge_strerror(int code);

@@ -19,10 +19,16 @@ PATH_NAMES = {PATH_VECTOR: "vector", PATH_LATENCY: "latency", PATH_SCALAR: "scal
 
 OK, EDTYPE, EDIMS, ENULL, ESTRIDE, EALIAS, ELAUNCH, EALIGN, EPATH, EUNSUP, ECUDA, ESCRATCH = (
     0, -1, -2, -3, -4, -5, -6, -7, -8, -9, -10, -11)
+EDEVICE = -12
+LAYOUT_BHRD, LAYOUT_RBHD = 0, 1
+HOST_MAX_CHUNKS = 64
+HOST_PIPELINE = 1
 CP_MAX_WORLD = 8
 CP_STATUS_OFFSET = 64
 CP_IPC_HANDLE_BYTES = 64
 CP_FLAG_CROSS_GPU_PROTOCOL = 1
+CP_FLAG_TEST_SILENT_LAST_RANK = 2
+CP_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # Every symbol include/lse_merge.h declares.
 EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merge_state_update",
@@ -31,7 +37,10 @@ EXPORTS = ("lse_merge", "lse_merge_with_path", "lse_merge_plan_query", "lse_merg
            "lse_merge_cp_validate", "lse_merge_cp_exchange_merge", "lse_merge_cp_workspace_create",
            "lse_merge_cp_workspace_destroy", "lse_merge_cp_ipc_handle", "lse_merge_cp_ipc_open",
            "lse_merge_cp_ipc_close", "lse_merge_cp_status", "lse_merge_cp_workspace_zero",
-           "lse_merge_cp_exchange_merge_noalloc")
+           "lse_merge_cp_exchange_merge_noalloc", "lse_merge_cp_noalloc_status",
+           "lse_merge_decode_workspace_bytes", "lse_merge_decode_attention_ws",
+           "lse_merge_host_stage_bytes", "lse_merge_host_create", "lse_merge_host_destroy",
+           "lse_merge_host")
 ABI_VERSION = 4
 
 
@@ -117,6 +126,18 @@ def _load() -> ctypes.CDLL:
     lib.lse_merge_decode_partials.restype = i
     lib.lse_merge_decode_attention.argtypes = attn + [i, vp, vp, vp]
     lib.lse_merge_decode_attention.restype = i
+    lib.lse_merge_decode_attention_ws.argtypes = attn + [i, vp, ctypes.c_int64, vp, vp, vp]
+    lib.lse_merge_decode_attention_ws.restype = i
+    lib.lse_merge_decode_workspace_bytes.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_int64)]
+    lib.lse_merge_decode_workspace_bytes.restype = i
+    lib.lse_merge_host_stage_bytes.argtypes = [i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int64)]
+    lib.lse_merge_host_stage_bytes.restype = i
+    lib.lse_merge_host_create.argtypes = [ctypes.c_int64, ctypes.POINTER(vp)]
+    lib.lse_merge_host_create.restype = i
+    lib.lse_merge_host_destroy.argtypes = [vp]
+    lib.lse_merge_host_destroy.restype = i
+    lib.lse_merge_host.argtypes = [vp, vp, vp, i, i, i, i, i, i, i, vp, vp, i, i, vp]
+    lib.lse_merge_host.restype = i
     lib.lse_merge_strerror.argtypes = [i]
     lib.lse_merge_strerror.restype = ctypes.c_char_p
     lib.lse_merge_last_cuda_error.argtypes = []
@@ -131,6 +152,8 @@ def _load() -> ctypes.CDLL:
     lib.lse_merge_cp_exchange_merge.restype = i
     lib.lse_merge_cp_exchange_merge_noalloc.argtypes = [ctypes.POINTER(CpArgs), vp]
     lib.lse_merge_cp_exchange_merge_noalloc.restype = i
+    lib.lse_merge_cp_noalloc_status.argtypes = [ctypes.POINTER(CpArgs), ctypes.POINTER(ctypes.c_uint32)]
+    lib.lse_merge_cp_noalloc_status.restype = i
     lib.lse_merge_cp_workspace_create.argtypes = [ctypes.c_int64, ctypes.POINTER(vp)]
     lib.lse_merge_cp_workspace_create.restype = i
     lib.lse_merge_cp_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -245,17 +268,62 @@ def _check(rc: int, check: bool) -> int:
 def decode_raw(q_ptr: int, k_ptr: int, v_ptr: int, kv_len_ptr: int, B: int, Hq: int, Hkv: int,
                L: int, D: int, R: int, scale: float, strides, dtype: int, out_ptr: int,
                out_lse_ptr: int, stream: int = 0, fused: bool = True, out_dtype: int = BF16,
-               check: bool = True) -> int:
-    """lse_merge_decode_attention (fused) or lse_merge_decode_partials (fp32
-    partials [B,Hq,R,D] / [B,Hq,R] into out_ptr / out_lse_ptr).  ``strides`` =
-    (q_b, q_h, k_b, k_h, k_l, v_b, v_h, v_l) in elements, or None (dense)."""
+               check: bool = True, workspace: int = 0, workspace_bytes: int = 0) -> int:
+    """lse_merge_decode_attention_ws (fused with a workspace pointer),
+    lse_merge_decode_attention (fused, no workspace: the cluster form) or
+    lse_merge_decode_partials (fp32 partials [B,Hq,R,D] / [B,Hq,R] into
+    out_ptr / out_lse_ptr).  ``strides`` = (q_b, q_h, k_b, k_h, k_l, v_b, v_h,
+    v_l) in elements, or None (dense)."""
     st = None if strides is None else ctypes.pointer(AttnStrides(*[int(x) for x in strides]))
     args = (q_ptr, k_ptr, v_ptr, kv_len_ptr or None, B, Hq, Hkv, L, D, R, float(scale), st, dtype)
-    if fused:
+    if fused and workspace:
+        rc = lib.lse_merge_decode_attention_ws(*args, out_dtype, workspace, int(workspace_bytes),
+                                               out_ptr, out_lse_ptr, stream or None)
+    elif fused:
         rc = lib.lse_merge_decode_attention(*args, out_dtype, out_ptr, out_lse_ptr, stream or None)
     else:
         rc = lib.lse_merge_decode_partials(*args, out_ptr, out_lse_ptr, stream or None)
     return _check(rc, check)
+
+
+def host_stage_bytes(R: int, B: int, H: int, D: int, in_dtype: int, out_dtype: int) -> int:
+    n = ctypes.c_int64(0)
+    rc = lib.lse_merge_host_stage_bytes(R, B, H, D, in_dtype, out_dtype, ctypes.byref(n))
+    if rc != OK:
+        _raise(rc)
+    return n.value
+
+
+def host_create(stage_bytes: int) -> int:
+    """lse_merge_host_create on the current device; returns the context handle."""
+    h = ctypes.c_void_p()
+    rc = lib.lse_merge_host_create(int(stage_bytes), ctypes.byref(h))
+    if rc != OK:
+        _raise(rc)
+    return h.value
+
+
+def host_destroy(ctx: int) -> None:
+    rc = lib.lse_merge_host_destroy(ctx)
+    if rc != OK:
+        _raise(rc)
+
+
+def host_merge_raw(ctx: int, h_o: int, h_lse: int, R: int, B: int, H: int, D: int, layout: int,
+                   in_dtype: int, out_dtype: int, h_out: int, h_out_lse: int, chunks: int,
+                   flags: int = 0, stream: int = 0, check: bool = True) -> int:
+    """lse_merge_host: the pipelined merge of partials in host memory."""
+    rc = lib.lse_merge_host(ctx, h_o, h_lse, R, B, H, D, layout, in_dtype, out_dtype, h_out,
+                            h_out_lse, chunks, flags, stream or None)
+    return _check(rc, check)
+
+
+def decode_workspace_bytes(B: int, Hq: int, Hkv: int, R: int, D: int) -> int:
+    n = ctypes.c_int64(0)
+    rc = lib.lse_merge_decode_workspace_bytes(B, Hq, Hkv, R, D, ctypes.byref(n))
+    if rc != OK:
+        _raise(rc)
+    return n.value
 
 
 def _raise(rc: int):
@@ -296,6 +364,17 @@ def cp_exchange_merge_noalloc_raw(args: CpArgs, stream: int = 0, check: bool = T
     if check and rc != OK:
         _raise(rc)
     return rc
+
+
+def cp_noalloc_status(args: CpArgs, check: bool = True):
+    """lse_merge_cp_noalloc_status: the status word of every rank of the last
+    no-alloc call with these sizes (0: all of that rank's waits completed).
+    Returns (code, [status of rank 0, ..., rank world-1])."""
+    st = (ctypes.c_uint32 * max(1, int(args.world)))()
+    rc = lib.lse_merge_cp_noalloc_status(ctypes.byref(args), st)
+    if check and rc != OK:
+        _raise(rc)
+    return rc, [int(st[q]) for q in range(int(args.world))]
 
 
 def cp_workspace_create(nbytes: int) -> int:

@@ -5,7 +5,8 @@ import threading
 
 from ._native import (BF16, F16, F32, PATH_AUTO, PATH_LATENCY, PATH_SCALAR, PATH_STREAM,
                       PATH_VECTOR,
-                      LseMergeError, decode_raw, merge_raw, plan_query, state_update_raw,
+                      LseMergeError, decode_raw, decode_workspace_bytes, merge_raw, plan_query,
+                      state_update_raw,
                       strerror)
 
 
@@ -79,79 +80,74 @@ def merge(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, out=N
     return out, out_lse
 
 
-_STREAMS: dict = {}
-_WORKSPACE: dict = {}
-# merge_host's caches are shared by every thread; one call at a time per
+# Host contexts of merge_host (lse_merge_host_create), one per device, kept
+# between calls and grown when a call needs a larger staging area.
+# merge_host's contexts are shared by every thread; one call at a time per
 # process uses them (the copies and merges it enqueues still overlap).
+_HOST_CTX: dict = {}
 _HOST_LOCK = threading.Lock()
 
 
 def release_host_workspace() -> None:
-    """Free the device staging buffers merge_host keeps between calls."""
+    """Free the host contexts (device staging areas, streams and events) that
+    merge_host keeps between calls; each waits for its last call first."""
+    from ._native import host_destroy
     with _HOST_LOCK:
-        _WORKSPACE.clear()
+        for (dev_index, _), ctx in list(_HOST_CTX.items()):
+            import torch
+            with torch.cuda.device(dev_index):
+                host_destroy(ctx)
+        _HOST_CTX.clear()
 
 
-def _workspace(device, o_shape, o_dtype, l_shape, B, H, D, out_dtype):
-    """Device staging buffers of merge_host, kept per device for the last
-    shape used (allocating them on every call would stall the stream on the
-    allocator).  Reuse is ordered by the streams: a call's first copy waits
-    for the previous call's last copy."""
+def _host_context(device, need: int) -> int:
+    """The host context of `device`, remade larger when `need` staging bytes
+    exceed its area (the old one is destroyed after its last call)."""
     import torch
-    key = (o_shape, o_dtype, l_shape, B, H, D, out_dtype)
-    ws = _WORKSPACE.get(device)
-    if ws is None or ws["key"] != key:
-        if ws is not None:
-            ws["done"].synchronize()   # the old buffers may still be in use
-        ws = {"key": key, "done": torch.cuda.Event(),
-              "bufs": (torch.empty(o_shape, dtype=o_dtype, device=device),
-                       torch.empty(l_shape, dtype=torch.float32, device=device),
-                       torch.empty((B, H, D), dtype=out_dtype, device=device),
-                       torch.empty((B, H), dtype=torch.float32, device=device))}
-        ws["done"].record(torch.cuda.current_stream(device))
-        _WORKSPACE[device] = ws
-    return ws
-
-
-def _side_streams(device):
-    import torch
-    key = device.index if device.index is not None else torch.cuda.current_device()
-    if key not in _STREAMS:
-        _STREAMS[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device),
-                         torch.cuda.Stream(device))
-    return _STREAMS[key]
+    from ._native import host_create, host_destroy
+    for key in [k for k in _HOST_CTX if k[0] == device.index]:
+        if key[1] >= need:
+            return _HOST_CTX[key]
+        with torch.cuda.device(device):
+            host_destroy(_HOST_CTX.pop(key))
+    with torch.cuda.device(device):
+        ctx = host_create(need)
+    _HOST_CTX[(device.index, need)] = ctx
+    return ctx
 
 
 def merge_host(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, chunks: int = 8,
                device=None, out=None, out_lse=None, sync: bool = True, pipeline: bool = False):
     """Merge partials that live in (pinned) host memory; results land in host memory.
 
-    The batch is cut into ``chunks`` slices along B.  Slice i is copied to the
-    GPU on one stream while slice i-1 is merged (one kernel launch on a second
-    stream) and slice i-2's result is copied back on a third, so the merge and
-    the device-to-host copies hide behind the host-to-device copy of the
-    partials, which bounds the whole call.  Layouts and dtypes as in merge().
+    One call of the C ABI's lse_merge_host on a host context this module
+    keeps per device: the batch is cut into ``chunks`` slices along B; slice
+    i is copied to the GPU on one stream while slice i-1 is merged (one kernel
+    launch on a second stream) and slice i-2's result is copied back on a
+    third, so the merge and the device-to-host copies hide behind the
+    host-to-device copy of the partials, which bounds the whole call.
+    Layouts ("bhrd" [B,H,R,D] or "rbhd" [R,B,H,D], dense) and dtypes as in
+    merge().  Pass pinned ``out``/``out_lse`` to avoid a host allocation per
+    call; pinned inputs for full copy speed.
 
-    Device staging buffers for one call's shapes are kept between calls (see
-    release_host_workspace); pass pinned ``out``/``out_lse`` to avoid a host
-    allocation per call.
-
-    Returns pinned host tensors (out [B, H, D], out_lse [B, H]).  With
+    Returns the host tensors (out [B, H, D], out_lse [B, H]).  With
     ``sync=False`` the call returns once everything is enqueued; the current
     stream of ``device`` is made to wait for the last copy, so synchronising
     that stream (or the device) makes the results valid.
 
     ``pipeline=True`` (with ``sync=False``, for a stream of batches) lets this
     call's uploads start as soon as the previous call's uploads end, instead
-    of after the previous call's last copy back: the staging buffers are
-    reused chunk by chunk once the previous call has merged that chunk and
-    copied its result back.  The uploads then no longer wait for the current
-    stream, so the host inputs must not be written by device work still
-    pending there (inputs filled by the CPU, the usual case, are fine); give
-    consecutive pipelined calls distinct host outputs, or read each call's
-    outputs before the next call's copies back can overwrite them.
+    of after the previous call's last copy back (LSE_MERGE_HOST_PIPELINE):
+    slice i's staging bytes are reused once the previous call has merged
+    slice i.  The uploads then no longer wait for the current stream, so the
+    host inputs must not be written by device work still pending there
+    (inputs filled by the CPU, the usual case, are fine); give consecutive
+    pipelined calls distinct host outputs, or read each call's outputs before
+    the next call's copies back can overwrite them.
     """
     import torch
+    from ._native import (HOST_MAX_CHUNKS, HOST_PIPELINE, LAYOUT_BHRD, LAYOUT_RBHD, host_merge_raw,
+                          host_stage_bytes)
     if partial_o.is_cuda or partial_lse.is_cuda:
         raise ValueError("merge_host takes host tensors; use merge() for device tensors")
     if partial_lse.dtype != torch.float32:
@@ -160,89 +156,31 @@ def merge_host(partial_o, partial_lse, *, layout: str = "bhrd", out_dtype=None, 
     if not (partial_o.is_contiguous() and partial_lse.is_contiguous()):
         raise ValueError("merge_host wants contiguous host tensors")
     device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if device.index is None:
+        device = torch.device("cuda", torch.cuda.current_device())
     out_dtype = out_dtype or partial_o.dtype
     if out is None:
         out = torch.empty((B, H, D), dtype=out_dtype).pin_memory()
     if out_lse is None:
         out_lse = torch.empty((B, H), dtype=torch.float32).pin_memory()
+    if out.is_cuda or out_lse.is_cuda:
+        raise ValueError("merge_host writes host tensors: out and out_lse must be on the CPU")
+    if tuple(out.shape) != (B, H, D) or not out.is_contiguous() or out.dtype != out_dtype:
+        raise ValueError("out must be a contiguous [B, H, D] tensor of out_dtype")
+    if tuple(out_lse.shape) != (B, H) or not out_lse.is_contiguous() or out_lse.dtype != torch.float32:
+        raise ValueError("out_lse must be a contiguous float32 [B, H] tensor")
+    ind, outd = dtype_code(partial_o.dtype), dtype_code(out_dtype)
+    chunks = max(1, min(int(chunks), B, HOST_MAX_CHUNKS))
     with _HOST_LOCK:
-        return _merge_host_locked(partial_o, partial_lse, layout, out_dtype, chunks, device, out,
-                                  out_lse, sync, pipeline, R, B, H, D)
-
-
-def _chunk_events(ws: dict, parity: int, n: int) -> list:
-    """The (landed, merged, copied-back) events of n chunks, in one of two sets
-    that alternate between calls: a call records into one set while the next
-    call waits on it and records into the other."""
-    import torch
-    sets = ws.setdefault("event_sets", [[], []])
-    evs = sets[parity]
-    while len(evs) < n:
-        evs.append((torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()))
-    return evs
-
-
-def _merge_host_locked(partial_o, partial_lse, layout, out_dtype, chunks, device, out, out_lse,
-                       sync, pipeline, R, B, H, D):
-    import torch
-    ws = _workspace(device, tuple(partial_o.shape), partial_o.dtype, tuple(partial_lse.shape),
-                    B, H, D, out_dtype)
-    d_o, d_l, d_out, d_out_lse = ws["bufs"]
-    cur = torch.cuda.current_stream(device)
-    s_in, s_merge, s_back = _side_streams(device)
-    nb = max(1, -(-B // max(1, int(chunks))))
-    n = -(-B // nb)
-    # The previous call's chunk events, if it cut the batch the same way.
-    prev = ws.get("chunks")
-    prev = prev[1] if (pipeline and prev is not None and prev[0] == nb) else None
-    if prev is None:
-        # The staging buffers are free once the previous call's last copy is
-        # done (its `done` event); the host inputs and outputs may be in use
-        # on the current stream.
-        for s_ in (s_in, s_back):
-            s_.wait_event(ws["done"])
-            s_.wait_stream(cur)
-    else:
-        # Pipelined: chunk i's staging buffers are free once the previous call
-        # merged chunk i and copied its result back, so this call's uploads
-        # follow the previous call's without waiting for its last copy back.
-        s_back.wait_stream(cur)      # the host outputs may be in use on the current stream
-    parity = ws.get("parity", 0) ^ 1
-    evs = _chunk_events(ws, parity, n)
-    for i, b0 in enumerate(range(0, B, nb)):
-        b1 = min(B, b0 + nb)
-        landed, merged, copied = evs[i]
-        with torch.cuda.stream(s_in):
-            if prev is not None:
-                s_in.wait_event(prev[i][1])
-            if layout == "bhrd":
-                d_o[b0:b1].copy_(partial_o[b0:b1], non_blocking=True)
-                d_l[b0:b1].copy_(partial_lse[b0:b1], non_blocking=True)
-                vo, vl = d_o[b0:b1], d_l[b0:b1]
-            else:
-                for r in range(R):
-                    d_o[r, b0:b1].copy_(partial_o[r, b0:b1], non_blocking=True)
-                    d_l[r, b0:b1].copy_(partial_lse[r, b0:b1], non_blocking=True)
-                vo, vl = d_o[:, b0:b1], d_l[:, b0:b1]
-            landed.record(s_in)
-        s_merge.wait_event(landed)
-        if prev is not None:
-            s_merge.wait_event(prev[i][2])
-        with torch.cuda.stream(s_merge):
-            merge(vo, vl, layout=layout, out_dtype=out_dtype, out=d_out[b0:b1],
-                  out_lse=d_out_lse[b0:b1])
-            merged.record(s_merge)
-        s_back.wait_event(merged)
-        with torch.cuda.stream(s_back):
-            out[b0:b1].copy_(d_out[b0:b1], non_blocking=True)
-            out_lse[b0:b1].copy_(d_out_lse[b0:b1], non_blocking=True)
-            copied.record(s_back)
-    ws["chunks"] = (nb, evs[:n])
-    ws["parity"] = parity
-    ws["done"].record(s_back)
-    cur.wait_stream(s_back)
+        with torch.cuda.device(device):
+            ctx = _host_context(device, host_stage_bytes(R, B, H, D, ind, outd))
+            s = torch.cuda.current_stream(device)
+            host_merge_raw(ctx, partial_o.data_ptr(), partial_lse.data_ptr(), R, B, H, D,
+                           LAYOUT_BHRD if layout == "bhrd" else LAYOUT_RBHD, ind, outd,
+                           out.data_ptr(), out_lse.data_ptr(), chunks,
+                           HOST_PIPELINE if pipeline else 0, s.cuda_stream)
     if sync:
-        s_back.synchronize()
+        s.synchronize()
     return out, out_lse
 
 
@@ -278,25 +216,44 @@ def merge_state_(o_acc, lse_acc, o_new, lse_new):
     return o_acc, lse_acc
 
 
+# Workspaces of the fused decode attention, one per (device, stream): zeroed
+# once when made, left ready (counters at 0) by every call, so calls on one
+# stream can share one; calls on different streams get different ones.
+_decode_ws: dict = {}
+_decode_ws_lock = threading.Lock()
+
+
+def _decode_workspace(dev, stream_handle: int, nbytes: int):
+    import torch
+    key = (dev.index, stream_handle)
+    with _decode_ws_lock:
+        ws = _decode_ws.get(key)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.zeros(max(nbytes, 1 << 16), dtype=torch.uint8, device=dev)
+            _decode_ws[key] = ws
+        return ws
+
+
 def decode_attention(q, k, v, *, splits: int | None = None, scale: float | None = None,
-                     kv_len=None, out_dtype=None, fused: bool | None = None):
+                     kv_len=None, out_dtype=None, fused: bool | str | None = None):
     """Split-KV decode attention on the GPU, its partials merged by LSE weight.
 
     q [B, Hq, D]; k, v [B, Hkv, L, D] (bf16 or fp16, stride 1 along D, other
     strides free); Hq a multiple of Hkv; D 64 or 128; kv_len an optional int32
     CUDA tensor [B] of valid key counts.  The keys of each sequence are cut
     into ``splits`` shards (default: enough shards for about two CTAs per SM,
-    a power of two of at least 64 keys each).  fused=True merges the shards
-    inside the attention kernel through a thread-block cluster (splits 1, 2,
-    4 or 8); fused=False writes the fp32 partials and merges them with
-    merge(), two launches.  By default the fused kernel is used below 128 MB
-    of keys and values when its splits still give every SM a CTA, where
-    saving a launch matters (measured on B200: 27.4 vs 28.9 us at B=4,
-    L=8192), and the two launches otherwise: above that size cluster
-    scheduling costs more than the second launch (166 vs 176 us at B=64,
-    L=4096), and few sequences need more than 8 splits (B=1 with one KV head
-    and 32768 keys: 15 us at 64 splits, 42 us at 8).  Returns (out [B, Hq, D],
-    lse [B, Hq]) with the natural-log lse of the scaled scores.
+    a power of two of at least 64 keys each, at most 64).
+
+    fused (default True): one launch; each shard's CTA writes its fp32
+    partial into a workspace kept for this device and stream, and the last
+    shard of each (sequence, KV head) to finish merges them
+    (lse_merge_decode_attention_ws).  fused="cluster": one launch in which the
+    shards of a (sequence, KV head) form a thread-block cluster and merge
+    through distributed shared memory, no workspace (splits 1, 2, 4 or 8;
+    cluster scheduling leaves SM slots idle, so it is slower on large
+    batches).  fused=False: the partials kernel, then merge(), two launches.
+    Returns (out [B, Hq, D], lse [B, Hq]) with the natural-log lse of the
+    scaled scores.
     """
     import math
     import torch
@@ -310,17 +267,17 @@ def decode_attention(q, k, v, *, splits: int | None = None, scale: float | None 
         raise ValueError("q, k and v must be contiguous along D")
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share one dtype")
-    dev = q.device
-    kv_bytes = 2 * B * Hkv * L * D * q.element_size()
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     if fused is None:
-        # fused: its (at most 8) splits must still give every SM a CTA
-        fused = (kv_bytes <= (128 << 20) and B * Hkv * 8 >= sms
-                 and (splits is None or splits in (1, 2, 4, 8)))
+        fused = True
+    if fused not in (True, False, "cluster"):
+        raise ValueError("fused must be True, False or 'cluster'")
+    dev = q.device
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     if splits is None:
         want = max(1, -(-2 * sms // (B * Hkv)))
+        cap = 8 if fused == "cluster" else 64
         splits = 1
-        while splits < want and splits < (8 if fused else 64) and splits * 64 < L:
+        while splits < want and splits < cap and splits * 64 < L:
             splits *= 2
     scale = (1.0 / math.sqrt(D)) if scale is None else float(scale)
     out_dtype = out_dtype or q.dtype
@@ -337,9 +294,14 @@ def decode_attention(q, k, v, *, splits: int | None = None, scale: float | None 
         if fused:
             out = torch.empty((B, Hq, D), dtype=out_dtype, device=dev)
             lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+            ws_ptr, ws_bytes = 0, 0
+            if fused is True:
+                ws_bytes = decode_workspace_bytes(B, Hq, Hkv, splits, D)
+                ws_ptr = _decode_workspace(dev, s, ws_bytes).data_ptr()
             decode_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), klen, B, Hq, Hkv, L, D, splits,
                        scale, st, dtype_code(q.dtype), out.data_ptr(), lse.data_ptr(), s,
-                       fused=True, out_dtype=dtype_code(out_dtype))
+                       fused=True, out_dtype=dtype_code(out_dtype), workspace=ws_ptr,
+                       workspace_bytes=ws_bytes)
             return out, lse
         po = torch.empty((B, Hq, splits, D), dtype=torch.float32, device=dev)
         pl = torch.empty((B, Hq, splits), dtype=torch.float32, device=dev)

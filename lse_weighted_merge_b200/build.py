@@ -15,7 +15,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblse_merge.so")
 SOURCES = [os.path.join(CSRC, "plan.cpp"), os.path.join(CSRC, "lse_merge.cu"),
-           os.path.join(CSRC, "decode_attention.cu"), os.path.join(CSRC, "cp_exchange.cu")]
+           os.path.join(CSRC, "decode_attention.cu"), os.path.join(CSRC, "cp_exchange.cu"),
+           os.path.join(CSRC, "host_pipeline.cpp")]
 HEADERS = [os.path.join(INCLUDE, "lse_merge.h"), os.path.join(CSRC, "plan.h"),
            os.path.join(CSRC, "device_common.cuh")]
 

@@ -90,6 +90,7 @@ struct CpParams {
     int64_t chunk;                    // send units per CTA
     unsigned long long share, share0; // arrival shares: CTA 0 share0, the others share
     int local;                        // every rank is played by this launch (one GPU)
+    int silent;                       // a rank that sends nothing (test flag), else -1
     uint64_t c_U, c_dv, c_Hq;         // fastdiv constants of U, dv and Hq
 };
 
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __gri
     // [c*chunk, (c+1)*chunk) of the rank's total.
     const int64_t total = (int64_t)w1 * p.U;
     const int64_t u0 = min(total, cta * p.chunk);
-    const int64_t u1 = min(total, u0 + p.chunk);
+    const int64_t u1 = me == p.silent ? u0 : min(total, u0 + p.chunk);
     int64_t u = u0 + threadIdx.x;
     SendBatch sb;
     load_batch(p, me, u, u1, src_o, src_l, sb);
@@ -443,6 +444,7 @@ int lse_merge_cp_exchange_merge(const lse_merge_cp_args* a, lse_merge_stream_t s
     kp.max_polls = a->timeout_ns / 256 + 1024;
     const int64_t send_units = (int64_t)(a->world - 1) * pl.U;
     kp.local = a->rank_count == a->world && !(a->flags & LSE_MERGE_CP_FLAG_CROSS_GPU_PROTOCOL);
+    kp.silent = (a->flags & LSE_MERGE_CP_FLAG_TEST_SILENT_LAST_RANK) ? a->world - 1 : -1;
     kp.c_U = fastdiv_c((uint32_t)pl.U);
     kp.c_dv = fastdiv_c(kp.dv);
     kp.c_Hq = fastdiv_c((uint32_t)pl.Hq);
@@ -559,33 +561,79 @@ namespace {
 constexpr int64_t kNoAllocBytes = LSE_MERGE_CP_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-// Device address of g_noalloc_scratch, looked up once per device.  In host
-// code the array's name is only a stand-in for the symbol, never an address
-// a kernel may be given.
+// Device address of g_noalloc_scratch, looked up once per device and
+// context.  In host code the array's name is only a stand-in for the symbol,
+// never an address a kernel may be given.  The address is kept with the id
+// of the context it was looked up in (cuCtxGetId, reached through the
+// runtime's driver entry points, so the library needs no libcuda link): a
+// later context on the device (after cudaDeviceReset) looks it up again.
 constexpr int kMaxDevices = 64;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoAllocAddr {
+    void* ptr;
+    unsigned long long ctx_id;   // 0: unknown
+};
+NoAllocAddr g_noalloc[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
+
+using CtxGetCurrentFn = int (*)(void**);                    // cuCtxGetCurrent
+using CtxGetIdFn = int (*)(void*, unsigned long long*);     // cuCtxGetId
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+bool g_ctx_fns_tried = false;
+
+// Id of the current context, or 0 when it cannot be told.  Caller holds g_noalloc_mu.
+unsigned long long current_ctx_id() {
+    if (!g_ctx_fns_tried) {
+        g_ctx_fns_tried = true;
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_id = reinterpret_cast<CtxGetIdFn>(f);
+        (void)cudaGetLastError();
+    }
+    if (!g_ctx_current || !g_ctx_id) return 0;
+    void* ctx = nullptr;
+    unsigned long long id = 0;
+    if (g_ctx_current(&ctx) != 0 || !ctx || g_ctx_id(ctx, &id) != 0) return 0;
+    return id;
+}
 
 int noalloc_scratch(void** ptr) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return (int)e;
-    if (dev >= 0 && dev < kMaxDevices) {
-        std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        if (g_noalloc_ptr[dev]) {
-            *ptr = g_noalloc_ptr[dev];
-            return 0;
-        }
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    const bool cacheable = dev >= 0 && dev < kMaxDevices;
+    const unsigned long long id = current_ctx_id();
+    if (cacheable && id != 0 && g_noalloc[dev].ptr && g_noalloc[dev].ctx_id == id) {
+        *ptr = g_noalloc[dev].ptr;
+        return 0;
     }
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return (int)e;
-    if (dev >= 0 && dev < kMaxDevices) {
-        std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        g_noalloc_ptr[dev] = p;
-    }
+    // The look-up makes the device's primary context current if it was not.
+    const unsigned long long id2 = id != 0 ? id : current_ctx_id();
+    if (cacheable) g_noalloc[dev] = NoAllocAddr{p, id2};
     *ptr = p;
     return 0;
+}
+
+// Where each rank's workspace lies in the array for these sizes: every
+// workspace starts on a 256-byte boundary, `pitch` bytes apart.
+int noalloc_layout(const lse_merge_cp_args* args, int64_t* pitch) {
+    int64_t ws_bytes = 0;
+    const int rc = lse_merge_cp_workspace_bytes(args->world, args->B, args->H, args->D,
+                                                args->in_dtype, &ws_bytes);
+    if (rc != LSE_MERGE_OK) return rc;
+    *pitch = (ws_bytes + 255) / 256 * 256;
+    if ((int64_t)args->world * *pitch > kNoAllocBytes) return LSE_MERGE_ESCRATCH;
+    return LSE_MERGE_OK;
 }
 
 }  // namespace
@@ -595,13 +643,10 @@ extern "C" int lse_merge_cp_exchange_merge_noalloc(const lse_merge_cp_args* args
                                                    lse_merge_stream_t stream) {
     using namespace lsem;
     if (!args) return LSE_MERGE_ENULL;
-    int64_t ws_bytes = 0;
-    int rc = lse_merge_cp_workspace_bytes(args->world, args->B, args->H, args->D, args->in_dtype,
-                                          &ws_bytes);
+    int64_t pitch = 0;
+    int rc = noalloc_layout(args, &pitch);
     if (rc != LSE_MERGE_OK) return rc;
     if (args->rank_begin != 0 || args->rank_count != args->world) return LSE_MERGE_EDIMS;
-    const int64_t pitch = (ws_bytes + 255) / 256 * 256;
-    if ((int64_t)args->world * pitch > kNoAllocBytes) return LSE_MERGE_ESCRATCH;
     void* base = nullptr;
     const int se = noalloc_scratch(&base);
     if (se != 0) return fail_cuda(LSE_MERGE_ECUDA, se);
@@ -617,4 +662,23 @@ extern "C" int lse_merge_cp_exchange_merge_noalloc(const lse_merge_cp_args* args
                                             (size_t)a.world, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(LSE_MERGE_ECUDA, (int)e);
     return lse_merge_cp_exchange_merge(&a, stream);
+}
+
+extern "C" int lse_merge_cp_noalloc_status(const lse_merge_cp_args* args, uint32_t* status) {
+    using namespace lsem;
+    if (!args || !status) return LSE_MERGE_ENULL;
+    int64_t pitch = 0;
+    const int rc = noalloc_layout(args, &pitch);
+    if (rc != LSE_MERGE_OK) return rc;
+    void* base = nullptr;
+    const int se = noalloc_scratch(&base);
+    if (se != 0) return fail_cuda(LSE_MERGE_ECUDA, se);
+    // every call already enqueued on the device, on any stream, first
+    cudaError_t e = cudaDeviceSynchronize();
+    for (int q = 0; q < args->world && e == cudaSuccess; ++q)
+        e = cudaMemcpy(status + q, static_cast<const char*>(base) + (int64_t)q * pitch +
+                                       LSE_MERGE_CP_STATUS_OFFSET,
+                       sizeof(uint32_t), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail_cuda(LSE_MERGE_ECUDA, (int)e);
+    return LSE_MERGE_OK;
 }

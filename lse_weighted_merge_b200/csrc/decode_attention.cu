@@ -21,11 +21,23 @@
 // LSE merge again, over the warps), giving the split's (o_r, lse_r).
 //
 //  * lse_merge_decode_partials writes (o_r, lse_r) to global memory.
+//  * lse_merge_decode_attention_ws merges them in the same kernel without a
+//    cluster: every split CTA writes its partial into the caller's
+//    workspace, makes it visible device-wide and adds 1 to the (b, KV head)
+//    counter there; the CTA that brings the counter to R merges the R
+//    partials (read back through L2, where they still are), writes the
+//    output and sets the counter back to 0 for the next call.  No CTA waits
+//    for another; the partials never need to reach HBM before the merge.
 //  * lse_merge_decode_attention launches the R splits of one (b, KV head) as
-//    a cluster: after a cluster barrier CTA r merges columns
-//    [r*D/R, (r+1)*D/R) of every head from all R partials, read from the
-//    other CTAs' shared memory (distributed shared memory), and a second
-//    barrier keeps every CTA alive until the others have read it.
+//    a cluster.  CTA r > 0 stores its split's partial into slot r of a
+//    receive buffer in CTA 0's shared memory (distributed shared memory),
+//    each thread then arrives, with release semantics at cluster scope, on
+//    an mbarrier in CTA 0, and the CTA exits at once.  CTA 0 writes its own
+//    partial into slot 0, waits on the mbarrier (bounded by the global
+//    timer) and merges the R slots.  Only CTA 0 waits for the slowest split;
+//    the others free their SM as soon as their keys are done.  The receive
+//    buffer lies outside the K/V ring, which CTA 0 may still be using when a
+//    sibling's partial arrives.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -46,6 +58,10 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// Longest wait of CTA 0 for its siblings' partials (the siblings run at the
+// same time as CTA 0, over as many keys, so the wait normally ends within a
+// few microseconds).
+constexpr uint64_t kFusedWaitNs = 2000000000ull;
 
 struct AParams {
     const char* q;
@@ -59,6 +75,10 @@ struct AParams {
     float* pl;             // [B, Hq, R]
     char* out;             // merged output [B, Hq, D] (fused)
     float* out_lse;        // [B, Hq]
+    unsigned* ws_cnt;      // workspace: arrived splits per (b, KV head) [B, Hkv]
+    float* ws_l;           // workspace: split lse [B, Hkv, R, G]
+    float* ws_o;           // workspace: split o [B, Hkv, R, G, D]
+    int Hkv;
 };
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -77,6 +97,48 @@ __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_grou
 template <int N>
 __device__ __forceinline__ void cp_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ---- cluster barrier and mbarrier (the fused merge's hand-off to CTA 0)
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Arrive on the mbarrier at shared address `bar` of cluster CTA `rank`, after
+// (release, cluster scope) this thread's earlier stores.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, uint32_t rank) {
+    uint32_t rbar;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(bar), "r"(rank));
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar) : "memory");
+}
+// One bounded probe of phase `parity` of the local mbarrier (acquire, cluster scope).
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\n"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// Add v to *p (gpu scope, acquire and release); returns the old value.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -144,7 +206,12 @@ __device__ __forceinline__ uint32_t tile_off(int row, int ch) {
     return (uint32_t)(row * (D * 2) + ((ch ^ (row & 7)) * 16));
 }
 
-template <typename T, int D, bool FUSED, typename TOut>
+// What the kernel does with a split's partial (kAttnMode* of plan.h).
+constexpr int kModePartials = kAttnModePartials;
+constexpr int kModeCluster = kAttnModeCluster;
+constexpr int kModeWorkspace = kAttnModeWorkspace;
+
+template <typename T, int D, int MODE, typename TOut>
 __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const AParams p) {
     constexpr int TK = kAttnTileKeys;
     constexpr int S = kAttnStages;
@@ -157,14 +224,33 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
     static_assert(TK == 16 || TK == 32, "key tile of 16 or 32");
     extern __shared__ __align__(128) unsigned char smem[];
 
-    pdl_wait();
-    pdl_release();
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int r = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     const int G = p.G, R = p.R;
     const int h0 = hk * G;
+
+    // Fused: CTA 0's receive buffer behind the ring and the warp states: the
+    // mbarrier (16 bytes), lse [R][G], then o [R][G][D] (fp32).  r is the
+    // CTA's rank in its cluster (the cluster spans the R splits along x).
+    constexpr int64_t kRing = (int64_t)kAttnWarps * S * 2 * TILE;
+    constexpr int64_t kStates = (int64_t)kAttnWarps * 16 * (D + 2) * 4;
+    constexpr int64_t kRecvOff = ((kRing > kStates ? kRing : kStates) + 15) / 16 * 16;
+    const uint32_t bar = smem_u32(smem + kRecvOff);
+    float* const recv_l = reinterpret_cast<float*>(smem + kRecvOff + 16);
+    float* const recv_o = recv_l + ((R * G + 3) & ~3);
+    if constexpr (MODE == kModeCluster) {
+        if (R > 1) {
+            if (r == 0 && threadIdx.x == 0) mbar_init(bar, (uint32_t)((R - 1) * blockDim.x));
+            // the barrier's init is visible to every CTA before any arrives on
+            // it: each thread waits on this cluster barrier before its first
+            // store into CTA 0
+            cluster_arrive_release();
+        }
+    }
+
+    pdl_wait();
+    pdl_release();
 
     int len = p.L;
     if (p.kv_len) len = min(max(__ldg(p.kv_len + b), 0), p.L);
@@ -324,8 +410,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
     float* st_m = reinterpret_cast<float*>(smem);
     float* st_l = st_m + kAttnWarps * 16;
     float* st_o = st_l + kAttnWarps * 16;
-    float* sp_o = st_o + kAttnWarps * 16 * D;   // the split's partial o [16][D]
-    float* sp_l = sp_o + 16 * D;                // and its lse [16] (natural log)
     if (t == 0) {
         st_m[warp * 16 + g] = m0;
         st_m[warp * 16 + g + 8] = m1;
@@ -343,6 +427,25 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
     }
     __syncthreads();
     const int64_t rows_b = (int64_t)b * p.Hq + h0;
+    // Cluster: this split's partial goes to slot r of CTA 0's receive buffer.
+    // Workspace: to slot r of this (b, KV head)'s block of the workspace.
+    const int64_t bh = (int64_t)b * p.Hkv + hk;
+    float* dst_o = recv_o;
+    float* dst_l = recv_l;
+    if constexpr (MODE == kModeWorkspace) {
+        dst_o = p.ws_o + bh * R * G * D;
+        dst_l = p.ws_l + bh * R * G;
+    }
+    if constexpr (MODE == kModeCluster) {
+        if (R > 1) {
+            cluster_wait_acquire();   // CTA 0's mbarrier is initialised
+            if (r != 0) {
+                cg::cluster_group cluster = cg::this_cluster();
+                dst_o = cluster.map_shared_rank(recv_o, 0);
+                dst_l = cluster.map_shared_rank(recv_l, 0);
+            }
+        }
+    }
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int gg = idx / D, d = idx - gg * D;
         float M = -INFINITY;
@@ -362,9 +465,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
         }
         const float o = den > 0.f ? num / den : 0.f;
         const float lse = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
-        if constexpr (FUSED) {
-            sp_o[gg * D + d] = o;
-            if (d == 0) sp_l[gg] = lse;
+        if constexpr (MODE != kModePartials) {
+            dst_o[(r * G + gg) * D + d] = o;
+            if (d == 0) dst_l[r * G + gg] = lse;
         } else {
             const int64_t row = rows_b + gg;
             p.po[(row * R + r) * D + d] = o;
@@ -372,74 +475,116 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
         }
     }
 
-    if constexpr (FUSED) {
-        // ---- merge the R splits of this (b, KV head) across the cluster
-        cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();   // every CTA's partial is in its shared memory
-        const int rank = (int)cluster.block_rank();
-        const int cols = D / R;
-        for (int idx = threadIdx.x; idx < G * cols; idx += blockDim.x) {
-            const int gg = idx / cols, d = rank * cols + (idx - gg * cols);
-            // all R remote loads of a kind are issued before any is used
-            float lj[8], oj[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                lj[j] = -INFINITY;
-                oj[j] = 0.f;
-                if (j < R) {
-                    lj[j] = *cluster.map_shared_rank(sp_l + gg, j);
-                    oj[j] = *cluster.map_shared_rank(sp_o + gg * D + d, j);
-                }
-            }
+    if constexpr (MODE == kModeWorkspace) {
+        // ---- count this split in; the last of the R splits merges them all.
+        // The CTA barrier orders every thread's partial stores before thread
+        // 0's count, whose release (gpu scope, cumulative) publishes them;
+        // the count's acquire makes the splits counted before visible to the
+        // last CTA, whose threads read them after the second barrier.
+        __shared__ int s_last;
+        __syncthreads();
+        if (threadIdx.x == 0) s_last = atom_add_acq_rel_gpu(p.ws_cnt + bh, 1u) == (unsigned)(R - 1);
+        __syncthreads();
+        if (!s_last) return;
+        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+            const int gg = idx / D, d = idx - gg * D;
             float M = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) M = fmaxf(M, lj[j]);
+            for (int j = 0; j < R; ++j) M = fmaxf(M, __ldcg(dst_l + j * G + gg));
             float den = 0.f, num = 0.f;
             if (M != -INFINITY) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (lj[j] != -INFINITY) {   // an empty split's o is not used
-                        const float e = expf(lj[j] - M);
+                for (int j = 0; j < R; ++j) {
+                    const float lj = __ldcg(dst_l + j * G + gg);
+                    if (lj != -INFINITY) {   // an empty split's o is not used
+                        const float e = expf(lj - M);
                         den += e;
-                        num += e * oj[j];
+                        num += e * __ldcg(dst_o + ((int64_t)j * G + gg) * D + d);
                     }
                 }
             }
             const int64_t row = rows_b + gg;
             store_out<TOut>(p.out + (row * D + d) * (int64_t)sizeof(TOut), den > 0.f ? num / den : 0.f);
-            if (rank == 0 && idx - gg * cols == 0)
-                p.out_lse[row] = den > 0.f ? M + logf(den) : -INFINITY;
+            if (d == 0) p.out_lse[row] = den > 0.f ? M + logf(den) : -INFINITY;
         }
-        cluster.sync();   // keep this CTA's shared memory alive until all have read it
+        if (threadIdx.x == 0) p.ws_cnt[bh] = 0u;   // every split of this call has counted
+    }
+    if constexpr (MODE == kModeCluster) {
+        // ---- hand the partial to CTA 0, which merges the R splits
+        if (R > 1 && r != 0) {
+            mbar_arrive_remote(bar, 0);   // after this thread's stores into CTA 0
+            return;                       // nothing reads this CTA's shared memory
+        }
+        bool ok = true;
+        if (R > 1) {
+            // every sibling thread arrives once: phase 0 completes when all
+            // R - 1 partials are in recv; bounded wait (a sibling that never
+            // arrives would be a bug: the result is then NaN, not a hang)
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait(bar, 0)) {
+                if (global_ns() - t0 > kFusedWaitNs) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        ok = __syncthreads_and(ok) != 0;   // also orders CTA 0's own slot-0 stores
+        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+            const int gg = idx / D, d = idx - gg * D;
+            float M = -INFINITY;
+            for (int j = 0; j < R; ++j) M = fmaxf(M, recv_l[j * G + gg]);
+            float den = 0.f, num = 0.f;
+            if (M != -INFINITY) {
+                for (int j = 0; j < R; ++j) {
+                    const float lj = recv_l[j * G + gg];
+                    if (lj != -INFINITY) {   // an empty split's o is not used
+                        const float e = expf(lj - M);
+                        den += e;
+                        num += e * recv_o[(j * G + gg) * D + d];
+                    }
+                }
+            }
+            const int64_t row = rows_b + gg;
+            float o = den > 0.f ? num / den : 0.f;
+            float lse = den > 0.f ? M + logf(den) : -INFINITY;
+            if (!ok) o = lse = __int_as_float(0x7fc00000);   // NaN: the hand-off never completed
+            store_out<TOut>(p.out + (row * D + d) * (int64_t)sizeof(TOut), o);
+            if (d == 0) p.out_lse[row] = lse;
+        }
     }
 }
 
 using AttnFn = void (*)(AParams);
 
-template <typename T, int D>
-AttnFn pick_d(bool fused, int out_dtype) {
-    if (!fused) return decode_attn_kernel<T, D, false, float>;
+template <typename T, int D, int MODE>
+AttnFn pick_o(int out_dtype) {
     switch (out_dtype) {
-        case LSE_MERGE_F32: return decode_attn_kernel<T, D, true, float>;
-        case LSE_MERGE_F16: return decode_attn_kernel<T, D, true, __half>;
-        default: return decode_attn_kernel<T, D, true, __nv_bfloat16>;
+        case LSE_MERGE_F32: return decode_attn_kernel<T, D, MODE, float>;
+        case LSE_MERGE_F16: return decode_attn_kernel<T, D, MODE, __half>;
+        default: return decode_attn_kernel<T, D, MODE, __nv_bfloat16>;
     }
 }
-template <typename T>
-AttnFn pick_t(int D, bool fused, int out_dtype) {
-    return D == 64 ? pick_d<T, 64>(fused, out_dtype) : pick_d<T, 128>(fused, out_dtype);
+template <typename T, int D>
+AttnFn pick_d(int mode, int out_dtype) {
+    if (mode == kModePartials) return decode_attn_kernel<T, D, kModePartials, float>;
+    return mode == kModeCluster ? pick_o<T, D, kModeCluster>(out_dtype)
+                                : pick_o<T, D, kModeWorkspace>(out_dtype);
 }
-AttnFn pick(int dtype, int D, bool fused, int out_dtype) {
-    return dtype == LSE_MERGE_F16 ? pick_t<__half>(D, fused, out_dtype)
-                                  : pick_t<__nv_bfloat16>(D, fused, out_dtype);
+template <typename T>
+AttnFn pick_t(int D, int mode, int out_dtype) {
+    return D == 64 ? pick_d<T, 64>(mode, out_dtype) : pick_d<T, 128>(mode, out_dtype);
+}
+AttnFn pick(int dtype, int D, int mode, int out_dtype) {
+    return dtype == LSE_MERGE_F16 ? pick_t<__half>(D, mode, out_dtype)
+                                  : pick_t<__nv_bfloat16>(D, mode, out_dtype);
 }
 
-// cudaFuncSetAttribute once per (kernel, device) for dynamic shared memory
-// above 48 KB.
+// cudaFuncSetAttribute per (kernel, device) for dynamic shared memory above
+// 48 KB, raised whenever a launch needs more than the size set so far (the
+// fused kernel's receive buffer grows with R and the group size).
 std::mutex g_attr_mu;
 struct AttrDone {
     const void* fn;
     int dev;
+    int64_t bytes;
 };
 AttrDone g_attr_done[128];
 int g_attr_n = 0;
@@ -449,24 +594,33 @@ cudaError_t ensure_smem(AttnFn fn, int64_t bytes) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lk(g_attr_mu);
+    AttrDone* slot = nullptr;
     for (int i = 0; i < g_attr_n; ++i)
-        if (g_attr_done[i].fn == (const void*)fn && g_attr_done[i].dev == dev) return cudaSuccess;
+        if (g_attr_done[i].fn == (const void*)fn && g_attr_done[i].dev == dev) slot = &g_attr_done[i];
+    if (slot && slot->bytes >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess && g_attr_n < 128) g_attr_done[g_attr_n++] = AttrDone{(const void*)fn, dev};
-    return e;
+    if (e != cudaSuccess) return e;
+    if (slot)
+        slot->bytes = bytes;
+    else if (g_attr_n < 128)
+        g_attr_done[g_attr_n++] = AttrDone{(const void*)fn, dev, bytes};
+    return cudaSuccess;
 }
 
 
 int launch(const void* q, const void* k, const void* v, const int32_t* kv_len, int B, int Hq,
            int Hkv, int L, int D, int R, float scale, const lse_merge_attn_strides* strides,
-           int dtype, int out_dtype, void* out_o, float* out_lse, bool fused, cudaStream_t stream) {
+           int dtype, int out_dtype, void* out_o, float* out_lse, int mode, void* ws,
+           int64_t ws_bytes, cudaStream_t stream) {
     if (Hq < 1 || Hkv < 1 || L < 1 || D < 1) return LSE_MERGE_EDIMS;
     const lse_merge_attn_strides st = strides ? *strides : default_attn_strides(Hq, Hkv, L, D);
+    const bool fused = mode != kModePartials;
     AttnPlan pl;
     const int rc = make_attn_plan(q, k, v, B, Hq, Hkv, L, D, R, scale, st, dtype,
-                                  fused ? out_dtype : LSE_MERGE_F32, out_o, out_lse, fused, &pl);
+                                  fused ? out_dtype : LSE_MERGE_F32, out_o, out_lse, mode, ws,
+                                  ws_bytes, &pl);
     if (rc != LSE_MERGE_OK) return rc;
-    AParams ap;
+    AParams ap{};
     ap.q = static_cast<const char*>(q);
     ap.k = static_cast<const char*>(k);
     ap.v = static_cast<const char*>(v);
@@ -480,6 +634,7 @@ int launch(const void* q, const void* k, const void* v, const int32_t* kv_len, i
     ap.v_h = st.v_h * 2;
     ap.v_l = st.v_l * 2;
     ap.Hq = Hq;
+    ap.Hkv = Hkv;
     ap.G = pl.G;
     ap.L = L;
     ap.R = R;
@@ -488,7 +643,13 @@ int launch(const void* q, const void* k, const void* v, const int32_t* kv_len, i
     ap.pl = fused ? nullptr : out_lse;
     ap.out = fused ? static_cast<char*>(out_o) : nullptr;
     ap.out_lse = fused ? out_lse : nullptr;
-    const AttnFn fn = pick(dtype, D, fused, out_dtype);
+    if (mode == kModeWorkspace) {
+        char* w = static_cast<char*>(ws);
+        ap.ws_cnt = reinterpret_cast<unsigned*>(w);
+        ap.ws_l = reinterpret_cast<float*>(w + pl.ws_l_off);
+        ap.ws_o = reinterpret_cast<float*>(w + pl.ws_o_off);
+    }
+    const AttnFn fn = pick(dtype, D, mode, out_dtype);
     cudaError_t e = ensure_smem(fn, pl.smem);
     if (e == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
@@ -503,7 +664,7 @@ int launch(const void* q, const void* k, const void* v, const int32_t* kv_len, i
             attr[na].val.programmaticStreamSerializationAllowed = 1;
             ++na;
         }
-        if (fused) {
+        if (mode == kModeCluster) {
             attr[na].id = cudaLaunchAttributeClusterDimension;
             attr[na].val.clusterDim.x = (unsigned)R;
             attr[na].val.clusterDim.y = 1;
@@ -533,8 +694,8 @@ int lse_merge_decode_partials(const void* q, const void* k, const void* v, const
                               const lse_merge_attn_strides* strides, int dtype,
                               float* partial_o, float* partial_lse, lse_merge_stream_t stream) {
     return lsem::attn::launch(q, k, v, kv_len, B, Hq, Hkv, L, D, R, scale, strides, dtype,
-                              LSE_MERGE_F32, partial_o, partial_lse, false,
-                              reinterpret_cast<cudaStream_t>(stream));
+                              LSE_MERGE_F32, partial_o, partial_lse, lsem::kAttnModePartials,
+                              nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int lse_merge_decode_attention(const void* q, const void* k, const void* v, const int32_t* kv_len,
@@ -542,8 +703,19 @@ int lse_merge_decode_attention(const void* q, const void* k, const void* v, cons
                                const lse_merge_attn_strides* strides, int dtype, int out_dtype,
                                void* out_o, float* out_lse, lse_merge_stream_t stream) {
     return lsem::attn::launch(q, k, v, kv_len, B, Hq, Hkv, L, D, R, scale, strides, dtype,
-                              out_dtype, out_o, out_lse, true,
+                              out_dtype, out_o, out_lse, lsem::kAttnModeCluster, nullptr, 0,
                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+int lse_merge_decode_attention_ws(const void* q, const void* k, const void* v,
+                                  const int32_t* kv_len, int B, int Hq, int Hkv, int L, int D,
+                                  int R, float scale, const lse_merge_attn_strides* strides,
+                                  int dtype, int out_dtype, void* workspace,
+                                  int64_t workspace_bytes, void* out_o, float* out_lse,
+                                  lse_merge_stream_t stream) {
+    return lsem::attn::launch(q, k, v, kv_len, B, Hq, Hkv, L, D, R, scale, strides, dtype,
+                              out_dtype, out_o, out_lse, lsem::kAttnModeWorkspace, workspace,
+                              workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -221,12 +221,27 @@ lse_merge_attn_strides default_attn_strides(int Hq, int Hkv, int L, int D) {
     return s;
 }
 
-// out_o / out_lse: the merged outputs (fused) or the partial buffers
+int attn_workspace_layout(int B, int Hq, int Hkv, int R, int D, AttnPlan* plan) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || R < 1 || D < 1 || Hq % Hkv != 0) return LSE_MERGE_EDIMS;
+    const auto up = [](i128 x) { return (x + 255) / 256 * 256; };
+    const i128 rows = (i128)B * Hq * R;   // = B * Hkv * R * G
+    const i128 l_off = up((i128)B * Hkv * 4);
+    const i128 o_off = up(l_off + rows * 4);
+    const i128 total = o_off + rows * D * 4;
+    if (total > ((i128)1 << 62)) return LSE_MERGE_EDIMS;
+    plan->ws_l_off = (int64_t)l_off;
+    plan->ws_o_off = (int64_t)o_off;
+    plan->ws_bytes = (int64_t)total;
+    return LSE_MERGE_OK;
+}
+
+// out_o / out_lse: the merged outputs (fused modes) or the partial buffers
 // (dense [B,Hq,R,D] and [B,Hq,R] fp32) of the unfused producer.
 int make_attn_plan(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int L,
                    int D, int R, float scale, const lse_merge_attn_strides& st, int dtype,
-                   int out_dtype, const void* out_o, const float* out_lse, int fused,
-                   AttnPlan* plan) {
+                   int out_dtype, const void* out_o, const float* out_lse, int mode,
+                   const void* ws, int64_t ws_bytes, AttnPlan* plan) {
+    const int fused = mode != kAttnModePartials;
     const int ob = elem_bytes(out_dtype);
     if (elem_bytes(dtype) == 0 || ob == 0) return LSE_MERGE_EDTYPE;
     if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || D < 1 || R < 1) return LSE_MERGE_EDIMS;
@@ -237,7 +252,8 @@ int make_attn_plan(const void* q, const void* k, const void* v, int B, int Hq, i
     if (dtype == LSE_MERGE_F32) return LSE_MERGE_EUNSUP;
     if (D != 64 && D != 128) return LSE_MERGE_EUNSUP;
     if (Hq % Hkv != 0 || Hq / Hkv > 16) return LSE_MERGE_EUNSUP;
-    if (fused && R != 1 && R != 2 && R != 4 && R != 8) return LSE_MERGE_EUNSUP;
+    if (mode == kAttnModeCluster && R != 1 && R != 2 && R != 4 && R != 8) return LSE_MERGE_EUNSUP;
+    if (mode == kAttnModeWorkspace && !ws) return LSE_MERGE_ENULL;
     if (B > 65535 || Hkv > 65535 || R > 65535) return LSE_MERGE_EDIMS;
     if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return LSE_MERGE_EDIMS;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out_o, ob) ||
@@ -265,14 +281,28 @@ int make_attn_plan(const void* q, const void* k, const void* v, int B, int Hq, i
         return LSE_MERGE_EALIAS;
     AttnPlan p{};
     p.G = Hq / Hkv;
-    p.fused = fused;
+    p.mode = mode;
+    if (mode == kAttnModeWorkspace) {
+        const int lrc = attn_workspace_layout(B, Hq, Hkv, R, D, &p);
+        if (lrc != LSE_MERGE_OK) return lrc;
+        if (!aligned(ws, 16)) return LSE_MERGE_EALIGN;
+        if (ws_bytes < p.ws_bytes) return LSE_MERGE_EDIMS;
+        const Span sw{(uintptr_t)ws, (i128)(uintptr_t)ws + p.ws_bytes};
+        if (overlap(sw, sq) || overlap(sw, sk) || overlap(sw, sv) || overlap(sw, so) ||
+            overlap(sw, sl))
+            return LSE_MERGE_EALIAS;
+    }
     const int64_t ring = (int64_t)kAttnWarps * kAttnStages * 2 * kAttnTileKeys * D * 2;
-    // after the key loop the ring is reused: each warp's state (16 rows of m, l
-    // and D accumulators) and, behind it, the split's merged partial
+    // after the key loop the ring is reused for each warp's state (16 rows of
+    // m, l and D accumulators)
     const int64_t states = (int64_t)kAttnWarps * 16 * (D + 2) * 4;
-    const int64_t split = (int64_t)16 * (D + 1) * 4;
-    const int64_t need = states + split;
-    p.smem = ring > need ? ring : need;
+    const int64_t base = ((ring > states ? ring : states) + 15) / 16 * 16;
+    // fused: behind them CTA 0's receive buffer of the R split partials (an
+    // mbarrier, lse [R][G] padded to 4 floats, o [R][G][D]), which siblings
+    // fill while CTA 0 may still use its ring
+    const int64_t rg = (int64_t)R * p.G;
+    p.smem = mode == kAttnModeCluster ? base + 16 + ((rg + 3) & ~(int64_t)3) * 4 + rg * D * 4 : base;
+    if (p.smem > kAttnMaxSmem) return LSE_MERGE_EUNSUP;
     *plan = p;
     return LSE_MERGE_OK;
 }
@@ -355,7 +385,8 @@ int make_cp_plan(const lse_merge_cp_args& a, CpPlan* plan) {
     if (a.rank_begin < 0 || a.rank_count < 1 || a.rank_begin + a.rank_count > a.world)
         return LSE_MERGE_EDIMS;
     if (a.timeout_ns <= 0 || a.timeout_ns > kCpMaxTimeoutNs) return LSE_MERGE_EDIMS;
-    if (a.flags & ~LSE_MERGE_CP_FLAG_CROSS_GPU_PROTOCOL) return LSE_MERGE_EDIMS;
+    if (a.flags & ~(LSE_MERGE_CP_FLAG_CROSS_GPU_PROTOCOL | LSE_MERGE_CP_FLAG_TEST_SILENT_LAST_RANK))
+        return LSE_MERGE_EDIMS;
     p.rank_begin = a.rank_begin;
     p.rank_count = a.rank_count;
     p.out_bytes = ob;
@@ -408,6 +439,14 @@ int lse_merge_cp_validate(const lse_merge_cp_args* args) {
     return lsem::make_cp_plan(*args, &p);
 }
 
+int lse_merge_decode_workspace_bytes(int B, int Hq, int Hkv, int R, int D, int64_t* bytes) {
+    if (!bytes) return LSE_MERGE_ENULL;
+    lsem::AttnPlan p{};
+    const int rc = lsem::attn_workspace_layout(B, Hq, Hkv, R, D, &p);
+    if (rc == LSE_MERGE_OK) *bytes = p.ws_bytes;
+    return rc;
+}
+
 int lse_merge_plan_query(const void* partial_o, const float* partial_lse, int R, int B, int H,
                          int D, const lse_merge_strides* strides, int in_dtype, int out_dtype,
                          const void* out_o, const float* out_lse, int path,
@@ -431,7 +470,8 @@ const char* lse_merge_strerror(int code) {
         case LSE_MERGE_EPATH: return "the requested kernel path cannot take these arguments";
         case LSE_MERGE_EUNSUP: return "shape not implemented by the decode-attention kernels (dtype, D, group, R)";
         case LSE_MERGE_ECUDA: return "a CUDA runtime call of a set-up function failed";
-        case LSE_MERGE_ESCRATCH: return "the problem needs more scratch memory than the static array holds (16 MiB)";
+        case LSE_MERGE_ESCRATCH: return "the problem needs more scratch or staging memory than the library's array or the host context holds";
+        case LSE_MERGE_EDEVICE: return "the current device is not the one the host context was made on";
         default: return "unknown lse_merge error code";
     }
 }

@@ -21,6 +21,14 @@ constexpr int kBlock = LSEM_BLOCK;
 #define LSEM_MINB 1
 #endif
 constexpr int kMinBlocks = LSEM_MINB;
+#ifndef LSEM_MINB_VEC1
+#define LSEM_MINB_VEC1 LSEM_MINB
+#endif
+#ifndef LSEM_MINB_STREAM
+#define LSEM_MINB_STREAM LSEM_MINB
+#endif
+constexpr int kMinBlocksVec1 = LSEM_MINB_VEC1;
+constexpr int kMinBlocksStream = LSEM_MINB_STREAM;
 // Launch with programmatic stream serialization (the next kernel in the
 // stream may be scheduled while this one drains; it waits before touching
 // memory).  Hides the launch gap between back-to-back merges.
@@ -28,6 +36,15 @@ constexpr int kMinBlocks = LSEM_MINB;
 #define LSEM_PDL 1
 #endif
 constexpr int kPdl = LSEM_PDL;
+// Before pdl_wait(), prefetch into L2 the lines of the loads a thread issues
+// first, so that a grid launched behind another one starts its first DRAM
+// round while the previous grid drains instead of after it has finished.
+// 0: off; n > 0: the persistent kernel prefetches its first n row slices,
+// the one-shot kernels their first batch of partial rows.
+#ifndef LSEM_PREFETCH
+#define LSEM_PREFETCH 1
+#endif
+constexpr int kPrefetch = LSEM_PREFETCH;
 // AUTO picks the persistent STREAM kernel for partials between
 // kStreamMinBytes and kStreamMaxBytes and the one-shot VECTOR kernel outside
 // that range.  Measured on B200: STREAM is 3-7 % faster from ~30 MB to
@@ -89,11 +106,19 @@ struct StatePlan {
     int64_t grid;
 };
 
+// Decode attention: what the kernel does with each split's partial.
+constexpr int kAttnModePartials = 0;    // writes it to the caller's partial buffers
+constexpr int kAttnModeCluster = 1;     // hands it to CTA 0 of the cluster, which merges
+constexpr int kAttnModeWorkspace = 2;   // workspace + counter: the last split merges
+
 // Decode attention: validated geometry.
 struct AttnPlan {
     int G;            // query heads per KV head
-    int fused;        // 1: cluster merge inside the kernel
+    int mode;         // kAttnMode*
     int64_t smem;     // dynamic shared memory per CTA
+    // workspace (kAttnModeWorkspace): counters [B, Hkv] u32 at 0, split lse
+    // [B, Hkv, R, G] f32 at ws_l_off, split o [B, Hkv, R, G, D] f32 at ws_o_off
+    int64_t ws_l_off, ws_o_off, ws_bytes;
 };
 constexpr int kAttnWarps = 4;     // warps per CTA, each a private K/V ring
 #ifndef LSEM_ATTN_TK
@@ -103,12 +128,15 @@ constexpr int kAttnWarps = 4;     // warps per CTA, each a private K/V ring
 #define LSEM_ATTN_STAGES 3
 #endif
 constexpr int kAttnTileKeys = LSEM_ATTN_TK;    // keys per K/V tile (16 or 32)
+constexpr int64_t kAttnMaxSmem = 227 * 1024;   // dynamic shared memory one CTA may take
 constexpr int kAttnStages = LSEM_ATTN_STAGES;  // tiles per warp ring
 
 int make_attn_plan(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int L,
                    int D, int R, float scale, const lse_merge_attn_strides& st, int dtype,
-                   int out_dtype, const void* out_o, const float* out_lse, int fused,
-                   AttnPlan* plan);
+                   int out_dtype, const void* out_o, const float* out_lse, int mode,
+                   const void* ws, int64_t ws_bytes, AttnPlan* plan);
+// Workspace layout of kAttnModeWorkspace for these sizes (no pointer checks).
+int attn_workspace_layout(int B, int Hq, int Hkv, int R, int D, AttnPlan* plan);
 lse_merge_attn_strides default_attn_strides(int Hq, int Hkv, int L, int D);
 
 // Validate the arguments of lse_merge_state_update and fill *plan.

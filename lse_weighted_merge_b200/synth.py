@@ -87,6 +87,9 @@ CP_WORKLOADS = {
         Workload("cp_w8_b64_h32_d128_masked", 8, 64, 32, 128, "bf16", "bf16", "rbhd", 1.0,
                  "normal", (6.0, 3.0), 1102, empty_shard_p=0.10, empty_row_p=0.01,
                  note="CP decode, 8 ranks, batch 64, 10% empty shards, 1% empty rows"),
+        Workload("cp_w8_b256_h64_d128", 8, 256, 64, 128, "bf16", "bf16", "rbhd", 1.0,
+                 "normal", (6.0, 3.0), 1103,
+                 note="CP decode, 8 ranks, batch 256: a bandwidth-bound exchange"),
     ]
 }
 

@@ -209,10 +209,14 @@ def test_state_update_validation(kw, code):
     assert sq(**kw) == code, (kw, nat.strerror(code))
 
 
+WS = 0x7f5000000000
+
+
 def dq(B=2, Hq=8, Hkv=2, L=100, D=128, R=4, scale=0.1, st=None, dt=nat.BF16, q=PO, k=PL,
-       v=0x7f4000000000, out=OUT, outl=OUTL, fused=True, odt=nat.BF16):
+       v=0x7f4000000000, out=OUT, outl=OUTL, fused=True, odt=nat.BF16, ws=0, wsb=1 << 30):
     return nat.decode_raw(q, k, v, 0, B, Hq, Hkv, L, D, R, scale, st, dt, out, outl,
-                          fused=fused, out_dtype=odt, check=False)
+                          fused=fused, out_dtype=odt, check=False, workspace=ws,
+                          workspace_bytes=wsb)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -234,8 +238,26 @@ def test_decode_attention_validation(kw, code):
 
 def test_decode_valid_arguments_pass_validation():
     # valid arguments get past validation (here, without a GPU, the launch itself fails)
-    for kw in (dict(), dict(R=3, fused=False), dict(R=64, fused=False), dict(D=64, Hq=16, Hkv=1)):
+    for kw in (dict(), dict(R=3, fused=False), dict(R=64, fused=False), dict(D=64, Hq=16, Hkv=1),
+               dict(ws=WS), dict(ws=WS, R=3), dict(ws=WS, R=64), dict(ws=WS, R=1000, L=50)):
         assert dq(**kw) in (nat.OK, nat.ELAUNCH), kw
+
+
+def test_decode_workspace_layout_and_validation():
+    # counters [B, Hkv] u32, then lse [B, Hq, R] and o [B, Hq, R, D] fp32, each part 256-aligned
+    B, Hq, Hkv, R, D = 2, 8, 2, 4, 128
+    need = nat.decode_workspace_bytes(B, Hq, Hkv, R, D)
+    assert need == 256 + 256 + B * Hq * R * D * 4
+    assert nat.decode_workspace_bytes(3, 4, 4, 5, 64) == 256 + 256 + 3 * 4 * 5 * 64 * 4
+    assert dq(ws=WS, wsb=need) in (nat.OK, nat.ELAUNCH)
+    assert dq(ws=WS, wsb=need - 1) == nat.EDIMS            # too short
+    assert dq(ws=WS + 8, wsb=need) == nat.EALIGN           # not 16-byte aligned
+    assert dq(ws=OUT - 64, wsb=need) == nat.EALIAS         # overlaps the output
+    assert dq(ws=PL + 128, wsb=need) == nat.EALIAS         # overlaps k
+    for bad in (dict(B=0), dict(Hq=6, Hkv=4), dict(R=0)):
+        args = {**dict(B=B, Hq=Hq, Hkv=Hkv, R=R, D=D), **bad}
+        with pytest.raises(nat.LseMergeError):
+            nat.decode_workspace_bytes(args["B"], args["Hq"], args["Hkv"], args["R"], args["D"])
 
 
 def test_fast_forwarding_extension_is_built_and_checks_its_arguments():
@@ -260,3 +282,21 @@ def test_fast_forwarding_extension_is_built_and_checks_its_arguments():
     for s in (st, ((64, 256, 128), (1, 4, 2)), nat.Strides(*st)):
         assert nat.merge_raw(PO, PL, 2, 1, 0, 64, s, nat.BF16, nat.BF16, OUT, OUTL, 0,
                              check=False) == nat.EDIMS
+
+
+def test_host_pipeline_stage_bytes_and_null_context():
+    # staging of one call: partials, lse, outputs, merged lse, each 256-aligned
+    R, B, H, D = 16, 512, 16, 512
+    up = lambda x: -(-x // 256) * 256
+    want = up(R * B * H * D * 2) + up(R * B * H * 4) + up(B * H * D * 4) + up(B * H * 4)
+    assert nat.host_stage_bytes(R, B, H, D, nat.BF16, nat.F32) == want
+    assert nat.host_stage_bytes(3, 5, 7, 9, nat.F32, nat.F16) == \
+        up(3 * 5 * 7 * 9 * 4) + up(3 * 5 * 7 * 4) + up(5 * 7 * 9 * 2) + up(5 * 7 * 4)
+    with pytest.raises(nat.LseMergeError):
+        nat.host_stage_bytes(0, B, H, D, nat.BF16, nat.F32)
+    with pytest.raises(nat.LseMergeError):
+        nat.host_stage_bytes(R, B, H, D, 9, nat.F32)
+    # no context: refused before any CUDA call
+    assert nat.host_merge_raw(0, PO, PL, R, B, H, D, nat.LAYOUT_BHRD, nat.BF16, nat.F32, OUT, OUTL,
+                              8, check=False) == nat.ENULL
+    assert nat.strerror(nat.EDEVICE) != nat.strerror(999)

@@ -71,6 +71,7 @@ def test_validate_accepts_good_arguments():
     assert nat.cp_validate(make(world=4, rank_begin=3, rank_count=1, H=8)) == nat.OK
     assert nat.cp_validate(make(i=nat.F32, o=nat.F16, D=4)) == nat.OK
     assert nat.cp_validate(make(flags=nat.CP_FLAG_CROSS_GPU_PROTOCOL)) == nat.OK
+    assert nat.cp_validate(make(flags=nat.CP_FLAG_TEST_SILENT_LAST_RANK)) == nat.OK
     # inputs are only read: two played ranks may share one input buffer
     assert nat.cp_validate(make(lo=[LO, LO], ll=[LL, LL])) == nat.OK
 
@@ -82,7 +83,7 @@ def test_validate_accepts_good_arguments():
     (dict(rank_begin=1, rank_count=2), nat.EDIMS), (dict(rank_begin=-1, rank_count=1), nat.EDIMS),
     (dict(rank_count=0), nat.EDIMS),
     (dict(timeout_ns=0), nat.EDIMS), (dict(timeout_ns=61 * 10**9), nat.EDIMS),
-    (dict(flags=2), nat.EDIMS),
+    (dict(flags=4), nat.EDIMS),
     (dict(D=4), nat.EALIGN), (dict(i=nat.F32, D=2), nat.EALIGN),
     (dict(ws=[WS, 0]), nat.ENULL), (dict(lo=[LO, 0]), nat.ENULL), (dict(ol=[0, OL]), nat.ENULL),
     (dict(ws=[WS, WS + STEP + 128]), nat.EALIGN), (dict(lo=[LO + 8, LO + STEP]), nat.EALIGN),

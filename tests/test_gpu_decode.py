@@ -1,5 +1,6 @@
 """Split-KV decode attention (the producer of the partials) on the GPU vs the
-fp64 oracle attention: the fused cluster kernel, the unfused partials, their
+fp64 oracle attention: the fused kernel in both forms (the workspace form,
+whose last split merges, and the cluster form), the unfused partials, their
 merge, ragged and empty sequences, grouped heads, strided caches, dtypes.
 
 Tolerance of the attention outputs (derived from the arithmetic, not from a
@@ -81,7 +82,19 @@ def check_rows(got, got_lse, want, want_lse, vmax, in_dt, out_dt, what):
     return worst
 
 
-def run(q, k, v, R, scale, kv_len=None, fused=True, out_dt="bf16"):
+def workspace(B, Hq, Hkv, R, D):
+    """A zeroed workspace of the fused workspace form."""
+    return torch.zeros(nat.decode_workspace_bytes(B, Hq, Hkv, R, D), dtype=torch.uint8, device="cuda")
+
+
+def counters_are_zero(ws, B, Hkv):
+    return bool((ws[:B * Hkv * 4].view(torch.int32) == 0).all())
+
+
+def run(q, k, v, R, scale, kv_len=None, fused=True, out_dt="bf16", mode="ws", ws=None):
+    """One call of the C ABI: fused (mode "ws": lse_merge_decode_attention_ws,
+    with `ws` or a fresh zeroed workspace; mode "cluster":
+    lse_merge_decode_attention) or the partials (fused=False)."""
     B, Hq, D = q.shape
     _, Hkv, L, _ = k.shape
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -93,11 +106,17 @@ def run(q, k, v, R, scale, kv_len=None, fused=True, out_dt="bf16"):
     if fused:
         out = torch.empty((B, Hq, D), dtype=TDT[out_dt], device="cuda")
         lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+        wkw = {}
+        if mode == "ws":
+            ws = workspace(B, Hq, Hkv, R, D) if ws is None else ws
+            wkw = dict(workspace=ws.data_ptr(), workspace_bytes=ws.numel())
         nat.decode_raw(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(),
                        klen.data_ptr() if klen is not None else 0, B, Hq, Hkv, L, D, R, scale,
                        st, dt, out.data_ptr(), lse.data_ptr(), s, fused=True,
-                       out_dtype={"bf16": nat.BF16, "f16": nat.F16, "f32": nat.F32}[out_dt])
+                       out_dtype={"bf16": nat.BF16, "f16": nat.F16, "f32": nat.F32}[out_dt], **wkw)
         torch.cuda.synchronize()
+        if mode == "ws":   # the call leaves its counters at 0, ready for the next one
+            assert counters_are_zero(ws, B, Hkv)
         return out.cpu(), lse.cpu()
     po = torch.empty((B, Hq, R, D), dtype=torch.float32, device="cuda")
     pl = torch.empty((B, Hq, R), dtype=torch.float32, device="cuda")
@@ -118,13 +137,42 @@ SHAPES = [  # B, Hq, Hkv, L, D, R
 ]
 
 
+@pytest.mark.parametrize("mode", ["ws", "cluster"])
 @pytest.mark.parametrize("B,Hq,Hkv,L,D,R", SHAPES)
-def test_fused_attention_matches_oracle(B, Hq, Hkv, L, D, R):
+def test_fused_attention_matches_oracle(B, Hq, Hkv, L, D, R, mode):
     q, k, v = make(B, Hq, Hkv, L, D, seed=L + R)
     scale = 1 / math.sqrt(D)
-    out, lse = run(q, k, v, R, scale)
+    out, lse = run(q, k, v, R, scale, mode=mode)
     want, want_lse, vmax = reference(q, k, v, scale, [L] * B)
-    check_rows(out, lse, want, want_lse, vmax, "bf16", "bf16", "fused")
+    check_rows(out, lse, want, want_lse, vmax, "bf16", "bf16", f"fused {mode}")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,D,R", [
+    (2, 8, 2, 300, 128, 3),     # a split count the cluster form does not take
+    (1, 4, 1, 2000, 64, 16),
+    (1, 8, 8, 4096, 128, 64),   # many splits of one sequence
+    (2, 4, 2, 10, 128, 32),     # more splits than keys: most splits empty
+])
+def test_workspace_form_takes_any_split_count(B, Hq, Hkv, L, D, R):
+    q, k, v = make(B, Hq, Hkv, L, D, seed=3 * L + R)
+    scale = 1 / math.sqrt(D)
+    out, lse = run(q, k, v, R, scale, mode="ws")
+    want, want_lse, vmax = reference(q, k, v, scale, [L] * B)
+    check_rows(out, lse, want, want_lse, vmax, "bf16", "bf16", f"ws R={R}")
+
+
+def test_workspace_reused_by_consecutive_calls():
+    """Three calls in a row share one workspace (zeroed once): each call's
+    last split resets its counters, so the next call merges its own
+    partials and nothing of the previous call leaks in."""
+    B, Hq, Hkv, L, D, R = 3, 8, 2, 700, 128, 4
+    ws = workspace(B, Hq, Hkv, R, D)
+    scale = 1 / math.sqrt(D)
+    for call in range(3):
+        q, k, v = make(B, Hq, Hkv, L, D, seed=100 + call)
+        out, lse = run(q, k, v, R, scale, mode="ws", ws=ws)
+        want, want_lse, vmax = reference(q, k, v, scale, [L] * B)
+        check_rows(out, lse, want, want_lse, vmax, "bf16", "bf16", f"call {call}")
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,L,D,R", SHAPES)
@@ -146,11 +194,12 @@ def test_partials_merged_equal_fused():
     scale = 0.1
     po, pl = run(q, k, v, R, scale, fused=False)
     mo, ml = merge(po.cuda(), pl.cuda(), out_dtype=torch.float32)
-    fo, fl = run(q, k, v, R, scale, fused=True, out_dt="f32")
-    torch.cuda.synchronize()
-    # both merge the same fp32 partials; only the summation order differs
-    assert torch.allclose(mo.cpu(), fo, rtol=0, atol=1e-5)
-    assert torch.allclose(ml.cpu(), fl, rtol=0, atol=1e-5)
+    for mode in ("ws", "cluster"):
+        fo, fl = run(q, k, v, R, scale, fused=True, out_dt="f32", mode=mode)
+        torch.cuda.synchronize()
+        # all merge the same fp32 partials; only the summation order differs
+        assert torch.allclose(mo.cpu(), fo, rtol=0, atol=1e-5), mode
+        assert torch.allclose(ml.cpu(), fl, rtol=0, atol=1e-5), mode
 
 
 def test_ragged_and_empty_sequences():
@@ -159,9 +208,9 @@ def test_ragged_and_empty_sequences():
     q, k, v = make(B, Hq, Hkv, L, D, seed=11)
     scale = 1 / math.sqrt(D)
     want, want_lse, vmax = reference(q, k, v, scale, lens)
-    for fused in (True, False):
+    for fused in (True, "cluster", False):
         if fused:
-            out, lse = run(q, k, v, R, scale, kv_len=lens)
+            out, lse = run(q, k, v, R, scale, kv_len=lens, mode="cluster" if fused == "cluster" else "ws")
         else:
             from lse_weighted_merge_b200 import merge
             po, pl = run(q, k, v, R, scale, kv_len=lens, fused=False)
@@ -171,12 +220,13 @@ def test_ragged_and_empty_sequences():
         assert torch.all(out[1] == 0) and torch.all(lse[1] == -math.inf)
 
 
+@pytest.mark.parametrize("mode", ["ws", "cluster"])
 @pytest.mark.parametrize("out_dt", ["bf16", "f16", "f32"])
-def test_fp16_inputs_and_out_dtypes(out_dt):
+def test_fp16_inputs_and_out_dtypes(out_dt, mode):
     B, Hq, Hkv, L, D, R = 2, 8, 4, 257, 128, 2
     q, k, v = make(B, Hq, Hkv, L, D, dtype="f16", seed=13)
     scale = 1 / math.sqrt(D)
-    out, lse = run(q, k, v, R, scale, out_dt=out_dt)
+    out, lse = run(q, k, v, R, scale, out_dt=out_dt, mode=mode)
     want, want_lse, vmax = reference(q, k, v, scale, [L] * B)
     check_rows(out, lse, want, want_lse, vmax, "f16", out_dt, "f16")
 
@@ -201,25 +251,34 @@ def test_large_decode_sampled_rows():
     from lse_weighted_merge_b200 import decode_attention
     out, lse = decode_attention(q, k, v, splits=R, fused=True)
     out2, lse2 = decode_attention(q, k, v, splits=R, fused=False)
+    out3, lse3 = decode_attention(q, k, v, splits=R, fused="cluster")
     torch.cuda.synchronize()
     rng = np.random.Generator(np.random.PCG64(5))
     rows = [(int(b), int(h)) for b, h in zip(rng.integers(0, B, 24), rng.integers(0, Hq, 24))]
     want, want_lse, vmax = reference(q.cpu(), k.cpu(), v.cpu(), scale, [L] * B, rows=rows)
     check_rows(out.cpu(), lse.cpu(), want, want_lse, vmax, "bf16", "bf16", "large fused")
     check_rows(out2.cpu(), lse2.cpu(), want, want_lse, vmax, "bf16", "bf16", "large unfused")
+    check_rows(out3.cpu(), lse3.cpu(), want, want_lse, vmax, "bf16", "bf16", "large cluster")
 
 
-def test_graph_capture_of_fused_attention():
+@pytest.mark.parametrize("fused", [True, "cluster"], ids=["ws", "cluster"])
+def test_graph_capture_of_fused_attention(fused):
     B, Hq, Hkv, L, D, R = 2, 8, 2, 512, 128, 8
     q, k, v = make(B, Hq, Hkv, L, D, seed=19)
     from lse_weighted_merge_b200 import decode_attention
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
-    eager, eager_lse = decode_attention(qd, kd, vd, splits=R, fused=True)
+    eager, eager_lse = decode_attention(qd, kd, vd, splits=R, fused=fused)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):   # the capture stream's workspace is made before capture
+        decode_attention(qd, kd, vd, splits=R, fused=fused)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        o, l = decode_attention(qd, kd, vd, splits=R, fused=True)
-    g.replay()
+    with torch.cuda.graph(g, stream=s):
+        o, l = decode_attention(qd, kd, vd, splits=R, fused=fused)
+    for _ in range(3):   # replays reuse the workspace: each leaves its counters at 0
+        g.replay()
     torch.cuda.synchronize()
     assert torch.equal(o, eager) and torch.equal(l, eager_lse)
     del g
@@ -237,10 +296,11 @@ def test_automatic_splits_and_fusion(B, Hq, Hkv, L):
     check_rows(out.cpu(), lse.cpu(), want, want_lse, vmax, "bf16", "bf16", "auto")
 
 
-@pytest.mark.parametrize("fused", [True, False], ids=["fused", "partials"])
+@pytest.mark.parametrize("fused", [True, "ws", False], ids=["cluster", "ws", "partials"])
 def test_outputs_written_exactly_in_bounds(fused):
-    """Outputs carved out of larger buffers with canary guard bytes: after a
-    call no guard byte has changed and q, k, v are left as they were."""
+    """Outputs (and the workspace) carved out of larger buffers with canary
+    guard bytes: after a call no guard byte has changed and q, k, v are left
+    as they were."""
     B, Hq, Hkv, L, D, R = 2, 8, 2, 300, 128, 4
     q, k, v = make(B, Hq, Hkv, L, D, seed=77)
     scale = 1 / math.sqrt(D)
@@ -251,14 +311,18 @@ def test_outputs_written_exactly_in_bounds(fused):
     l_bytes = B * Hq * 4 if fused else B * Hq * R * 4
     o_buf = torch.full((G + o_bytes + G,), canary, dtype=torch.uint8, device="cuda")
     l_buf = torch.full((G + l_bytes + G,), canary, dtype=torch.uint8, device="cuda")
+    w_bytes = nat.decode_workspace_bytes(B, Hq, Hkv, R, D)
+    w_buf = torch.full((G + w_bytes + G,), canary, dtype=torch.uint8, device="cuda")
+    w_buf[G:G + w_bytes].zero_()
+    wkw = dict(workspace=w_buf.data_ptr() + G, workspace_bytes=w_bytes) if fused == "ws" else {}
     st = (qd.stride(0), qd.stride(1), kd.stride(0), kd.stride(1), kd.stride(2),
           vd.stride(0), vd.stride(1), vd.stride(2))
     nat.decode_raw(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), 0, B, Hq, Hkv, L, D, R, scale, st,
                    nat.BF16, o_buf.data_ptr() + G, l_buf.data_ptr() + G,
-                   torch.cuda.current_stream().cuda_stream, fused=fused,
-                   **({"out_dtype": nat.BF16} if fused else {}))
+                   torch.cuda.current_stream().cuda_stream, fused=bool(fused),
+                   **({"out_dtype": nat.BF16} if fused else {}), **wkw)
     torch.cuda.synchronize()
-    for buf, n in ((o_buf, o_bytes), (l_buf, l_bytes)):
+    for buf, n in ((o_buf, o_bytes), (l_buf, l_bytes), (w_buf, w_bytes)):
         assert bool((buf[:G] == canary).all()) and bool((buf[G + n:] == canary).all())
     assert torch.equal(qd, q0) and torch.equal(kd, k0) and torch.equal(vd, v0)
     if fused:

@@ -304,3 +304,37 @@ def test_many_partials_wide_path(R, B, H, D):
                               (inp["o_strides"], inp["lse_strides"]), nat.BF16, nat.BF16,
                               0x7f2000000000, 0x7f3000000000)
     assert plan["path"] == nat.PATH_WIDE
+
+
+def test_host_context_through_the_c_abi():
+    """lse_merge_host on a context of its own: a call whose staging needs
+    exceed the context's area is refused before anything is enqueued; a
+    call that fits merges host partials into host outputs, matching the
+    oracle; the context is destroyed after its last call."""
+    w = W["r4_b64_h32_d128_masked"]
+    inp = synth.make_inputs(w, B=16, seed=31, poison_empty=True)
+    R, B, H, D = inp["R"], inp["B"], inp["H"], inp["D"]
+    h_o = torch.from_numpy(inp["o"].view(np.int16)).pin_memory()
+    h_l = torch.from_numpy(inp["lse"]).pin_memory()
+    out = torch.full((B, H, D), float("nan"), dtype=torch.bfloat16).pin_memory()
+    out_lse = torch.full((B, H), float("nan"), dtype=torch.float32).pin_memory()
+    need = nat.host_stage_bytes(R, B, H, D, nat.BF16, nat.BF16)
+    small = nat.host_create(need - 256)
+    try:
+        rc = nat.host_merge_raw(small, h_o.data_ptr(), h_l.data_ptr(), R, B, H, D, nat.LAYOUT_BHRD,
+                                nat.BF16, nat.BF16, out.data_ptr(), out_lse.data_ptr(), 4,
+                                check=False)
+        assert rc == nat.ESCRATCH
+    finally:
+        nat.host_destroy(small)
+    ctx = nat.host_create(need)
+    try:
+        s = torch.cuda.current_stream()
+        nat.host_merge_raw(ctx, h_o.data_ptr(), h_l.data_ptr(), R, B, H, D, nat.LAYOUT_BHRD,
+                           nat.BF16, nat.BF16, out.data_ptr(), out_lse.data_ptr(), 5,
+                           stream=s.cuda_stream)
+        s.synchronize()
+    finally:
+        nat.host_destroy(ctx)
+    want, want_lse = run_oracle(inp)
+    check(out.double().numpy(), out_lse.double().numpy(), want, want_lse, "bf16", "host context")
