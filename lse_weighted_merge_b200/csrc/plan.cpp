@@ -301,7 +301,9 @@ int make_attn_plan(const void* q, const void* k, const void* v, int B, int Hq, i
     // mbarrier, lse [R][G] padded to 4 floats, o [R][G][D]), which siblings
     // fill while CTA 0 may still use its ring
     const int64_t rg = (int64_t)R * p.G;
-    p.smem = mode == kAttnModeCluster ? base + 16 + ((rg + 3) & ~(int64_t)3) * 4 + rg * D * 4 : base;
+    p.smem = base;
+    // cluster: CTA 0's receive buffer behind the ring
+    if (mode == kAttnModeCluster) p.smem = base + 16 + ((rg + 3) & ~(int64_t)3) * 4 + rg * D * 4;
     if (p.smem > kAttnMaxSmem) return LSE_MERGE_EUNSUP;
     *plan = p;
     return LSE_MERGE_OK;

@@ -25,10 +25,20 @@ constexpr int kMinBlocks = LSEM_MINB;
 #define LSEM_MINB_VEC1 LSEM_MINB
 #endif
 #ifndef LSEM_MINB_STREAM
-#define LSEM_MINB_STREAM LSEM_MINB
+#define LSEM_MINB_STREAM 0
 #endif
 constexpr int kMinBlocksVec1 = LSEM_MINB_VEC1;
 constexpr int kMinBlocksStream = LSEM_MINB_STREAM;
+// Resident CTAs per SM the persistent kernel is compiled for (caps its
+// registers; 0 in LSEM_MINB_STREAM picks per instantiation).  Measured on B200
+// back to back: the 16-partial kernel (R=16 B=512 H=16 D=512, bf16 -> fp32) at
+// 120 registers (8 CTAs of 2 warps per SM) 26.3 us, capped for 8 CTAs (112
+// registers, 9 fit) 25.2 us; the 8-partial two-column kernel (rank-major R=8
+// B=256 H=64 D=128, fp16) at 158 registers (6 CTAs) 8.9 us, capped for 7 CTAs
+// (122 registers, 8 fit) 7.3 us, capped for 8 (128 registers) 7.9 us.
+constexpr int stream_min_blocks(int rc, int nv) {
+    return kMinBlocksStream > 0 ? kMinBlocksStream : (rc == 8 && nv == 2 ? 7 : 8);
+}
 // Launch with programmatic stream serialization (the next kernel in the
 // stream may be scheduled while this one drains; it waits before touching
 // memory).  Hides the launch gap between back-to-back merges.

@@ -54,6 +54,22 @@ def test_state_update_dtype_pairs(acc_dt, new_dt, D):
     check(got, got_lse, want, want_lse, acc_dt, f"{acc_dt}<-{new_dt} D{D}")
 
 
+@pytest.mark.parametrize("acc_dt,new_dt", [("f32", "bf16"), ("bf16", "f16"), ("f16", "f32")])
+@pytest.mark.parametrize("D", [264, 300, 512, 520, 1000])
+def test_state_update_long_rows(acc_dt, new_dt, D):
+    """Rows of more than 32 chunks of 8, which one group of 32 lanes folds
+    in two or more passes (D = 264 ... 1000), the last pass ragged for most;
+    300 and 1000 take the element path."""
+    B, H = 3, 5
+    acc, la, new, ln = make(B, H, D, acc_dt, new_dt, seed=D + 7)
+    la[2] = -np.inf
+    ln[6] = -np.inf
+    want, want_lse = oracle.state_update(acc, la, synth.DTYPES[acc_dt], new, ln,
+                                         synth.DTYPES[new_dt], B, H, D)
+    got, got_lse = run(acc, la, new, ln, B, H, D, acc_dt, new_dt)
+    check(got, got_lse, want, want_lse, acc_dt, f"{acc_dt}<-{new_dt} D{D}")
+
+
 def test_empty_sides_are_not_read():
     B, H, D = 3, 4, 64
     acc, la, new, ln = make(B, H, D, "bf16", "bf16", seed=1)
@@ -112,7 +128,8 @@ def test_large_state_update_full_parity():
     check(got, got_lse, want, want_lse, "f32", "large")
 
 
-@pytest.mark.parametrize("acc_dt,D", [("f32", 96), ("bf16", 100), ("f16", 8)])
+@pytest.mark.parametrize("acc_dt,D", [("f32", 96), ("bf16", 100), ("f16", 8), ("f32", 300),
+                                      ("bf16", 512), ("f32", 1000)])
 def test_writes_stay_inside_the_accumulator(acc_dt, D):
     """The accumulator and its lse are carved out of larger buffers whose
     guard bytes hold a canary pattern: after a fold no guard byte has
