@@ -486,24 +486,64 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
         if (threadIdx.x == 0) s_last = atom_add_acq_rel_gpu(p.ws_cnt + bh, 1u) == (unsigned)(R - 1);
         __syncthreads();
         if (!s_last) return;
-        for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-            const int gg = idx / D, d = idx - gg * D;
-            float M = -INFINITY;
-            for (int j = 0; j < R; ++j) M = fmaxf(M, __ldcg(dst_l + j * G + gg));
-            float den = 0.f, num = 0.f;
-            if (M != -INFINITY) {
-                for (int j = 0; j < R; ++j) {
-                    const float lj = __ldcg(dst_l + j * G + gg);
-                    if (lj != -INFINITY) {   // an empty split's o is not used
-                        const float e = expf(lj - M);
-                        den += e;
-                        num += e * __ldcg(dst_o + ((int64_t)j * G + gg) * D + d);
+        // The merge: each thread takes up to kMergeOut output elements and
+        // walks the splits in batches of kMergeBatch, the lse and o loads of a
+        // whole batch (L2: the partials were written moments ago) issued
+        // before any is used, then folded into a running (max, weight sum,
+        // weighted sum) per element -- one L2 round trip per batch, none
+        // for the weights alone.  An empty split has lse -inf and o 0.
+        constexpr int kMergeBatch = 4, kMergeOut = 4;
+        const int GD = G * D;
+        for (int base = threadIdx.x; base < GD; base += kMergeOut * blockDim.x) {
+            float mx[kMergeOut], den[kMergeOut], num[kMergeOut];
+#pragma unroll
+            for (int k = 0; k < kMergeOut; ++k) {
+                mx[k] = -INFINITY;
+                den[k] = num[k] = 0.f;
+            }
+            for (int j0 = 0; j0 < R; j0 += kMergeBatch) {
+                float lv[kMergeOut][kMergeBatch], ov[kMergeOut][kMergeBatch];
+#pragma unroll
+                for (int k = 0; k < kMergeOut; ++k) {
+                    const int idx = base + k * blockDim.x;
+                    const int gg = idx < GD ? idx / D : 0, d = idx - gg * D;
+#pragma unroll
+                    for (int u = 0; u < kMergeBatch; ++u) {
+                        const int j = j0 + u;
+                        const bool in = idx < GD && j < R;
+                        lv[k][u] = in ? __ldcg(dst_l + j * G + gg) : -INFINITY;
+                        ov[k][u] = in ? __ldcg(dst_o + ((int64_t)j * G + gg) * D + d) : 0.f;
                     }
                 }
+#pragma unroll
+                for (int k = 0; k < kMergeOut; ++k) {
+                    float bm = mx[k];
+#pragma unroll
+                    for (int u = 0; u < kMergeBatch; ++u) bm = fmaxf(bm, lv[k][u]);
+                    const float ref = bm == -INFINITY ? 0.f : bm;
+                    const float sc = expf(mx[k] - ref);   // 0 while nothing was seen
+                    den[k] *= sc;
+                    num[k] *= sc;
+#pragma unroll
+                    for (int u = 0; u < kMergeBatch; ++u) {
+                        const float e = expf(lv[k][u] - ref);   // 0 for an empty split
+                        den[k] += e;
+                        num[k] = fmaf(e, ov[k][u], num[k]);
+                    }
+                    mx[k] = bm;
+                }
             }
-            const int64_t row = rows_b + gg;
-            store_out<TOut>(p.out + (row * D + d) * (int64_t)sizeof(TOut), den > 0.f ? num / den : 0.f);
-            if (d == 0) p.out_lse[row] = den > 0.f ? M + logf(den) : -INFINITY;
+#pragma unroll
+            for (int k = 0; k < kMergeOut; ++k) {
+                const int idx = base + k * blockDim.x;
+                if (idx < GD) {
+                    const int gg = idx / D, d = idx - gg * D;
+                    const int64_t row = rows_b + gg;
+                    store_out<TOut>(p.out + (row * D + d) * (int64_t)sizeof(TOut),
+                                    den[k] > 0.f ? num[k] / den[k] : 0.f);
+                    if (d == 0) p.out_lse[row] = den[k] > 0.f ? mx[k] + logf(den[k]) : -INFINITY;
+                }
+            }
         }
         if (threadIdx.x == 0) p.ws_cnt[bh] = 0u;   // every split of this call has counted
     }
