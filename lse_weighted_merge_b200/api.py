@@ -244,14 +244,16 @@ def decode_attention(q, k, v, *, splits: int | None = None, scale: float | None 
     into ``splits`` shards (default: enough shards for about two CTAs per SM,
     a power of two of at least 64 keys each, at most 64).
 
-    fused (default True): one launch; each shard's CTA writes its fp32
-    partial into a workspace kept for this device and stream, and the last
-    shard of each (sequence, KV head) to finish merges them
-    (lse_merge_decode_attention_ws).  fused="cluster": one launch in which the
-    shards of a (sequence, KV head) form a thread-block cluster and merge
-    through distributed shared memory, no workspace (splits 1, 2, 4 or 8;
-    cluster scheduling leaves SM slots idle, so it is slower on large
-    batches).  fused=False: the partials kernel, then merge(), two launches.
+    fused=False (the default): the partials kernel, then merge(), two
+    launches; on B200 the fastest form (the partials stay in L2 and the
+    second launch overlaps the first one's drain).  fused=True: one launch;
+    each shard's CTA writes its fp32 partial into a workspace kept for this
+    device and stream, and the last shard of each (sequence, KV head) to
+    finish merges them (lse_merge_decode_attention_ws), within about 1 % of
+    the two launches.  fused="cluster": one launch in which the shards of a
+    (sequence, KV head) form a thread-block cluster and merge through
+    distributed shared memory, no workspace (splits 1, 2, 4 or 8; cluster
+    scheduling leaves SM slots idle, so it is slower on large batches).
     Returns (out [B, Hq, D], lse [B, Hq]) with the natural-log lse of the
     scaled scores.
     """
@@ -268,7 +270,7 @@ def decode_attention(q, k, v, *, splits: int | None = None, scale: float | None 
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise TypeError("q, k and v must share one dtype")
     if fused is None:
-        fused = True
+        fused = False
     if fused not in (True, False, "cluster"):
         raise ValueError("fused must be True, False or 'cluster'")
     dev = q.device
