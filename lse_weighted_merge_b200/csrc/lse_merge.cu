@@ -431,6 +431,133 @@ __global__ void __launch_bounds__(kBlock, stream_min_blocks(RC, NV)) merge_strea
 }
 
 
+// Persistent form for R > RC partials: the units a lane group walks are
+// (row slice, chunk of RC partials) pairs -- chunk 0..nch-1 of slice grp,
+// then of slice grp + G, ...  The group keeps a running (max M, weight sum,
+// fp32 accumulator) over the chunks of its slice, rescaled by exp(M_old -
+// M_new) when a chunk raises the max (the online form of the same LSE
+// combine), and stores the slice after its last chunk.  As in the kernel
+// above, partial i of the next unit is loaded into x[i] as soon as partial i
+// of this unit is folded, so RC loads per lane stay in flight across chunk
+// and slice boundaries.
+template <typename TIn, typename TOut, int RC>
+__global__ void __launch_bounds__(kBlock, stream_min_blocks(RC, 1)) merge_stream_long_kernel(const KParams p, const int64_t G) {
+    constexpr int N = Elem<TIn>::kVec;
+    constexpr int N2 = N / 2;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int j = (int)(t & (p.lanes - 1));
+    const int64_t grp0 = t >> p.lg;
+    const int64_t grp_w = (t & ~(int64_t)31) >> p.lg;
+    const int64_t trips = grp_w < p.groups ? (p.groups - grp_w + G - 1) / G : 0;
+    const int nch = (p.R + RC - 1) / RC;   // chunks per slice, the same for every group
+
+    struct Slice {
+        const char* o;
+        const float* l;
+        int64_t row;
+        int v, slice;
+        bool live, cl;
+    };
+    auto locate = [&](int64_t g) {
+        Slice s;
+        s.live = g < p.groups;
+        const RowIdx ri = row_of(p, s.live ? g : 0);
+        s.row = ri.row;
+        s.slice = ri.slice;
+        s.v = ri.slice * p.lanes + j;
+        s.cl = s.live && s.v < p.dv;
+        s.o = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)s.v * 16;
+        s.l = p.lse + ri.b * p.l_b + ri.h * p.l_h;
+        return s;
+    };
+    // partial r0 + i of slice s (0 past the row's partials or the row)
+    auto load_chunk = [&](const Slice& s, int r0, uint4 (&x)[RC]) {
+#pragma unroll
+        for (int i = 0; i < RC; ++i) {
+            x[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (s.cl && r0 + i < p.R) x[i] = ld_stream16(s.o + (int64_t)(r0 + i) * p.o_r);
+        }
+    };
+    auto load_lse = [&](const Slice& s, int r0) {
+        return (s.live && j < RC && r0 + j < p.R) ? __ldg(s.l + (int64_t)(r0 + j) * p.l_r) : -INFINITY;
+    };
+
+    Slice cur = locate(grp0);
+    if (kPrefetch && trips > 0) {   // the first chunk's lines, while the previous grid drains
+#pragma unroll
+        for (int i = 0; i < RC; ++i)
+            if (cur.cl && i < p.R) prefetch_l2(cur.o + (int64_t)i * p.o_r);
+        if (cur.live && j < RC && j < p.R) prefetch_l2(cur.l + (int64_t)j * p.l_r);
+    }
+    pdl_wait();
+    pdl_release();
+    uint4 x[RC];
+    load_chunk(cur, 0, x);
+    float l = load_lse(cur, 0);
+
+    float M = -INFINITY, es = 0.f;
+    uint64_t acc[N2];
+#pragma unroll
+    for (int q = 0; q < N2; ++q) acc[q] = 0ull;
+    for (int64_t it = 0; it < trips; ++it) {
+        for (int c = 0; c < nch; ++c) {
+            const bool last = c + 1 == nch;
+            const Slice nxt = last ? locate(grp0 + (it + 1) * G) : cur;
+            const int rn = last ? 0 : (c + 1) * RC;   // first partial of the next unit
+            const float ln = load_lse(nxt, rn);
+
+            // fold chunk c: rescale the running state to the new max first
+            const float Mn = fmaxf(M, group_max(l, p.lanes));
+            const float ref = (Mn == -INFINITY) ? 0.f : Mn;   // all empty so far: no NaN
+            const float sc = expf(M - ref);                   // 0 while the state is empty
+            const uint64_t sc2 = pack2f(sc, sc);
+#pragma unroll
+            for (int q = 0; q < N2; ++q) mul2(acc[q], sc2);
+            const float e = expf(l - ref);                    // 0 for an empty shard
+            es = es * sc + group_sum(e, p.lanes);
+            M = Mn;
+            const int r0 = c * RC;
+            const bool any_zero = __any_sync(kFull, j < RC && r0 + j < p.R && e == 0.f);
+#pragma unroll
+            for (int i = 0; i < RC; ++i) {
+                const float w = __shfl_sync(kFull, e, i, p.lanes);
+                if (r0 + i < p.R) {
+                    if (!any_zero || w != 0.f) {
+                        uint64_t xx[N2];
+                        Elem<TIn>::unpack2(x[i], xx);
+                        const uint64_t ww = pack2f(w, w);
+#pragma unroll
+                        for (int q = 0; q < N2; ++q) fma2(acc[q], xx[q], ww);
+                    }
+                }
+                x[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (nxt.cl && rn + i < p.R) x[i] = ld_stream16(nxt.o + (int64_t)(rn + i) * p.o_r);
+            }
+            if (last) {
+                const float inv = es > 0.f ? 1.f / es : 0.f;
+                if (cur.cl) {
+                    float f[N];
+#pragma unroll
+                    for (int q = 0; q < N2; ++q) {
+                        unpack2f(acc[q], f[2 * q], f[2 * q + 1]);
+                        f[2 * q] *= inv;
+                        f[2 * q + 1] *= inv;
+                    }
+                    store_vec<TOut, N>(p.out + (cur.row * p.D + (int64_t)cur.v * N) * (int64_t)sizeof(TOut), f);
+                }
+                if (cur.live && cur.slice == 0 && j == 0)
+                    p.out_lse[cur.row] = es > 0.f ? M + logf(es) : -INFINITY;
+                M = -INFINITY;
+                es = 0.f;
+#pragma unroll
+                for (int q = 0; q < N2; ++q) acc[q] = 0ull;
+            }
+            cur = nxt;
+            l = ln;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ wide kernel
 
 // For R > 16, and for a handful of rows of any R (at most kWideMaxSlices row
@@ -788,6 +915,27 @@ StateFn pick_state(int acc_dtype, int new_dtype, bool vec) {
 using KernelFn = void (*)(KParams);
 using StreamFn = void (*)(KParams, int64_t);
 
+template <typename TIn, typename TOut>
+StreamFn pick_long_rc(int rc) {
+    return rc == 4 ? merge_stream_long_kernel<TIn, TOut, 4>
+                   : rc == 8 ? merge_stream_long_kernel<TIn, TOut, 8> : merge_stream_long_kernel<TIn, TOut, 16>;
+}
+template <typename TIn>
+StreamFn pick_long_out(int rc, int out_dtype) {
+    switch (out_dtype) {
+        case LSE_MERGE_F32: return pick_long_rc<TIn, float>(rc);
+        case LSE_MERGE_F16: return pick_long_rc<TIn, __half>(rc);
+        default: return pick_long_rc<TIn, __nv_bfloat16>(rc);
+    }
+}
+StreamFn pick_stream_long(int rc, int in_dtype, int out_dtype) {
+    switch (in_dtype) {
+        case LSE_MERGE_F32: return pick_long_out<float>(rc, out_dtype);
+        case LSE_MERGE_F16: return pick_long_out<__half>(rc, out_dtype);
+        default: return pick_long_out<__nv_bfloat16>(rc, out_dtype);
+    }
+}
+
 // (rc, nv) pairs the planner produces: rc * nv <= 16 loads of 16 bytes per lane.
 template <typename TIn, typename TOut>
 StreamFn pick_stream_kernel(int rc, int nv) {
@@ -950,7 +1098,8 @@ int run(const void* partial_o, const float* partial_lse, int R, int B, int H, in
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e;
     if (pl.path == LSE_MERGE_PATH_STREAM) {
-        const StreamFn fn = pick_stream(pl.rc, pl.nv, in_dtype, out_dtype);
+        const StreamFn fn = R > pl.rc ? pick_stream_long(pl.rc, in_dtype, out_dtype)
+                                      : pick_stream(pl.rc, pl.nv, in_dtype, out_dtype);
         const int64_t want = (pl.groups * pl.lanes + pl.block - 1) / pl.block;
         int grid = 0;
         const int qe = persistent_grid((const void*)fn, pl.block, want, &grid);

@@ -107,7 +107,7 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
     lse_merge_plan p{};
     if (vec_ok && path != LSE_MERGE_PATH_SCALAR) {
         const int dv = D / vec;
-        const int rc = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
+        int rc = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
         // lanes and slices for nv columns per lane
         auto shape = [&](int nv, int* lanes, int* slices) {
             const int cols = (dv + nv - 1) / nv;
@@ -120,21 +120,30 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
         int lanes1, slices1;
         shape(1, &lanes1, &slices1);
         const bool small = rows * slices1 * lanes1 <= kLatencyMaxThreads;
-        const bool stream_ok = R <= rc;   // every partial of a row slice in one batch
+        // STREAM takes a row slice's partials in one batch when R <= rc, and
+        // in chunks of 16 with a running max (the long form) beyond.
         const i128 in_bytes = (i128)R * rows * D * ib;
         int chosen = path;
         if (chosen == LSE_MERGE_PATH_AUTO) {
             if (small)
                 chosen = LSE_MERGE_PATH_LATENCY;
-            else if (!stream_ok || rows * slices1 <= kWideMaxSlices)
+            else if (rows * slices1 <= kWideMaxSlices)
                 chosen = LSE_MERGE_PATH_WIDE;
+            else if (R > rc) {
+                // the long form when its lanes (one column each) fill most of
+                // a wave; otherwise WIDE, which also spreads a row's partials
+                // over the warps of a CTA
+                const int lanes_d = next_pow2(dv < 32 ? dv : 32);
+                const i128 threads = rows * ((dv + lanes_d - 1) / lanes_d) * (lanes_d < 4 ? 4 : lanes_d);
+                chosen = kAutoStreamLong && threads >= kLongMinThreads ? LSE_MERGE_PATH_STREAM
+                                                                       : LSE_MERGE_PATH_WIDE;
+            }
             else if (kAutoStream && in_bytes >= kStreamMinBytes && in_bytes <= kStreamMaxBytes)
                 chosen = LSE_MERGE_PATH_STREAM;
             else
                 chosen = LSE_MERGE_PATH_VECTOR;
         }
         if (chosen == LSE_MERGE_PATH_LATENCY && !small) return LSE_MERGE_EPATH;
-        if (chosen == LSE_MERGE_PATH_STREAM && !stream_ok) return LSE_MERGE_EPATH;
         if (chosen == LSE_MERGE_PATH_WIDE) {
             // One 16-byte column per lane, at least 4 lanes.  Just enough
             // warps (at most 4) that the lane groups hold every partial of the
@@ -164,7 +173,12 @@ int make_plan(const void* o, const float* lse, int R, int B, int H, int D,
             return LSE_MERGE_OK;
         }
         int nv = 1;
-        if (chosen != LSE_MERGE_PATH_LATENCY) {
+        if (chosen == LSE_MERGE_PATH_STREAM && R > rc) {
+            // the long form: chunks of as many partials as a row has
+            // 16-byte columns (4..16), one column per lane
+            const int lanes_d = next_pow2(dv < 32 ? dv : 32);
+            rc = lanes_d < 4 ? 4 : (lanes_d > 16 ? 16 : lanes_d);
+        } else if (chosen != LSE_MERGE_PATH_LATENCY) {
             nv = 16 / rc < kMaxNv ? 16 / rc : kMaxNv;
             while (nv > 1 && (dv + nv - 1) / nv < rc) nv >>= 1;
         }

@@ -64,6 +64,18 @@ constexpr int kPrefetch = LSEM_PREFETCH;
 #define LSEM_AUTO_STREAM 1
 #endif
 constexpr int kAutoStream = LSEM_AUTO_STREAM;
+// AUTO takes R > 16 partials over more than kWideMaxSlices row slices with
+// the long form of the persistent kernel (chunks of 16) instead of WIDE.
+#ifndef LSEM_AUTO_STREAM_LONG
+#define LSEM_AUTO_STREAM_LONG 1
+#endif
+constexpr int kAutoStreamLong = LSEM_AUTO_STREAM_LONG;
+// Threads (one 16-byte column per lane) from which AUTO prefers the long form
+// for R > 16: about 0.6 of a B200 wave (148 SMs x 8 CTAs x 64 threads).
+// Measured, graph-replayed: R=24 over 4096 rows of D=128 (65536 threads) long
+// 7.7 us, WIDE 8.6; R=32 over 2048 rows (32768) long 6.3, WIDE 5.3; R=64 over
+// 2048 rows 10.3 and 10.2; R=128 over 512 rows long 13.5, WIDE 5.6.
+constexpr long long kLongMinThreads = 48 * 1024;
 #ifndef LSEM_STREAM_MAX_MB
 #define LSEM_STREAM_MAX_MB 256
 #endif

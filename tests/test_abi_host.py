@@ -61,7 +61,6 @@ def q(R=2, B=1, H=2, D=64, strides=None, i=nat.BF16, o=nat.BF16, po=PO, pl=PL, o
     (dict(out=PL), nat.EALIAS),
     (dict(path=7), nat.EPATH),
     (dict(D=60, path=nat.PATH_WIDE), nat.EPATH),
-    (dict(R=17, B=64, H=64, path=nat.PATH_STREAM), nat.EPATH),
     (dict(D=60, path=nat.PATH_STREAM), nat.EPATH),
     (dict(B=64, H=64, path=nat.PATH_LATENCY), nat.EPATH),
     (dict(B=1, H=32, path=nat.PATH_LATENCY), nat.EPATH),     # 128 threads > one 64-thread CTA
@@ -137,7 +136,8 @@ def test_fallback_to_scalar_and_forced_paths():
 @pytest.mark.parametrize("R,want_rc,want_nv,want_lanes,want_path", [
     (1, 4, 2, 4, nat.PATH_VECTOR), (3, 4, 2, 4, nat.PATH_VECTOR), (5, 8, 1, 8, nat.PATH_VECTOR),
     (9, 16, 1, 16, nat.PATH_VECTOR), (16, 16, 1, 16, nat.PATH_STREAM),   # 16 x 0.5 MB = 8 MB
-    (17, 8, 1, 8, nat.PATH_WIDE), (33, 8, 1, 8, nat.PATH_WIDE), (100, 8, 1, 8, nat.PATH_WIDE)])
+    (17, 8, 1, 8, nat.PATH_WIDE), (33, 8, 1, 8, nat.PATH_WIDE),            # 4096 rows x 8 lanes:
+    (100, 8, 1, 8, nat.PATH_WIDE)])                                        # too few for the long form
 def test_rc_nv_and_lanes_follow_R(R, want_rc, want_nv, want_lanes, want_path):
     rc, plan = q(R=R, D=64, B=64, H=64)      # 8 vectors per row, beyond one CTA, < 8 MB
     assert rc == 0 and (plan["rc"], plan["nv"], plan["lanes"], plan["path"]) == \
@@ -176,9 +176,16 @@ def test_stream_only_below_its_size_limit():
     assert big["path"] == nat.PATH_VECTOR and big["grid"] > 0
     small = q(R=16, B=512, H=16, D=512, o=nat.F32)[1]
     assert small["path"] == nat.PATH_STREAM and small["grid"] == 0
-    # R > 16: the partials of a row spread over one CTA (WIDE)
-    assert q(R=17, B=64, H=64)[1]["path"] == nat.PATH_WIDE
+    # R > 16 over many rows: the persistent kernel in chunks of partials; over a
+    # few rows (<= 128 slices): the partials of a row spread over one CTA (WIDE)
+    long = q(R=17, B=64, H=128)[1]                 # 8192 rows x 8 lanes (D=64): the long form
+    assert long["path"] == nat.PATH_STREAM and long["rc"] == 8 and long["nv"] == 1
+    assert q(R=17, B=64, H=64)[1]["path"] == nat.PATH_WIDE   # 4096 x 8 lanes: WIDE
+    assert q(R=24, B=128, H=32, D=128)[1]["path"] == nat.PATH_STREAM
+    assert q(R=128, B=16, H=32, D=128)[1]["path"] == nat.PATH_WIDE
+    assert q(R=64, B=4, H=8)[1]["path"] == nat.PATH_WIDE
     assert q(R=17, B=64, H=64, path=nat.PATH_VECTOR)[1]["path"] == nat.PATH_VECTOR
+    assert q(R=17, B=64, H=64, path=nat.PATH_WIDE)[1]["path"] == nat.PATH_WIDE
 
 
 @pytest.mark.parametrize("D,lanes,nv,slices", [(8, 4, 1, 1), (24, 4, 1, 1), (128, 8, 2, 1),

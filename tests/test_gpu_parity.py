@@ -156,8 +156,9 @@ def test_public_merge_both_layouts():
         merge(o_rbhd.cpu(), l_rbhd.cpu(), layout="rbhd")
 
 
-def test_outputs_written_exactly_in_bounds():
-    inp = synth.make_inputs(W["r4_b64_h32_d128_masked"], B=3, H=5)
+@pytest.mark.parametrize("R,D", [(4, 128), (37, 72)], ids=["R4", "R37-long-form"])
+def test_outputs_written_exactly_in_bounds(R, D):
+    inp = synth.make_inputs(W["r4_b64_h32_d128_masked"], B=3, H=5, R=R, D=D)
     R, B, H, D = inp["R"], inp["B"], inp["H"], inp["D"]
     d_o = torch.from_numpy(inp["o"].view(np.int16)).cuda()
     d_l = torch.from_numpy(inp["lse"]).cuda()
@@ -292,18 +293,40 @@ def test_merge_host_pipelined_calls_in_a_row(layout):
               f"call {k} {plan[k]}")
 
 
-@pytest.mark.parametrize("R,B,H,D", [(64, 1, 8, 128), (64, 64, 32, 128), (128, 4, 8, 512),
-                                     (48, 2, 3, 64)])
-def test_many_partials_wide_path(R, B, H, D):
-    """Large R (many KV splits): the AUTO (wide) path against the oracle, with
-    empty shards and an all-empty row among the inputs."""
+@pytest.mark.parametrize("R,B,H,D,want", [(64, 1, 8, 128, nat.PATH_WIDE), (128, 4, 8, 512, nat.PATH_WIDE),
+                                          (48, 2, 3, 64, nat.PATH_WIDE), (64, 64, 32, 128, nat.PATH_WIDE),
+                                          (24, 128, 32, 128, nat.PATH_STREAM)])
+def test_many_partials_auto_path(R, B, H, D, want):
+    """Large R (many KV splits) against the oracle, with empty shards holding
+    NaN and all-empty rows among the inputs: a few rows take the wide path,
+    many rows the persistent kernel's long form."""
     w = W["r4_b64_h32_d128_masked"]
     inp = synth.make_inputs(w, R=R, B=B, H=H, D=D, seed=R + B, poison_empty=True)
-    stats = parity(inp, what=f"wide R{R}")
+    parity(inp, what=f"auto R{R}")
     rc, plan = nat.plan_query(0x7f0000000000, 0x7f1000000000, R, B, H, D,
                               (inp["o_strides"], inp["lse_strides"]), nat.BF16, nat.BF16,
                               0x7f2000000000, 0x7f3000000000)
-    assert plan["path"] == nat.PATH_WIDE
+    assert plan["path"] == want
+
+
+@pytest.mark.parametrize("R,D,layout,in_dt,out_dt", [
+    (17, 128, "bhrd", "bf16", "bf16"),    # one chunk of 16 and a ragged one of 1
+    (32, 512, "bhrd", "bf16", "f32"),     # two slices per row, two full chunks
+    (33, 64, "rbhd", "f16", "f16"),       # chunks of 8 (8 columns a row), rank-major
+    (100, 8, "bhrd", "f32", "bf16"),      # chunks of 4 (two fp32 columns a row: 4 lanes)
+    (257, 256, "rbhd", "bf16", "bf16"),   # many chunks
+    (24, 1000, "bhrd", "f16", "f32"),     # ragged last slice of a long row
+])
+def test_long_form_of_the_persistent_kernel(R, D, layout, in_dt, out_dt):
+    """R > 16 on the persistent kernel (chunks with a running max): every
+    dtype pair and both layouts against the oracle, with empty shards holding
+    NaN and all-empty rows; the same inputs forced through the wide path
+    agree too."""
+    w = W["r4_b64_h32_d128_masked"]
+    inp = synth.make_inputs(w, R=R, B=12, H=16, D=D, layout=layout, in_dtype=in_dt,
+                            out_dtype=out_dt, seed=R * 7 + D, poison_empty=True)
+    parity(inp, nat.PATH_STREAM, what=f"long R{R} D{D} {layout} {in_dt}->{out_dt}")
+    parity(inp, nat.PATH_WIDE, what=f"wide R{R} D{D} {layout} {in_dt}->{out_dt}")
 
 
 def test_host_context_through_the_c_abi():
