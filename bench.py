@@ -278,11 +278,13 @@ class DeviceSets:
         self.args = [(self.o[i].data_ptr(), self.lse[i].data_ptr(), self.out[i].data_ptr(),
                       self.out_lse[i].data_ptr()) for i in range(n)]
 
+    path = 0   # AUTO
+
     def launch(self, i: int, stream_handle: int):
         from lse_weighted_merge_b200 import _native as nat
         o, l, out, ol = self.args[i % self.n]
         rc = nat.merge_raw(o, l, self.R, self.B, self.H, self.D, self.strides, self.ind,
-                           self.outd, out, ol, stream_handle, check=False)
+                           self.outd, out, ol, stream_handle, self.path, check=False)
         if rc != 0:
             raise RuntimeError(f"lse_merge returned {rc}: {nat.strerror(rc)}")
 
@@ -757,11 +759,39 @@ def extra_workloads(device, l2: int, dist, clock, trials: int = 5):
         del sets
         torch.cuda.empty_cache()
     extra = {"state_update": time_state_update(device, l2, peak, trials=trials),
+             "many_partials": time_many_partials(device, l2, peak, trials=trials),
              "decode_attention": time_decode_attention(device, peak, trials=trials),
              "cp_exchange_merge": time_cp_exchange(device, peak, trials=trials),
              "workload_detail": detail,
              "workloads": compact}
     return extra, captured
+
+
+def time_many_partials(device, l2: int, peak: float, trials: int = 5) -> dict:
+    """A merge of R=32 partials (bf16 [B,H,R,D], B=256 H=16 D=512, 139 MB):
+    graph-replayed us/call (100 calls x 50 replays, median of `trials`) of
+    the AUTO choice (the persistent kernel's long form, chunks of 16 partials
+    with a running max) and of the WIDE path forced, inputs rotated past L2."""
+    import torch
+    from lse_weighted_merge_b200 import _native as nat
+    from lse_weighted_merge_b200 import synth
+    w = synth.Workload("r32_b256_h16_d512", 32, 256, 16, 512, "bf16", "bf16", "bhrd", 1.0,
+                       "normal", (8.0, 4.0), 1200)
+    inp = synth.make_inputs(w)
+    sets = DeviceSets(inp, n_sets(w.bytes_total(), l2), device)
+    row = {"shape": "R=32 B=256 H=16 D=512, bf16 [B,H,R,D] -> bf16", "bytes_per_call": w.bytes_total()}
+    for tag, path in (("auto", nat.PATH_AUTO), ("wide", nat.PATH_WIDE)):
+        sets.path = path
+        us, _, _ = time_graph(sets, 100, 50, device, trials)
+        row[tag] = {"graph_us_per_call": us, "gbs": w.bytes_total() / (us * 1e-6) / 1e9,
+                    "frac_of_measured_hbm": w.bytes_total() / (us * 1e-6) / 1e9 / peak}
+    st = synth.strides(w.layout, w.R, w.B, w.H, w.D)
+    rc, plan = nat.plan_query(sets.args[0][0], sets.args[0][1], w.R, w.B, w.H, w.D, st,
+                              nat.BF16, nat.BF16, sets.args[0][2], sets.args[0][3])
+    row["auto"]["path"] = plan["path_name"] + (" (long form)" if w.R > plan["rc"] else "")
+    del sets
+    torch.cuda.empty_cache()
+    return row
 
 
 def time_cp_exchange(device, peak: float, only: str | None = None, trials: int = 5) -> dict:

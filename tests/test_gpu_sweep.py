@@ -20,6 +20,14 @@ def _cases(n=48, seed=2024):
     out = []
     for i in range(n):
         kind = i % 4
+        if i % 8 == 7:     # R > 16 over many rows: the persistent kernel's long form
+            R, B, H = int(rng.choice([17, 20, 33])), int(rng.choice([64, 128])), 64
+            D = int(rng.choice([128, 200, 256]))
+            ind, outd = DTS[int(rng.integers(0, 3))], DTS[int(rng.integers(0, 3))]
+            layout = "bhrd" if rng.random() < 0.6 else "rbhd"
+            out.append(dict(R=R, B=B, H=H, D=D, in_dtype=ind, out_dtype=outd, layout=layout,
+                            seed=3000 + i, base=base))
+            continue
         if kind == 0:      # few rows: LATENCY / WIDE boundary
             R, B, H = int(rng.integers(1, 40)), int(rng.integers(1, 4)), int(rng.integers(1, 9))
         elif kind == 1:    # R around 16: STREAM/VECTOR vs WIDE
@@ -63,6 +71,7 @@ def test_the_sweep_takes_every_path():
     """Host only: the planner's choice for each case, from pointer values alone
     (plan_query never dereferences them), covers all five kernel paths."""
     seen = set()
+    long_form = 0
     for case in CASES:
         c = dict(case)
         base = c.pop("base")
@@ -74,4 +83,6 @@ def test_the_sweep_takes_every_path():
                                   synth.DTYPES[w.out_dtype], 0x7F2000000000, 0x7F3000000000)
         assert rc == nat.OK
         seen.add(plan["path_name"])
+        long_form += plan["path"] == nat.PATH_STREAM and w.R > plan["rc"]
     assert seen == {"latency", "wide", "vector", "stream", "scalar"}, seen
+    assert long_form >= 3, long_form
