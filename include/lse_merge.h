@@ -80,9 +80,10 @@ typedef struct {
 #define LSE_MERGE_PATH_LATENCY 2  /* the vector kernel as one small CTA (tiny B*H) */
 #define LSE_MERGE_PATH_SCALAR 3   /* element loads, any alignment of strides and D */
 #define LSE_MERGE_PATH_STREAM 4   /* persistent vector kernel, loads of the next row slice
-                                     issued as the current one is consumed (R <= 16) */
+                                     issued as the current one is consumed; R > 16 in
+                                     chunks of partials with a running max */
 #define LSE_MERGE_PATH_WIDE 5     /* one CTA per row slice, the partials spread over its
-                                     lane groups and their states merged (for large R) */
+                                     lane groups and their states merged (large R, few rows) */
 
 /*
  * Merge R partials of B*H rows.

@@ -55,7 +55,10 @@ namespace lsem {
 namespace {
 
 constexpr int kMaxWorld = LSE_MERGE_CP_MAX_WORLD;
-constexpr int kSendUnroll = 4;   // 16-byte units in flight per thread while sending
+#ifndef LSEM_CP_SEND_UNROLL
+#define LSEM_CP_SEND_UNROLL 4
+#endif
+constexpr int kSendUnroll = LSEM_CP_SEND_UNROLL;   // 16-byte units in flight per thread while sending
 // Poll back-off of the landed-counter wait (measured on B200 with every rank
 // in one launch: 32..256 ns gave 4.43 us per call for 2 ranks of one head,
 // 64..2048 ns 4.53 us).

@@ -55,11 +55,12 @@ constexpr int kPdl = LSEM_PDL;
 #define LSEM_PREFETCH 1
 #endif
 constexpr int kPrefetch = LSEM_PREFETCH;
-// AUTO picks the persistent STREAM kernel for partials between
-// kStreamMinBytes and kStreamMaxBytes and the one-shot VECTOR kernel outside
-// that range.  Measured on B200: STREAM is 3-7 % faster from ~30 MB to
-// ~150 MB of partials; VECTOR is faster below one wave of work (2.1 MB:
-// 2.13 vs 2.36 us graph-replayed) and from ~300 MB on.
+// AUTO picks the persistent STREAM kernel from kStreamMinBytes of partials
+// (up to kStreamMaxBytes) and the one-shot VECTOR kernel below.  Measured on
+// B200: VECTOR is faster below one wave of work (2.1 MB: 2.13 vs 2.36 us
+// graph-replayed); with the register caps and the L2 prefetch STREAM is
+// faster at every larger size, 606 MB of [B,H,R,D] partials included (96.5
+// vs 104.0 us) and 537 MB rank-major (97.3 vs 113.3 us).
 #ifndef LSEM_AUTO_STREAM
 #define LSEM_AUTO_STREAM 1
 #endif
@@ -77,7 +78,7 @@ constexpr int kAutoStreamLong = LSEM_AUTO_STREAM_LONG;
 // 2048 rows 10.3 and 10.2; R=128 over 512 rows long 13.5, WIDE 5.6.
 constexpr long long kLongMinThreads = 48 * 1024;
 #ifndef LSEM_STREAM_MAX_MB
-#define LSEM_STREAM_MAX_MB 256
+#define LSEM_STREAM_MAX_MB (1 << 30)
 #endif
 constexpr long long kStreamMaxBytes = (long long)LSEM_STREAM_MAX_MB << 20;
 constexpr long long kStreamMinBytes = 8ll << 20;

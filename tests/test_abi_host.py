@@ -170,10 +170,10 @@ def test_path_choice_by_size():
     assert q(R=8, B=64, H=64, D=128, o=nat.F32)[1]["path"] == nat.PATH_STREAM
 
 
-def test_stream_only_below_its_size_limit():
-    # 16 partials of 512 bf16 in 1100 batches x 16 heads = 288 MB of partials: one-shot VECTOR
+def test_stream_from_its_size_threshold_up():
+    # 16 partials of 512 bf16 in 1100 batches x 16 heads = 288 MB of partials: still STREAM
     big = q(R=16, B=1100, H=16, D=512, o=nat.F32, out=0x7fa000000000, outl=0x7fb000000000)[1]
-    assert big["path"] == nat.PATH_VECTOR and big["grid"] > 0
+    assert big["path"] == nat.PATH_STREAM and big["grid"] == 0
     small = q(R=16, B=512, H=16, D=512, o=nat.F32)[1]
     assert small["path"] == nat.PATH_STREAM and small["grid"] == 0
     # R > 16 over many rows: the persistent kernel in chunks of partials; over a
