@@ -93,9 +93,10 @@ constexpr int kWideBlock = 128;
 #define LSEM_MAX_NV 2
 #endif
 constexpr int kMaxNv = LSEM_MAX_NV;
-// Size the persistent grid so that every CTA gets the same number of rounds
-// (ceil(work / capacity) rounds, spread evenly), instead of filling the
-// device and leaving a partial last round.
+// When the last round of a full persistent grid would be less than half
+// full, size the grid so that every CTA gets the same number of rounds
+// (ceil(work / capacity) rounds, spread evenly); see balanced() in
+// lse_merge.cu.  0 always fills the device.
 #ifndef LSEM_BALANCE
 #define LSEM_BALANCE 1
 #endif
