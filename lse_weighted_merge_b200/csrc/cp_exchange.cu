@@ -55,10 +55,13 @@ namespace lsem {
 namespace {
 
 constexpr int kMaxWorld = LSE_MERGE_CP_MAX_WORLD;
-#ifndef LSEM_CP_SEND_UNROLL
-#define LSEM_CP_SEND_UNROLL 4
-#endif
-constexpr int kSendUnroll = LSEM_CP_SEND_UNROLL;   // 16-byte units in flight per thread while sending
+// 16-byte units in flight per thread while sending: kSendShallow when each
+// thread sends at most that many, else kSendDeep (measured on B200, every
+// rank in one launch, graph-replayed: 8 ranks x B=256 H=64 D=128 took
+// 21.5 us at 8 against 22.8 us at 4; 2 ranks x B=1 H=2 D=64 took 3.5 us at
+// 4 against 3.7 us at 8).
+constexpr int kSendShallow = 4;
+constexpr int kSendDeep = 8;
 // Poll back-off of the landed-counter wait (measured on B200 with every rank
 // in one launch: 32..256 ns gave 4.43 us per call for 2 ranks of one head,
 // 64..2048 ns 4.53 us).
@@ -138,21 +141,24 @@ __device__ __forceinline__ void divmod(int64_t n, uint64_t c, int64_t d, int64_t
     r = (int64_t)((uint32_t)n - qq * (uint32_t)d);
 }
 
-// kSendUnroll units of one sending thread: units u, u + kThreads, ... .
+// UNROLL units of one sending thread: units u, u + kThreads, ... .
+template <int UNROLL>
 struct SendBatch {
-    uint4 x[kSendUnroll];
-    float lv[kSendUnroll];
-    int64_t rem[kSendUnroll];   // unit index inside the receiver's block
-    int64_t row[kSendUnroll];   // row (b * Hq + head) inside the receiver's block
-    int q[kSendUnroll];         // receiver, or -1 past the CTA's range
+    uint4 x[UNROLL];
+    float lv[UNROLL];
+    int64_t rem[UNROLL];   // unit index inside the receiver's block
+    int64_t row[UNROLL];   // row (b * Hq + head) inside the receiver's block
+    int q[UNROLL];         // receiver, or -1 past the CTA's range
 };
 
 // Load the partial columns (and, for a row's first column, the lse) of the
 // batch at u; nothing here depends on the call number.
+template <int UNROLL>
 __device__ __forceinline__ void load_batch(const CpParams& p, int me, int64_t u, int64_t u1,
-                                           const char* src_o, const float* src_l, SendBatch& sb) {
+                                           const char* src_o, const float* src_l,
+                                           SendBatch<UNROLL>& sb) {
 #pragma unroll
-    for (int k = 0; k < kSendUnroll; ++k) {
+    for (int k = 0; k < UNROLL; ++k) {
         const int64_t uk = u + (int64_t)k * kThreads;
         sb.q[k] = -1;
         sb.lv[k] = 0.f;
@@ -176,10 +182,11 @@ __device__ __forceinline__ void load_batch(const CpParams& p, int me, int64_t u,
 }
 
 // Store the batch into the receivers' slots of sender me, parity par.
+template <int UNROLL>
 __device__ __forceinline__ void store_batch(const CpParams& p, int me, int w1, int par,
-                                            const SendBatch& sb) {
+                                            const SendBatch<UNROLL>& sb) {
 #pragma unroll
-    for (int k = 0; k < kSendUnroll; ++k) {
+    for (int k = 0; k < UNROLL; ++k) {
         const int q = sb.q[k];
         if (q < 0) continue;
         const int slot = me - (me > q ? 1 : 0);   // sender slot at q
@@ -190,7 +197,7 @@ __device__ __forceinline__ void store_batch(const CpParams& p, int me, int w1, i
     }
 }
 
-template <typename TIn, typename TOut>
+template <typename TIn, typename TOut, int UNROLL>
 __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __grid_constant__ CpParams p) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
@@ -219,7 +226,7 @@ __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __gri
     const int64_t u0 = min(total, cta * p.chunk);
     const int64_t u1 = me == p.silent ? u0 : min(total, u0 + p.chunk);
     int64_t u = u0 + threadIdx.x;
-    SendBatch sb;
+    SendBatch<UNROLL> sb;
     load_batch(p, me, u, u1, src_o, src_l, sb);
     // Receive slot of this call.  Ranks on different GPUs alternate two slots
     // by the parity of e, so a rank may start call e + 1 while a peer still
@@ -234,7 +241,7 @@ __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __gri
     }
     for (;;) {
         store_batch(p, me, w1, par, sb);
-        u += (int64_t)kThreads * kSendUnroll;
+        u += (int64_t)kThreads * UNROLL;
         if (u >= u1) break;
         load_batch(p, me, u, u1, src_o, src_l, sb);
     }
@@ -350,20 +357,21 @@ __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __gri
 
 using CpFn = void (*)(CpParams);
 
-template <typename TIn>
+template <typename TIn, int UNROLL>
 CpFn pick_out(int out_dtype) {
     switch (out_dtype) {
-        case LSE_MERGE_F32: return cp_exchange_merge_kernel<TIn, float>;
-        case LSE_MERGE_F16: return cp_exchange_merge_kernel<TIn, __half>;
-        default: return cp_exchange_merge_kernel<TIn, __nv_bfloat16>;
+        case LSE_MERGE_F32: return cp_exchange_merge_kernel<TIn, float, UNROLL>;
+        case LSE_MERGE_F16: return cp_exchange_merge_kernel<TIn, __half, UNROLL>;
+        default: return cp_exchange_merge_kernel<TIn, __nv_bfloat16, UNROLL>;
     }
 }
 
+template <int UNROLL>
 CpFn pick_cp(int in_dtype, int out_dtype) {
     switch (in_dtype) {
-        case LSE_MERGE_F32: return pick_out<float>(out_dtype);
-        case LSE_MERGE_F16: return pick_out<__half>(out_dtype);
-        default: return pick_out<__nv_bfloat16>(out_dtype);
+        case LSE_MERGE_F32: return pick_out<float, UNROLL>(out_dtype);
+        case LSE_MERGE_F16: return pick_out<__half, UNROLL>(out_dtype);
+        default: return pick_out<__nv_bfloat16, UNROLL>(out_dtype);
     }
 }
 
@@ -452,19 +460,26 @@ int lse_merge_cp_exchange_merge(const lse_merge_cp_args* a, lse_merge_stream_t s
     kp.c_dv = fastdiv_c(kp.dv);
     kp.c_Hq = fastdiv_c((uint32_t)pl.Hq);
 
-    const CpFn fn = pick_cp(a->in_dtype, a->out_dtype);
-    int64_t capacity = 0;
-    const int ce = co_resident((const void*)fn, &capacity);
-    if (ce != 0) return fail_cuda(LSE_MERGE_ELAUNCH, ce);
-    const int64_t cap = capacity / a->rank_count;
-    if (cap < 1) return fail_cuda(LSE_MERGE_ELAUNCH, (int)cudaErrorCooperativeLaunchTooLarge);
     // One CTA per kThreads units of the larger phase, at most what is
-    // co-resident.
+    // co-resident; the deep send batch once a thread sends more units than
+    // the shallow one holds.
     const int64_t work = send_units > pl.U ? send_units : pl.U;
-    int64_t ctas = (work + kThreads - 1) / kThreads;
-    if (ctas > cap) ctas = cap;
-    if (ctas < 1) ctas = 1;
-    kp.chunk = (send_units + ctas - 1) / ctas;
+    CpFn fn = nullptr;
+    int64_t ctas = 0;
+    for (int deep = 0; deep < 2; ++deep) {
+        fn = deep ? pick_cp<kSendDeep>(a->in_dtype, a->out_dtype)
+                  : pick_cp<kSendShallow>(a->in_dtype, a->out_dtype);
+        int64_t capacity = 0;
+        const int ce = co_resident((const void*)fn, &capacity);
+        if (ce != 0) return fail_cuda(LSE_MERGE_ELAUNCH, ce);
+        const int64_t cap = capacity / a->rank_count;
+        if (cap < 1) return fail_cuda(LSE_MERGE_ELAUNCH, (int)cudaErrorCooperativeLaunchTooLarge);
+        ctas = (work + kThreads - 1) / kThreads;
+        if (ctas > cap) ctas = cap;
+        if (ctas < 1) ctas = 1;
+        kp.chunk = (send_units + ctas - 1) / ctas;
+        if (kp.chunk <= (int64_t)kSendShallow * kThreads) break;
+    }
     kp.share = kCallShares / (unsigned long long)ctas;
     kp.share0 = kCallShares - (unsigned long long)(ctas - 1) * kp.share;
 
