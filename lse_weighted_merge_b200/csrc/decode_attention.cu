@@ -211,17 +211,364 @@ constexpr int kModePartials = kAttnModePartials;
 constexpr int kModeCluster = kAttnModeCluster;
 constexpr int kModeWorkspace = kAttnModeWorkspace;
 
-template <typename T, int D, int MODE, typename TOut>
-__global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const AParams p) {
+// One work unit: split r of the keys of (batch b, KV head hk).  [lo, hi) are
+// its keys; `mine` is how many of its key tiles the calling warp takes (the
+// warps take tiles w, w + kAttnWarps, ...).
+struct Unit {
+    int b, hk, r, lo, hi, mine;
+    const char* kb;   // K of (b, hk)
+    const char* vb;   // V of (b, hk)
+};
+
+// Units are numbered with the split fastest, then the KV head, then the batch.
+__device__ __forceinline__ Unit unit_of(const AParams& p, int r, int hk, int b, int warp) {
+    constexpr int TK = kAttnTileKeys;
+    Unit x;
+    x.r = r;
+    x.hk = hk;
+    x.b = b;
+    int len = p.L;
+    if (p.kv_len) len = min(max(__ldg(p.kv_len + b), 0), p.L);
+    const int per = (len + p.R - 1) / p.R;
+    x.lo = min(len, r * per);
+    x.hi = min(len, x.lo + per);
+    const int ntiles = (x.hi - x.lo + TK - 1) / TK;
+    x.mine = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
+    x.kb = p.k + (int64_t)b * p.k_b + (int64_t)hk * p.k_h;
+    x.vb = p.v + (int64_t)b * p.v_b + (int64_t)hk * p.v_h;
+    return x;
+}
+
+// Q as the A operand of Q K^T: rows g and g+8 are query heads h0+g, h0+g+8
+// (zero beyond the group), columns 16*ks + 2t (+1) and + 8.
+template <int D>
+__device__ __forceinline__ void load_q(const AParams& p, int b, int h0, int g, int t,
+                                       uint32_t (&qa)[D / 16][4]) {
+    const char* qb = p.q + (int64_t)b * p.q_b;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        const int c0 = (ks * 16 + 2 * t) * 2;
+        qa[ks][0] = qa[ks][1] = qa[ks][2] = qa[ks][3] = 0u;
+        if (g < p.G) {
+            const char* row = qb + (int64_t)(h0 + g) * p.q_h;
+            qa[ks][0] = __ldg(reinterpret_cast<const unsigned int*>(row + c0));
+            qa[ks][2] = __ldg(reinterpret_cast<const unsigned int*>(row + c0 + 16));
+        }
+        if (g + 8 < p.G) {
+            const char* row = qb + (int64_t)(h0 + g + 8) * p.q_h;
+            qa[ks][1] = __ldg(reinterpret_cast<const unsigned int*>(row + c0));
+            qa[ks][3] = __ldg(reinterpret_cast<const unsigned int*>(row + c0 + 16));
+        }
+    }
+}
+
+// Copy key tile `i` of the calling warp in unit `x` (keys lo + (warp +
+// i*kAttnWarps)*TK ...) into the ring stage at shared address `kd` (K) and
+// kd + TILE (V); keys at or past hi are zero-filled.
+template <int D>
+__device__ __forceinline__ void issue_tile(const AParams& p, const Unit& x, int warp, int i,
+                                           uint32_t kd, int lane) {
+    constexpr int TK = kAttnTileKeys;
+    constexpr int CPR = D / 8;   // 16-byte chunks per K/V row
+    constexpr int TILE = TK * D * 2;
+    const int key0 = x.lo + (warp + i * kAttnWarps) * TK;
+    const uint32_t vd = kd + TILE;
+#pragma unroll 4
+    for (int c = lane; c < TK * CPR; c += 32) {
+        const int row = c / CPR, ch = c - row * CPR;
+        const int key = key0 + row;
+        const bool ok = key < x.hi;
+        const int64_t src_key = ok ? key : x.lo;
+        cp_async16(kd + tile_off<D>(row, ch), x.kb + src_key * p.k_l + ch * 16, ok ? 16 : 0);
+        cp_async16(vd + tile_off<D>(row, ch), x.vb + src_key * p.v_l + ch * 16, ok ? 16 : 0);
+    }
+}
+
+// The running state of a warp's online softmax over its key tiles: rows g
+// and g+8 of the 16-row tile, in log2 units.
+template <int D>
+struct WarpState {
+    float m0, m1;   // running max
+    float l0, l1;   // this thread's share of the running sums
+    float o[D / 8][4];
+    __device__ __forceinline__ void reset() {
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    }
+};
+
+// Fold one K/V tile (K at shared address ks_u, V at ks_u + TILE; first key
+// key0) into the warp's state: S = Q K^T, online softmax, O += P V.
+template <typename T, int D>
+__device__ __forceinline__ void attend_tile(uint32_t ks_u, const uint32_t (&qa)[D / 16][4],
+                                            int key0, int hi, float scale_log2, int lane,
+                                            WarpState<D>& w) {
+    constexpr int TK = kAttnTileKeys;
+    constexpr int KS = D / 16;   // k-steps of Q K^T
+    constexpr int NT = D / 8;    // n-tiles of P V
+    constexpr int TILE = TK * D * 2;
+    constexpr int NJ = TK / 8;   // n-tiles of Q K^T (8 keys each)
+    constexpr int KK = TK / 16;  // k-steps of P V (16 keys each)
+    const uint32_t vs_u = ks_u + TILE;
+    const int t = lane & 3;
+
+    // ---- S = Q K^T: NJ n-tiles of 8 keys
+    float sacc[NJ][4];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+        for (int jp = 0; jp < NJ / 2; ++jp) {
+            const int mi = lane >> 3, rr = lane & 7;
+            const int row = (2 * jp + (mi >> 1)) * 8 + rr;
+            const int ch = 2 * ks + (mi & 1);
+            uint32_t bf[4];
+            ldsm_x4(ks_u + tile_off<D>(row, ch), bf);
+            Mma<T>::run(sacc[2 * jp], qa[ks], bf[0], bf[1]);
+            Mma<T>::run(sacc[2 * jp + 1], qa[ks], bf[2], bf[3]);
+        }
+    }
+
+    // ---- online softmax over this tile (scores in log2 units)
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const bool ok = key0 + 8 * j + 2 * t + e < hi;
+            sacc[j][e] = ok ? sacc[j][e] * scale_log2 : -INFINITY;
+            sacc[j][e + 2] = ok ? sacc[j][e + 2] * scale_log2 : -INFINITY;
+            mx0 = fmaxf(mx0, sacc[j][e]);
+            mx1 = fmaxf(mx1, sacc[j][e + 2]);
+        }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
+    // every tile holds at least one valid key, so the new maxima are finite
+    const float n0 = fmaxf(w.m0, mx0), n1 = fmaxf(w.m1, mx1);
+    const float a0 = exp2f(w.m0 - n0), a1 = exp2f(w.m1 - n1);   // 0 on the first tile
+    w.m0 = n0;
+    w.m1 = n1;
+    w.l0 *= a0;
+    w.l1 *= a1;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        w.o[n][0] *= a0;
+        w.o[n][1] *= a0;
+        w.o[n][2] *= a1;
+        w.o[n][3] *= a1;
+    }
+    uint32_t pa[KK][4];   // P as the A operand of the 16-key k-steps
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+        const float p0 = exp2f(sacc[j][0] - n0), p1 = exp2f(sacc[j][1] - n0);
+        const float p2 = exp2f(sacc[j][2] - n1), p3 = exp2f(sacc[j][3] - n1);
+        w.l0 += p0 + p1;
+        w.l1 += p2 + p3;
+        pa[j >> 1][(j & 1) * 2 + 0] = Mma<T>::pack(p0, p1);
+        pa[j >> 1][(j & 1) * 2 + 1] = Mma<T>::pack(p2, p3);
+    }
+
+    // ---- O += P V: D/8 n-tiles, KK k-steps of 16 keys
+#pragma unroll
+    for (int kk = 0; kk < KK; ++kk) {
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+            const int mi = lane >> 3, rr = lane & 7;
+            const int row = 16 * kk + (mi & 1) * 8 + rr;
+            const int ch = 2 * np + (mi >> 1);
+            uint32_t bf[4];
+            ldsm_x4_t(vs_u + tile_off<D>(row, ch), bf);
+            Mma<T>::run(w.o[2 * np], pa[kk], bf[0], bf[1]);
+            Mma<T>::run(w.o[2 * np + 1], pa[kk], bf[2], bf[3]);
+        }
+    }
+}
+
+// Run the calling warp's share of unit `x`: its ring (shared address ring_u,
+// kAttnStages stages) already holds, or is being filled with, its first
+// kAttnStages - 1 tiles (one cp.async group each).  On return every copy of
+// the ring has landed and been read, and w holds the warp's state with the
+// sums l0, l1 complete over the quad.
+template <typename T, int D>
+__device__ __forceinline__ void attend_unit(const AParams& p, const Unit& x, int warp, int lane,
+                                            uint32_t ring_u, const uint32_t (&qa)[D / 16][4],
+                                            WarpState<D>& w) {
     constexpr int TK = kAttnTileKeys;
     constexpr int S = kAttnStages;
-    constexpr int KS = D / 16;         // k-steps of Q K^T
-    constexpr int NT = D / 8;          // n-tiles of P V
-    constexpr int CPR = D / 8;         // 16-byte chunks per K/V row
-    constexpr int TILE = TK * D * 2;   // bytes of one K (or V) tile
-    constexpr int NJ = TK / 8;         // n-tiles of Q K^T (8 keys each)
-    constexpr int KK = TK / 16;        // k-steps of P V (16 keys each)
-    static_assert(TK == 16 || TK == 32, "key tile of 16 or 32");
+    constexpr int TILE = TK * D * 2;
+    w.reset();
+    for (int i = 0; i < x.mine; ++i) {
+        if (i + S - 1 < x.mine)
+            issue_tile<D>(p, x, warp, i + S - 1, ring_u + (uint32_t)(((i + S - 1) % S) * 2 * TILE), lane);
+        cp_commit();
+        cp_wait<S - 1>();
+        __syncwarp();
+        const int key0 = x.lo + (warp + i * kAttnWarps) * TK;
+        attend_tile<T, D>(ring_u + (uint32_t)((i % S) * 2 * TILE), qa, key0, x.hi, p.scale_log2, lane, w);
+        __syncwarp();
+    }
+    cp_wait<0>();
+    __syncwarp();
+    w.l0 += __shfl_xor_sync(kFull, w.l0, 1);
+    w.l0 += __shfl_xor_sync(kFull, w.l0, 2);
+    w.l1 += __shfl_xor_sync(kFull, w.l1, 1);
+    w.l1 += __shfl_xor_sync(kFull, w.l1, 2);
+}
+
+// Issue the first kAttnStages - 1 tiles of the calling warp's share of unit
+// x into its ring, one cp.async group per stage (empty groups past `mine`).
+template <int D>
+__device__ __forceinline__ void issue_prologue(const AParams& p, const Unit& x, int warp, int lane,
+                                               uint32_t ring_u) {
+    constexpr int S = kAttnStages;
+    constexpr int TILE = kAttnTileKeys * D * 2;
+#pragma unroll
+    for (int s = 0; s < S - 1; ++s) {
+        if (s < x.mine) issue_tile<D>(p, x, warp, s, ring_u + (uint32_t)(s * 2 * TILE), lane);
+        cp_commit();
+    }
+}
+
+// Warp states in shared memory for the merge over the warps, G rows per
+// warp: m [kAttnWarps*G], l [kAttnWarps*G], o [kAttnWarps*G][D] (fp32).
+template <int D>
+__device__ __forceinline__ void store_warp_state(float* st, int G, int warp, int lane,
+                                                 const WarpState<D>& w) {
+    const int g = lane >> 2, t = lane & 3;
+    float* st_m = st;
+    float* st_l = st_m + kAttnWarps * G;
+    float* st_o = st_l + kAttnWarps * G;
+    if (t == 0) {
+        if (g < G) {
+            st_m[warp * G + g] = w.m0;
+            st_l[warp * G + g] = w.l0;
+        }
+        if (g + 8 < G) {
+            st_m[warp * G + g + 8] = w.m1;
+            st_l[warp * G + g + 8] = w.l1;
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+        if (g < G) {
+            float* o0 = st_o + (warp * G + g) * D + 8 * n + 2 * t;
+            o0[0] = w.o[n][0];
+            o0[1] = w.o[n][1];
+        }
+        if (g + 8 < G) {
+            float* o1 = st_o + (warp * G + g + 8) * D + 8 * n + 2 * t;
+            o1[0] = w.o[n][2];
+            o1[1] = w.o[n][3];
+        }
+    }
+}
+
+// The split's (o, lse) of element (gg, d): the LSE merge of the warps'
+// states (lse in natural-log units; an empty split gives 0 and -inf).
+template <int D>
+__device__ __forceinline__ void merge_warp_states(const float* st, int G, int gg, int d, float& o,
+                                                  float& lse) {
+    const float* st_m = st;
+    const float* st_l = st_m + kAttnWarps * G;
+    const float* st_o = st_l + kAttnWarps * G;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, st_m[w * G + gg]);
+    float den = 0.f, num = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) {
+            const float mw = st_m[w * G + gg];
+            if (mw != -INFINITY) {
+                const float e = exp2f(mw - M);
+                den += e * st_l[w * G + gg];
+                num += e * st_o[(w * G + gg) * D + d];
+            }
+        }
+    }
+    o = den > 0.f ? num / den : 0.f;
+    lse = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+}
+
+// Workspace form, in the CTA that brought the (b, KV head) counter to R:
+// merge the R split partials of the group (ws_o [R][G][D], ws_l [R][G],
+// written moments ago, so read through L2) into the output rows
+// rows_b .. rows_b + G - 1.  Each thread takes up to kMergeOut output
+// elements and walks the splits in batches of kMergeBatch, the lse and o
+// loads of a whole batch issued before any is used, then folded into a
+// running (max, weight sum, weighted sum) per element -- one L2 round trip
+// per batch, none for the weights alone.  An empty split has lse -inf, o 0.
+template <typename TOut, int D>
+__device__ __forceinline__ void merge_workspace(const AParams& p, const float* ws_o,
+                                                const float* ws_l, int64_t rows_b, int tid,
+                                                int nthr) {
+    constexpr int kMergeBatch = 4, kMergeOut = 4;
+    const int G = p.G, R = p.R;
+    const int GD = G * D;
+    for (int base = tid; base < GD; base += kMergeOut * nthr) {
+        float mx[kMergeOut], den[kMergeOut], num[kMergeOut];
+#pragma unroll
+        for (int k = 0; k < kMergeOut; ++k) {
+            mx[k] = -INFINITY;
+            den[k] = num[k] = 0.f;
+        }
+        for (int j0 = 0; j0 < R; j0 += kMergeBatch) {
+            float lv[kMergeOut][kMergeBatch], ov[kMergeOut][kMergeBatch];
+#pragma unroll
+            for (int k = 0; k < kMergeOut; ++k) {
+                const int idx = base + k * nthr;
+                const int gg = idx < GD ? idx / D : 0, d = idx - gg * D;
+#pragma unroll
+                for (int u = 0; u < kMergeBatch; ++u) {
+                    const int j = j0 + u;
+                    const bool in = idx < GD && j < R;
+                    lv[k][u] = in ? __ldcg(ws_l + j * G + gg) : -INFINITY;
+                    ov[k][u] = in ? __ldcg(ws_o + ((int64_t)j * G + gg) * D + d) : 0.f;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kMergeOut; ++k) {
+                float bm = mx[k];
+#pragma unroll
+                for (int u = 0; u < kMergeBatch; ++u) bm = fmaxf(bm, lv[k][u]);
+                const float ref = bm == -INFINITY ? 0.f : bm;
+                const float sc = expf(mx[k] - ref);   // 0 while nothing was seen
+                den[k] *= sc;
+                num[k] *= sc;
+#pragma unroll
+                for (int u = 0; u < kMergeBatch; ++u) {
+                    const float e = expf(lv[k][u] - ref);   // 0 for an empty split
+                    den[k] += e;
+                    num[k] = fmaf(e, ov[k][u], num[k]);
+                }
+                mx[k] = bm;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kMergeOut; ++k) {
+            const int idx = base + k * nthr;
+            if (idx < GD) {
+                const int gg = idx / D, d = idx - gg * D;
+                const int64_t row = rows_b + gg;
+                store_out<TOut>(p.out + (row * D + d) * (int64_t)sizeof(TOut),
+                                den[k] > 0.f ? num[k] / den[k] : 0.f);
+                if (d == 0) p.out_lse[row] = den[k] > 0.f ? mx[k] + logf(den[k]) : -INFINITY;
+            }
+        }
+    }
+}
+
+// One CTA per unit (grid R x Hkv x B); the cluster form needs this shape
+// (the R splits of a (b, KV head) are one cluster along x).
+template <typename T, int D, int MODE, typename TOut>
+__global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const AParams p) {
+    constexpr int TILE = kAttnTileKeys * D * 2;
     extern __shared__ __align__(128) unsigned char smem[];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -230,10 +577,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
     const int G = p.G, R = p.R;
     const int h0 = hk * G;
 
-    // Fused: CTA 0's receive buffer behind the ring and the warp states: the
-    // mbarrier (16 bytes), lse [R][G], then o [R][G][D] (fp32).  r is the
-    // CTA's rank in its cluster (the cluster spans the R splits along x).
-    constexpr int64_t kRing = (int64_t)kAttnWarps * S * 2 * TILE;
+    // Cluster: CTA 0's receive buffer behind the ring and the warp states:
+    // the mbarrier (16 bytes), lse [R][G], then o [R][G][D] (fp32).  r is
+    // the CTA's rank in its cluster (the cluster spans the R splits along x).
+    constexpr int64_t kRing = (int64_t)kAttnWarps * kAttnStages * 2 * TILE;
     constexpr int64_t kStates = (int64_t)kAttnWarps * 16 * (D + 2) * 4;
     constexpr int64_t kRecvOff = ((kRing > kStates ? kRing : kStates) + 15) / 16 * 16;
     const uint32_t bar = smem_u32(smem + kRecvOff);
@@ -252,179 +599,18 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
     pdl_wait();
     pdl_release();
 
-    int len = p.L;
-    if (p.kv_len) len = min(max(__ldg(p.kv_len + b), 0), p.L);
-    const int per = (len + R - 1) / R;
-    const int lo = min(len, r * per), hi = min(len, lo + per);
-    const int ntiles = (hi - lo + TK - 1) / TK;
-    const int mine = ntiles > warp ? (ntiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
-
-    const char* kb = p.k + (int64_t)b * p.k_b + (int64_t)hk * p.k_h;
-    const char* vb = p.v + (int64_t)b * p.v_b + (int64_t)hk * p.v_h;
-    unsigned char* ring = smem + (size_t)warp * S * 2 * TILE;
-    const uint32_t ring_u = smem_u32(ring);
-
-    // Q as the A operand: rows g and g+8 are query heads h0+g, h0+g+8 (zero
-    // beyond the group), columns 16*ks + 2t (+1) and + 8.
-    uint32_t qa[KS][4];
-    {
-        const char* qb = p.q + (int64_t)b * p.q_b;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            const int c0 = (ks * 16 + 2 * t) * 2;
-            qa[ks][0] = qa[ks][1] = qa[ks][2] = qa[ks][3] = 0u;
-            if (g < G) {
-                const char* row = qb + (int64_t)(h0 + g) * p.q_h;
-                qa[ks][0] = __ldg(reinterpret_cast<const unsigned int*>(row + c0));
-                qa[ks][2] = __ldg(reinterpret_cast<const unsigned int*>(row + c0 + 16));
-            }
-            if (g + 8 < G) {
-                const char* row = qb + (int64_t)(h0 + g + 8) * p.q_h;
-                qa[ks][1] = __ldg(reinterpret_cast<const unsigned int*>(row + c0));
-                qa[ks][3] = __ldg(reinterpret_cast<const unsigned int*>(row + c0 + 16));
-            }
-        }
-    }
-
-    // Copy key tile `i` of this warp (keys lo + (warp + i*kAttnWarps)*TK ...)
-    // into ring stage `s`; keys at or past `hi` are zero-filled.
-    auto issue = [&](int i, int s) {
-        const int key0 = lo + (warp + i * kAttnWarps) * TK;
-        const uint32_t kd = ring_u + (uint32_t)(s * 2 * TILE);
-        const uint32_t vd = kd + TILE;
-#pragma unroll 4
-        for (int c = lane; c < TK * CPR; c += 32) {
-            const int row = c / CPR, ch = c - row * CPR;
-            const int key = key0 + row;
-            const bool ok = key < hi;
-            const int64_t src_key = ok ? key : lo;
-            cp_async16(kd + tile_off<D>(row, ch), kb + src_key * p.k_l + ch * 16, ok ? 16 : 0);
-            cp_async16(vd + tile_off<D>(row, ch), vb + src_key * p.v_l + ch * 16, ok ? 16 : 0);
-        }
-    };
-
-    float m0 = -INFINITY, m1 = -INFINITY;   // running max (log2 units) of rows g, g+8
-    float l0 = 0.f, l1 = 0.f;               // this thread's share of the running sums
-    float oacc[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
-
-#pragma unroll
-    for (int s = 0; s < S - 1; ++s) {
-        if (s < mine) issue(s, s);
-        cp_commit();
-    }
-    for (int i = 0; i < mine; ++i) {
-        if (i + S - 1 < mine) issue(i + S - 1, (i + S - 1) % S);
-        cp_commit();
-        cp_wait<S - 1>();
-        __syncwarp();
-        const uint32_t ks_u = ring_u + (uint32_t)((i % S) * 2 * TILE);
-        const uint32_t vs_u = ks_u + TILE;
-        const int key0 = lo + (warp + i * kAttnWarps) * TK;
-
-        // ---- S = Q K^T: NJ n-tiles of 8 keys
-        float sacc[NJ][4];
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-#pragma unroll
-            for (int jp = 0; jp < NJ / 2; ++jp) {
-                const int mi = lane >> 3, rr = lane & 7;
-                const int row = (2 * jp + (mi >> 1)) * 8 + rr;
-                const int ch = 2 * ks + (mi & 1);
-                uint32_t bf[4];
-                ldsm_x4(ks_u + tile_off<D>(row, ch), bf);
-                Mma<T>::run(sacc[2 * jp], qa[ks], bf[0], bf[1]);
-                Mma<T>::run(sacc[2 * jp + 1], qa[ks], bf[2], bf[3]);
-            }
-        }
-
-        // ---- online softmax over this tile (scores in log2 units)
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const bool ok = key0 + 8 * j + 2 * t + e < hi;
-                sacc[j][e] = ok ? sacc[j][e] * p.scale_log2 : -INFINITY;
-                sacc[j][e + 2] = ok ? sacc[j][e + 2] * p.scale_log2 : -INFINITY;
-                mx0 = fmaxf(mx0, sacc[j][e]);
-                mx1 = fmaxf(mx1, sacc[j][e + 2]);
-            }
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
-        // every tile holds at least one valid key, so the new maxima are finite
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);   // 0 on the first tile
-        m0 = n0;
-        m1 = n1;
-        l0 *= a0;
-        l1 *= a1;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            oacc[n][0] *= a0;
-            oacc[n][1] *= a0;
-            oacc[n][2] *= a1;
-            oacc[n][3] *= a1;
-        }
-        uint32_t pa[KK][4];   // P as the A operand of the 16-key k-steps
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-            const float p0 = exp2f(sacc[j][0] - n0), p1 = exp2f(sacc[j][1] - n0);
-            const float p2 = exp2f(sacc[j][2] - n1), p3 = exp2f(sacc[j][3] - n1);
-            l0 += p0 + p1;
-            l1 += p2 + p3;
-            pa[j >> 1][(j & 1) * 2 + 0] = Mma<T>::pack(p0, p1);
-            pa[j >> 1][(j & 1) * 2 + 1] = Mma<T>::pack(p2, p3);
-        }
-
-        // ---- O += P V: D/8 n-tiles, KK k-steps of 16 keys
-#pragma unroll
-        for (int kk = 0; kk < KK; ++kk) {
-#pragma unroll
-            for (int np = 0; np < NT / 2; ++np) {
-                const int mi = lane >> 3, rr = lane & 7;
-                const int row = 16 * kk + (mi & 1) * 8 + rr;
-                const int ch = 2 * np + (mi >> 1);
-                uint32_t bf[4];
-                ldsm_x4_t(vs_u + tile_off<D>(row, ch), bf);
-                Mma<T>::run(oacc[2 * np], pa[kk], bf[0], bf[1]);
-                Mma<T>::run(oacc[2 * np + 1], pa[kk], bf[2], bf[3]);
-            }
-        }
-        __syncwarp();
-    }
-    cp_wait<0>();
-    l0 += __shfl_xor_sync(kFull, l0, 1);
-    l0 += __shfl_xor_sync(kFull, l0, 2);
-    l1 += __shfl_xor_sync(kFull, l1, 1);
-    l1 += __shfl_xor_sync(kFull, l1, 2);
+    const Unit x = unit_of(p, r, hk, b, warp);
+    const uint32_t ring_u = smem_u32(smem + (size_t)warp * kAttnStages * 2 * TILE);
+    uint32_t qa[D / 16][4];
+    load_q<D>(p, b, h0, g, t, qa);
+    issue_prologue<D>(p, x, warp, lane, ring_u);
+    WarpState<D> w;
+    attend_unit<T, D>(p, x, warp, lane, ring_u, qa, w);
     __syncthreads();   // every warp is done with its ring: reuse the shared memory
 
-    // ---- merge the warps' states: per warp m[16], l[16], O[16][D]
-    float* st_m = reinterpret_cast<float*>(smem);
-    float* st_l = st_m + kAttnWarps * 16;
-    float* st_o = st_l + kAttnWarps * 16;
-    if (t == 0) {
-        st_m[warp * 16 + g] = m0;
-        st_m[warp * 16 + g + 8] = m1;
-        st_l[warp * 16 + g] = l0;
-        st_l[warp * 16 + g + 8] = l1;
-    }
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        float* o0 = st_o + (warp * 16 + g) * D + 8 * n + 2 * t;
-        float* o1 = st_o + (warp * 16 + g + 8) * D + 8 * n + 2 * t;
-        o0[0] = oacc[n][0];
-        o0[1] = oacc[n][1];
-        o1[0] = oacc[n][2];
-        o1[1] = oacc[n][3];
-    }
+    // ---- merge the warps' states
+    float* st = reinterpret_cast<float*>(smem);
+    store_warp_state<D>(st, G, warp, lane, w);
     __syncthreads();
     const int64_t rows_b = (int64_t)b * p.Hq + h0;
     // Cluster: this split's partial goes to slot r of CTA 0's receive buffer.
@@ -448,23 +634,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
     }
     for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
         const int gg = idx / D, d = idx - gg * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, st_m[w * 16 + gg]);
-        float den = 0.f, num = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < kAttnWarps; ++w) {
-                const float mw = st_m[w * 16 + gg];
-                if (mw != -INFINITY) {
-                    const float e = exp2f(mw - M);
-                    den += e * st_l[w * 16 + gg];
-                    num += e * st_o[(w * 16 + gg) * D + d];
-                }
-            }
-        }
-        const float o = den > 0.f ? num / den : 0.f;
-        const float lse = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+        float o, lse;
+        merge_warp_states<D>(st, G, gg, d, o, lse);
         if constexpr (MODE != kModePartials) {
             dst_o[(r * G + gg) * D + d] = o;
             if (d == 0) dst_l[r * G + gg] = lse;
@@ -486,65 +657,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1) decode_attn_kernel(const A
         if (threadIdx.x == 0) s_last = atom_add_acq_rel_gpu(p.ws_cnt + bh, 1u) == (unsigned)(R - 1);
         __syncthreads();
         if (!s_last) return;
-        // The merge: each thread takes up to kMergeOut output elements and
-        // walks the splits in batches of kMergeBatch, the lse and o loads of a
-        // whole batch (L2: the partials were written moments ago) issued
-        // before any is used, then folded into a running (max, weight sum,
-        // weighted sum) per element -- one L2 round trip per batch, none
-        // for the weights alone.  An empty split has lse -inf and o 0.
-        constexpr int kMergeBatch = 4, kMergeOut = 4;
-        const int GD = G * D;
-        for (int base = threadIdx.x; base < GD; base += kMergeOut * blockDim.x) {
-            float mx[kMergeOut], den[kMergeOut], num[kMergeOut];
-#pragma unroll
-            for (int k = 0; k < kMergeOut; ++k) {
-                mx[k] = -INFINITY;
-                den[k] = num[k] = 0.f;
-            }
-            for (int j0 = 0; j0 < R; j0 += kMergeBatch) {
-                float lv[kMergeOut][kMergeBatch], ov[kMergeOut][kMergeBatch];
-#pragma unroll
-                for (int k = 0; k < kMergeOut; ++k) {
-                    const int idx = base + k * blockDim.x;
-                    const int gg = idx < GD ? idx / D : 0, d = idx - gg * D;
-#pragma unroll
-                    for (int u = 0; u < kMergeBatch; ++u) {
-                        const int j = j0 + u;
-                        const bool in = idx < GD && j < R;
-                        lv[k][u] = in ? __ldcg(dst_l + j * G + gg) : -INFINITY;
-                        ov[k][u] = in ? __ldcg(dst_o + ((int64_t)j * G + gg) * D + d) : 0.f;
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < kMergeOut; ++k) {
-                    float bm = mx[k];
-#pragma unroll
-                    for (int u = 0; u < kMergeBatch; ++u) bm = fmaxf(bm, lv[k][u]);
-                    const float ref = bm == -INFINITY ? 0.f : bm;
-                    const float sc = expf(mx[k] - ref);   // 0 while nothing was seen
-                    den[k] *= sc;
-                    num[k] *= sc;
-#pragma unroll
-                    for (int u = 0; u < kMergeBatch; ++u) {
-                        const float e = expf(lv[k][u] - ref);   // 0 for an empty split
-                        den[k] += e;
-                        num[k] = fmaf(e, ov[k][u], num[k]);
-                    }
-                    mx[k] = bm;
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < kMergeOut; ++k) {
-                const int idx = base + k * blockDim.x;
-                if (idx < GD) {
-                    const int gg = idx / D, d = idx - gg * D;
-                    const int64_t row = rows_b + gg;
-                    store_out<TOut>(p.out + (row * D + d) * (int64_t)sizeof(TOut),
-                                    den[k] > 0.f ? num[k] / den[k] : 0.f);
-                    if (d == 0) p.out_lse[row] = den[k] > 0.f ? mx[k] + logf(den[k]) : -INFINITY;
-                }
-            }
-        }
+        merge_workspace<TOut, D>(p, dst_o, dst_l, rows_b, threadIdx.x, blockDim.x);
         if (threadIdx.x == 0) p.ws_cnt[bh] = 0u;   // every split of this call has counted
     }
     if constexpr (MODE == kModeCluster) {
@@ -646,7 +759,6 @@ cudaError_t ensure_smem(AttnFn fn, int64_t bytes) {
         g_attr_done[g_attr_n++] = AttrDone{(const void*)fn, dev, bytes};
     return cudaSuccess;
 }
-
 
 int launch(const void* q, const void* k, const void* v, const int32_t* kv_len, int B, int Hq,
            int Hkv, int L, int D, int R, float scale, const lse_merge_attn_strides* strides,

@@ -307,8 +307,8 @@ int make_attn_plan(const void* q, const void* k, const void* v, int B, int Hq, i
             return LSE_MERGE_EALIAS;
     }
     const int64_t ring = (int64_t)kAttnWarps * kAttnStages * 2 * kAttnTileKeys * D * 2;
-    // after the key loop the ring is reused for each warp's state (16 rows of
-    // m, l and D accumulators)
+    // after the key loop the ring is reused for each warp's state (G <= 16
+    // rows of m, l and D accumulators; sized for 16)
     const int64_t states = (int64_t)kAttnWarps * 16 * (D + 2) * 4;
     const int64_t base = ((ring > states ? ring : states) + 15) / 16 * 16;
     // fused: behind them CTA 0's receive buffer of the R split partials (an

@@ -220,6 +220,27 @@ def test_ragged_and_empty_sequences():
         assert torch.all(out[1] == 0) and torch.all(lse[1] == -math.inf)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_many_units_ragged_lengths(D):
+    """Many (batch, KV head, split) units, several waves of CTAs, with ragged
+    lengths (empty, shorter than a tile, shorter than the split count) that
+    change the tile counts from unit to unit.  Every row is checked, fused
+    and unfused."""
+    from lse_weighted_merge_b200 import merge
+    B, Hq, Hkv, L, R = 96, 8, 2, 150, 8   # 1536 units
+    rng = np.random.Generator(np.random.PCG64(21 + D))
+    lens = [int(x) for x in rng.integers(0, L + 1, B)]
+    lens[:4] = [0, 1, 7, L]
+    q, k, v = make(B, Hq, Hkv, L, D, seed=23 + D)
+    scale = 1 / math.sqrt(D)
+    want, want_lse, vmax = reference(q, k, v, scale, lens)
+    out, lse = run(q, k, v, R, scale, kv_len=lens, mode="ws")
+    check_rows(out, lse, want, want_lse, vmax, "bf16", "bf16", "many units ws")
+    po, pl = run(q, k, v, R, scale, kv_len=lens, fused=False)
+    mo, ml = merge(po.cuda(), pl.cuda(), out_dtype=torch.bfloat16)
+    check_rows(mo.cpu(), ml.cpu(), want, want_lse, vmax, "bf16", "bf16", "many units partials")
+
+
 @pytest.mark.parametrize("mode", ["ws", "cluster"])
 @pytest.mark.parametrize("out_dt", ["bf16", "f16", "f32"])
 def test_fp16_inputs_and_out_dtypes(out_dt, mode):
@@ -296,12 +317,14 @@ def test_automatic_splits_and_fusion(B, Hq, Hkv, L):
     check_rows(out.cpu(), lse.cpu(), want, want_lse, vmax, "bf16", "bf16", "auto")
 
 
+@pytest.mark.parametrize("B", [2, 80])
 @pytest.mark.parametrize("fused", [True, "ws", False], ids=["cluster", "ws", "partials"])
-def test_outputs_written_exactly_in_bounds(fused):
+def test_outputs_written_exactly_in_bounds(fused, B):
     """Outputs (and the workspace) carved out of larger buffers with canary
     guard bytes: after a call no guard byte has changed and q, k, v are left
-    as they were."""
-    B, Hq, Hkv, L, D, R = 2, 8, 2, 300, 128, 4
+    as they were.  B=80 gives 640 units, more CTAs than the device holds
+    at once."""
+    Hq, Hkv, L, D, R = 8, 2, 300, 128, 4
     q, k, v = make(B, Hq, Hkv, L, D, seed=77)
     scale = 1 / math.sqrt(D)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
