@@ -683,7 +683,7 @@ def run_ours(args):
                 e = errs.get(wname)
                 if e:
                     row.update({"err": _r(e["max_scaled_err"], 3), "tol": e["tol"],
-                                "lse_err": _r(e["lse_err_over_bound"], 3), "ok": e["ok"]})
+                                "lse_over_bound": _r(e["lse_err_over_bound"], 3), "ok": e["ok"]})
         cpu = cpu_baselines(inp, max(1, w.B // 8), args.cpu_seconds)
 
     if dist is not None:
