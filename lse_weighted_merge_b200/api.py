@@ -249,8 +249,8 @@ def decode_attention(q, k, v, *, splits: int | None = None, scale: float | None 
     second launch overlaps the first one's drain).  fused=True: one launch;
     each shard's CTA writes its fp32 partial into a workspace kept for this
     device and stream, and the last shard of each (sequence, KV head) to
-    finish merges them (lse_merge_decode_attention_ws), within about 1 % of
-    the two launches.  fused="cluster": one launch in which the shards of a
+    finish merges them (lse_merge_decode_attention_ws), 1-3 % slower than
+    the two launches on large batches.  fused="cluster": one launch in which the shards of a
     (sequence, KV head) form a thread-block cluster and merge through
     distributed shared memory, no workspace (splits 1, 2, 4 or 8; cluster
     scheduling leaves SM slots idle, so it is slower on large batches).
