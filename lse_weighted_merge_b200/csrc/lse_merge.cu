@@ -31,6 +31,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "device_common.cuh"
 #include "lse_merge.h"
@@ -203,17 +204,21 @@ __global__ void __launch_bounds__(kBlock, kMinBlocksVec1) merge_vec1_kernel(cons
                 for (int i = 0; i < RC; ++i)
                     if (vlive && s0 + i < cn) x[i] = ld_stream16(orow + (int64_t)(c + s0 + i) * p.o_r);
             }
+            auto fold_chunk = [&](auto check) {
 #pragma unroll
-            for (int i = 0; i < RC; ++i) {
-                const float w = __shfl_sync(kFull, e, s0 + i, p.lanes);
-                if (s0 + i < cn && (!any_zero || w != 0.f)) {
-                    uint64_t xx[N2];
-                    Elem<TIn>::unpack2(x[i], xx);
-                    const uint64_t ww = pack2f(w, w);
+                for (int i = 0; i < RC; ++i) {
+                    const float w = __shfl_sync(kFull, e, s0 + i, p.lanes);
+                    if (s0 + i < cn && (!decltype(check)::value || w != 0.f)) {
+                        uint64_t xx[N2];
+                        Elem<TIn>::unpack2(x[i], xx);
+                        const uint64_t ww = pack2f(w, w);
 #pragma unroll
-                    for (int k = 0; k < N2; ++k) fma2(acc[k], xx[k], ww);
+                        for (int k = 0; k < N2; ++k) fma2(acc[k], xx[k], ww);
+                    }
                 }
-            }
+            };
+            if (any_zero) fold_chunk(std::true_type{});
+            else fold_chunk(std::false_type{});
         }
     }
     esum = group_sum(esum, p.lanes);
@@ -316,11 +321,15 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KPa
                         if (cl[k] && s0 + i < cn)
                             x[i][k] = ld_stream16(orow + (int64_t)(c + s0 + i) * p.o_r + k * p.lanes * 16);
             }
+            auto fold_chunk = [&](auto check) {
 #pragma unroll
-            for (int i = 0; i < RC; ++i) {
-                const float w = __shfl_sync(kFull, e, s0 + i, p.lanes);
-                if (s0 + i < cn && (!any_zero || w != 0.f)) fold<TIn, NV, N2>(acc, x[i], w);
-            }
+                for (int i = 0; i < RC; ++i) {
+                    const float w = __shfl_sync(kFull, e, s0 + i, p.lanes);
+                    if (s0 + i < cn && (!decltype(check)::value || w != 0.f)) fold<TIn, NV, N2>(acc, x[i], w);
+                }
+            };
+            if (any_zero) fold_chunk(std::true_type{});
+            else fold_chunk(std::false_type{});
         }
     }
     esum = group_sum(esum, p.lanes);
@@ -338,8 +347,15 @@ __global__ void __launch_bounds__(kBlock, kMinBlocks) merge_vec_kernel(const KPa
 // as partial i of the current slice has been folded into the accumulator,
 // its registers are refilled with partial i of the next slice, so every lane
 // keeps up to R*NV 16-byte loads in flight across slice boundaries and no
-// warp ever waits for a CTA to retire or launch.
-template <typename TIn, typename TOut, int RC, int NV>
+// warp ever waits for a CTA to retire or launch.  FULL: R == RC, so no
+// partial index needs a bound check.  A warp whose slices hold no empty
+// shard folds every partial without a per-partial test (the common case);
+// only a warp that has one checks each weight.  Measured on B200, back to
+// back: R=16 B=512 H=16 D=512 24.6 -> 22.2 us, rank-major R=8 B=256 H=64
+// D=128 7.7 -> 7.05 us (6.77 graph-replayed).  Refill loads of a column
+// outside the next slice are skipped, not redirected: redirecting every
+// lane's last refill to one shared address made a hot spot in L2 (30.2 us).
+template <typename TIn, typename TOut, int RC, int NV, bool FULL>
 __global__ void __launch_bounds__(kBlock, stream_min_blocks(RC, NV)) merge_stream_kernel(const KParams p, const int64_t G) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
@@ -350,9 +366,11 @@ __global__ void __launch_bounds__(kBlock, stream_min_blocks(RC, NV)) merge_strea
     const int64_t grp0 = t >> p.lg;
     const int64_t grp_w = (t & ~(int64_t)31) >> p.lg;
     const int64_t trips = grp_w < p.groups ? (p.groups - grp_w + G - 1) / G : 0;
+    const int R = FULL ? RC : p.R;
 
     struct Slice {
-        const char* o;
+        const char* o;    // this lane's first column of partial 0
+        const char* o0;   // column 0 of partial 0 of the row
         const float* l;
         int64_t row;
         int v0, slice;
@@ -368,9 +386,16 @@ __global__ void __launch_bounds__(kBlock, stream_min_blocks(RC, NV)) merge_strea
         s.v0 = ri.slice * p.lanes * NV + j;
 #pragma unroll
         for (int k = 0; k < NV; ++k) s.cl[k] = s.live && s.v0 + k * p.lanes < p.dv;
-        s.o = p.o + ri.b * p.o_b + ri.h * p.o_h + (int64_t)s.v0 * 16;
+        s.o0 = p.o + ri.b * p.o_b + ri.h * p.o_h;
+        s.o = s.o0 + (int64_t)s.v0 * 16;
         s.l = p.lse + ri.b * p.l_b + ri.h * p.l_h;
         return s;
+    };
+    // Partial i of slice s into x[i] (the columns inside the slice).
+    auto load = [&](uint4 (&xi)[NV], const Slice& s, int i) {
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (s.cl[k]) xi[k] = ld_stream16(s.o + (int64_t)i * p.o_r + k * p.lanes * 16);
     };
 
     Slice cur = locate(grp0);
@@ -381,44 +406,61 @@ __global__ void __launch_bounds__(kBlock, stream_min_blocks(RC, NV)) merge_strea
         for (int i = 0; i < RC; ++i)
 #pragma unroll
             for (int k = 0; k < NV; ++k)
-                if (s.cl[k] && i < p.R) prefetch_l2(s.o + (int64_t)i * p.o_r + k * p.lanes * 16);
-        if (s.live && j < p.R) prefetch_l2(s.l + (int64_t)j * p.l_r);
+                if (s.cl[k] && i < R) prefetch_l2(s.o + (int64_t)i * p.o_r + k * p.lanes * 16);
+        if (s.live && j < R) prefetch_l2(s.l + (int64_t)j * p.l_r);
     }
     pdl_wait();
     pdl_release();
+    // The first slice's loads go out without branches: a column outside the
+    // slice reads column 0 of the same partial row instead (never used; a
+    // different address for every row, so no L2 hot spot).  Measured:
+    // R=16 B=512 H=16 D=512 22.6 -> 22.2 us graph-replayed.
     uint4 x[RC][NV];
 #pragma unroll
     for (int i = 0; i < RC; ++i)
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
             x[i][k] = make_uint4(0u, 0u, 0u, 0u);
-            if (cur.cl[k] && i < p.R) x[i][k] = ld_stream16(cur.o + (int64_t)i * p.o_r + k * p.lanes * 16);
+            if (i < R)
+                x[i][k] = ld_stream16((cur.cl[k] ? cur.o + k * p.lanes * 16 : cur.o0) + (int64_t)i * p.o_r);
         }
-    float l = (cur.live && j < p.R) ? __ldg(cur.l + (int64_t)j * p.l_r) : -INFINITY;
+    float l = (cur.live && j < R) ? __ldg(cur.l + (int64_t)j * p.l_r) : -INFINITY;
 
     for (int64_t it = 0; it < trips; ++it) {
         const Slice nxt = locate(grp0 + (it + 1) * G);
-        const float ln = (nxt.live && j < p.R) ? __ldg(nxt.l + (int64_t)j * p.l_r) : -INFINITY;
+        const float ln = (nxt.live && j < R) ? __ldg(nxt.l + (int64_t)j * p.l_r) : -INFINITY;
 
         const float m = group_max(l, p.lanes);
         const float mref = (m == -INFINITY) ? 0.f : m;
         const float e = expf(l - mref);
         const float esum = group_sum(e, p.lanes);
-        const bool any_zero = __any_sync(kFull, j < p.R && e == 0.f);
+        const bool any_zero = __any_sync(kFull, j < R && e == 0.f);
 
         uint64_t acc[NV][N2];
 #pragma unroll
         for (int k = 0; k < NV; ++k)
 #pragma unroll
             for (int q = 0; q < N2; ++q) acc[k][q] = 0ull;
+        // The two loops are written out: the generic-lambda form of the
+        // other kernels measured 2-5 % slower here (rank-major R=8).
+        if (!any_zero) {
 #pragma unroll
-        for (int i = 0; i < RC; ++i) {
-            const float w = __shfl_sync(kFull, e, i, p.lanes);
-            if (i < p.R) {
-                if (!any_zero || w != 0.f) fold<TIn, NV, N2>(acc, x[i], w);
+            for (int i = 0; i < RC; ++i) {
+                const float w = __shfl_sync(kFull, e, i, p.lanes);
+                if (i < R) {
+                    fold<TIn, NV, N2>(acc, x[i], w);
+                    load(x[i], nxt, i);
+                }
+            }
+        } else {
+            // a partial of weight 0 may hold NaN: it must not reach the sum
 #pragma unroll
-                for (int k = 0; k < NV; ++k)
-                    if (nxt.cl[k]) x[i][k] = ld_stream16(nxt.o + (int64_t)i * p.o_r + k * p.lanes * 16);
+            for (int i = 0; i < RC; ++i) {
+                const float w = __shfl_sync(kFull, e, i, p.lanes);
+                if (i < R) {
+                    if (w != 0.f) fold<TIn, NV, N2>(acc, x[i], w);
+                    load(x[i], nxt, i);
+                }
             }
         }
         const float inv = esum > 0.f ? 1.f / esum : 0.f;
@@ -518,20 +560,36 @@ __global__ void __launch_bounds__(kBlock, stream_min_blocks(RC, 1)) merge_stream
             M = Mn;
             const int r0 = c * RC;
             const bool any_zero = __any_sync(kFull, j < RC && r0 + j < p.R && e == 0.f);
+            // written out like the persistent kernel's (the generic-lambda
+            // form measured 4 % slower at R=32)
+            if (!any_zero) {
 #pragma unroll
-            for (int i = 0; i < RC; ++i) {
-                const float w = __shfl_sync(kFull, e, i, p.lanes);
-                if (r0 + i < p.R) {
-                    if (!any_zero || w != 0.f) {
+                for (int i = 0; i < RC; ++i) {
+                    const float w = __shfl_sync(kFull, e, i, p.lanes);
+                    if (r0 + i < p.R) {
                         uint64_t xx[N2];
                         Elem<TIn>::unpack2(x[i], xx);
                         const uint64_t ww = pack2f(w, w);
 #pragma unroll
                         for (int q = 0; q < N2; ++q) fma2(acc[q], xx[q], ww);
                     }
+                    x[i] = make_uint4(0u, 0u, 0u, 0u);
+                    if (nxt.cl && rn + i < p.R) x[i] = ld_stream16(nxt.o + (int64_t)(rn + i) * p.o_r);
                 }
-                x[i] = make_uint4(0u, 0u, 0u, 0u);
-                if (nxt.cl && rn + i < p.R) x[i] = ld_stream16(nxt.o + (int64_t)(rn + i) * p.o_r);
+            } else {
+#pragma unroll
+                for (int i = 0; i < RC; ++i) {
+                    const float w = __shfl_sync(kFull, e, i, p.lanes);
+                    if (r0 + i < p.R && w != 0.f) {
+                        uint64_t xx[N2];
+                        Elem<TIn>::unpack2(x[i], xx);
+                        const uint64_t ww = pack2f(w, w);
+#pragma unroll
+                        for (int q = 0; q < N2; ++q) fma2(acc[q], xx[q], ww);
+                    }
+                    x[i] = make_uint4(0u, 0u, 0u, 0u);
+                    if (nxt.cl && rn + i < p.R) x[i] = ld_stream16(nxt.o + (int64_t)(rn + i) * p.o_r);
+                }
             }
             if (last) {
                 const float inv = es > 0.f ? 1.f / es : 0.f;
@@ -637,18 +695,22 @@ __global__ void __launch_bounds__(kWideWarps * 32) merge_wide_kernel(const KPara
         es = es * sc + group_sum(e, p.lanes);
         m = mn;
         const bool any_zero = __any_sync(kFull, j < RC && rj < p.R && e == 0.f);
+        auto fold_chunk = [&](auto check) {
 #pragma unroll
-        for (int i = 0; i < RC; ++i) {
-            const float w = __shfl_sync(kFull, e, i, p.lanes);
-            const int r = s + S * (bt * RC + i);
-            if (r < p.R && (!any_zero || w != 0.f)) {
-                uint64_t xx[N2];
-                Elem<TIn>::unpack2(x[i], xx);
-                const uint64_t ww = pack2f(w, w);
+            for (int i = 0; i < RC; ++i) {
+                const float w = __shfl_sync(kFull, e, i, p.lanes);
+                const int r = s + S * (bt * RC + i);
+                if (r < p.R && (!decltype(check)::value || w != 0.f)) {
+                    uint64_t xx[N2];
+                    Elem<TIn>::unpack2(x[i], xx);
+                    const uint64_t ww = pack2f(w, w);
 #pragma unroll
-                for (int q = 0; q < N2; ++q) fma2(acc[q], xx[q], ww);
+                    for (int q = 0; q < N2; ++q) fma2(acc[q], xx[q], ww);
+                }
             }
-        }
+        };
+        if (any_zero) fold_chunk(std::true_type{});
+        else fold_chunk(std::false_type{});
     }
     float f[N];
 #pragma unroll
@@ -937,26 +999,29 @@ StreamFn pick_stream_long(int rc, int in_dtype, int out_dtype) {
 }
 
 // (rc, nv) pairs the planner produces: rc * nv <= 16 loads of 16 bytes per lane.
-template <typename TIn, typename TOut>
+// FULL instantiations serve R == rc.
+template <typename TIn, typename TOut, bool FULL>
 StreamFn pick_stream_kernel(int rc, int nv) {
-    if (rc == 4) return nv == 4 ? merge_stream_kernel<TIn, TOut, 4, 4>
-                      : nv == 2 ? merge_stream_kernel<TIn, TOut, 4, 2> : merge_stream_kernel<TIn, TOut, 4, 1>;
-    if (rc == 8) return nv == 2 ? merge_stream_kernel<TIn, TOut, 8, 2> : merge_stream_kernel<TIn, TOut, 8, 1>;
-    return merge_stream_kernel<TIn, TOut, 16, 1>;
+    if constexpr (kMaxNv >= 4)
+        if (rc == 4 && nv == 4) return merge_stream_kernel<TIn, TOut, 4, 4, FULL>;
+    if (rc == 4) return nv == 2 ? merge_stream_kernel<TIn, TOut, 4, 2, FULL> : merge_stream_kernel<TIn, TOut, 4, 1, FULL>;
+    if (rc == 8) return nv == 2 ? merge_stream_kernel<TIn, TOut, 8, 2, FULL> : merge_stream_kernel<TIn, TOut, 8, 1, FULL>;
+    return merge_stream_kernel<TIn, TOut, 16, 1, FULL>;
 }
 template <typename TIn>
-StreamFn pick_stream_out(int rc, int nv, int out_dtype) {
+StreamFn pick_stream_out(int rc, int nv, bool full, int out_dtype) {
     switch (out_dtype) {
-        case LSE_MERGE_F32: return pick_stream_kernel<TIn, float>(rc, nv);
-        case LSE_MERGE_F16: return pick_stream_kernel<TIn, __half>(rc, nv);
-        default: return pick_stream_kernel<TIn, __nv_bfloat16>(rc, nv);
+        case LSE_MERGE_F32: return full ? pick_stream_kernel<TIn, float, true>(rc, nv) : pick_stream_kernel<TIn, float, false>(rc, nv);
+        case LSE_MERGE_F16: return full ? pick_stream_kernel<TIn, __half, true>(rc, nv) : pick_stream_kernel<TIn, __half, false>(rc, nv);
+        default: return full ? pick_stream_kernel<TIn, __nv_bfloat16, true>(rc, nv)
+                             : pick_stream_kernel<TIn, __nv_bfloat16, false>(rc, nv);
     }
 }
-StreamFn pick_stream(int rc, int nv, int in_dtype, int out_dtype) {
+StreamFn pick_stream(int rc, int nv, bool full, int in_dtype, int out_dtype) {
     switch (in_dtype) {
-        case LSE_MERGE_F32: return pick_stream_out<float>(rc, nv, out_dtype);
-        case LSE_MERGE_F16: return pick_stream_out<__half>(rc, nv, out_dtype);
-        default: return pick_stream_out<__nv_bfloat16>(rc, nv, out_dtype);
+        case LSE_MERGE_F32: return pick_stream_out<float>(rc, nv, full, out_dtype);
+        case LSE_MERGE_F16: return pick_stream_out<__half>(rc, nv, full, out_dtype);
+        default: return pick_stream_out<__nv_bfloat16>(rc, nv, full, out_dtype);
     }
 }
 
@@ -1099,7 +1164,7 @@ int run(const void* partial_o, const float* partial_lse, int R, int B, int H, in
     cudaError_t e;
     if (pl.path == LSE_MERGE_PATH_STREAM) {
         const StreamFn fn = R > pl.rc ? pick_stream_long(pl.rc, in_dtype, out_dtype)
-                                      : pick_stream(pl.rc, pl.nv, in_dtype, out_dtype);
+                                      : pick_stream(pl.rc, pl.nv, R == pl.rc, in_dtype, out_dtype);
         const int64_t want = (pl.groups * pl.lanes + pl.block - 1) / pl.block;
         int grid = 0;
         const int qe = persistent_grid((const void*)fn, pl.block, want, &grid);
