@@ -198,7 +198,7 @@ __device__ __forceinline__ void store_batch(const CpParams& p, int me, int w1, i
 }
 
 template <typename TIn, typename TOut, int UNROLL>
-__global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __grid_constant__ CpParams p) {
+__global__ void __launch_bounds__(kThreads, 2) cp_exchange_merge_kernel(const __grid_constant__ CpParams p) {
     constexpr int N = Elem<TIn>::kVec;
     constexpr int N2 = N / 2;
     const int pr = blockIdx.y;
@@ -294,34 +294,42 @@ __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __gri
     __syncthreads();
 
     // ---- 4. merge the owned rows over all senders (skipped after a timeout)
+    // A thread takes units w and w + stride together: the loads of both go
+    // out before either is merged, so twice as many are in flight.
     char* const dst_o = p.out_o[pr];
     float* const dst_l = p.out_lse[pr];
     const int64_t wend = s_ok ? p.U : 0;
-    for (int64_t w = cta * kThreads + threadIdx.x; w < wend; w += (int64_t)gridDim.x * kThreads) {
-        int64_t row, v, b, hq;
-        divmod(w, p.c_dv, p.dv, row, v);
-        divmod(row, p.c_Hq, p.Hq, b, hq);
-        const int64_t srow = b * p.H + (int64_t)me * p.Hq + hq;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    struct Unit {
+        int64_t w, row, v;
         uint4 x[kMaxWorld];
         float l[kMaxWorld];
+    };
+    auto load_unit = [&](Unit& u) {
+        int64_t b, hq;
+        divmod(u.w, p.c_dv, p.dv, u.row, u.v);
+        divmod(u.row, p.c_Hq, p.Hq, b, hq);
+        const int64_t srow = b * p.H + (int64_t)me * p.Hq + hq;
 #pragma unroll
         for (int s = 0; s < kMaxWorld; ++s) {
-            x[s] = make_uint4(0u, 0u, 0u, 0u);
-            l[s] = -INFINITY;
+            u.x[s] = make_uint4(0u, 0u, 0u, 0u);
+            u.l[s] = -INFINITY;
             if (s < p.world) {
                 if (s == me) {
-                    x[s] = ld_stream16(src_o + srow * p.rowbytes + v * 16);
-                    l[s] = __ldg(src_l + srow);
+                    u.x[s] = ld_stream16(src_o + srow * p.rowbytes + u.v * 16);
+                    u.l[s] = __ldg(src_l + srow);
                 } else {
                     const int64_t blk = (int64_t)par * w1 + (s - (s > me ? 1 : 0));
-                    x[s] = ld_cg16(mine + p.o_off + blk * p.slot_o + w * 16);
-                    l[s] = ld_cg_f32(reinterpret_cast<const float*>(mine + p.l_off + blk * p.slot_l) + row);
+                    u.x[s] = ld_cg16(mine + p.o_off + blk * p.slot_o + u.w * 16);
+                    u.l[s] = ld_cg_f32(reinterpret_cast<const float*>(mine + p.l_off + blk * p.slot_l) + u.row);
                 }
             }
         }
+    };
+    auto merge_unit = [&](const Unit& u) {
         float m = -INFINITY;
 #pragma unroll
-        for (int s = 0; s < kMaxWorld; ++s) m = fmaxf(m, l[s]);
+        for (int s = 0; s < kMaxWorld; ++s) m = fmaxf(m, u.l[s]);
         // An all-empty row has m = -inf; subtracting 0 keeps every weight
         // exp(-inf) = 0 instead of NaN.
         const float mref = (m == -INFINITY) ? 0.f : m;
@@ -331,11 +339,11 @@ __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __gri
         float esum = 0.f;
 #pragma unroll
         for (int s = 0; s < kMaxWorld; ++s) {
-            const float e = expf(l[s] - mref);   // 0 for an empty partial or s >= world
+            const float e = expf(u.l[s] - mref);   // 0 for an empty partial or s >= world
             esum += e;
-            if (e != 0.f) {                      // an empty partial's o (maybe NaN) is not read
+            if (e != 0.f) {                        // an empty partial's o (maybe NaN) is not read
                 uint64_t xx[N2];
-                Elem<TIn>::unpack2(x[s], xx);
+                Elem<TIn>::unpack2(u.x[s], xx);
                 const uint64_t ww = pack2f(e, e);
 #pragma unroll
                 for (int k = 0; k < N2; ++k) fma2(acc[k], xx[k], ww);
@@ -349,10 +357,19 @@ __global__ void __launch_bounds__(kThreads) cp_exchange_merge_kernel(const __gri
             f[2 * k] *= inv;
             f[2 * k + 1] *= inv;
         }
-        store_vec<TOut, N>(dst_o + w * N * (int64_t)sizeof(TOut), f);
-        if (v == 0) dst_l[row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+        store_vec<TOut, N>(dst_o + u.w * N * (int64_t)sizeof(TOut), f);
+        if (u.v == 0) dst_l[u.row] = esum > 0.f ? m + logf(esum) : -INFINITY;
+    };
+    for (int64_t w = cta * kThreads + threadIdx.x; w < wend; w += 2 * stride) {
+        Unit a, b;
+        a.w = w;
+        b.w = w + stride;
+        load_unit(a);
+        const bool two = b.w < wend;
+        if (two) load_unit(b);
+        merge_unit(a);
+        if (two) merge_unit(b);
     }
-
 }
 
 using CpFn = void (*)(CpParams);
