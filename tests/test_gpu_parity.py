@@ -63,6 +63,33 @@ def test_dtype_pairs(in_dt, out_dt):
         parity(inp, path=path, what=f"{in_dt}->{out_dt}/{path}")
 
 
+@pytest.mark.parametrize("R", [4, 8, 16])
+@pytest.mark.parametrize("in_dt,out_dt", [("f16", "f32"), ("f32", "bf16"), ("bf16", "f16"),
+                                          ("f32", "f32")])
+@pytest.mark.parametrize("poison", [False, True], ids=["no_empty", "empty_nan"])
+def test_stream_with_r_equal_to_its_partial_count(R, in_dt, out_dt, poison):
+    """R = 4, 8 or 16 on the persistent kernel runs its R == RC instantiation
+    (no partial-index checks).  Without empty shards every warp takes the
+    fold loop with no per-partial test; with NaN-poisoned empty shards and
+    all-empty rows the warps that hold one take the checked loop.  6144
+    rows, more slices than the full persistent grid has lane groups, so
+    lanes walk several slices; D=200 leaves lanes past the last column (the
+    first loads of those read column 0 of their row instead)."""
+    w = W["r4_b64_h32_d128_masked"]
+    kw = dict(R=R, B=256, H=24, D=200, in_dtype=in_dt, out_dtype=out_dt, seed=R * 31 + len(in_dt))
+    if not poison:
+        kw.update(empty_shard_p=0.0, empty_row_p=0.0)
+    inp = synth.make_inputs(w, poison_empty=poison, **kw)
+    rc, plan = nat.plan_query(0x7f0000000000, 0x7f1000000000, R, 256, 24, 200,
+                              (inp["o_strides"], inp["lse_strides"]), synth.DTYPES[in_dt],
+                              synth.DTYPES[out_dt], 0x7f2000000000, 0x7f3000000000,
+                              path=nat.PATH_STREAM)
+    assert rc == nat.OK and plan["rc"] == R
+    stats = parity(inp, path=nat.PATH_STREAM, what=f"R{R} {in_dt}->{out_dt} poison={poison}")
+    if poison:
+        assert stats["empty_rows"] > 0
+
+
 @pytest.mark.parametrize("R", [1, 2, 3, 5, 8, 9, 16, 17, 33, 40, 64, 100, 257])
 @pytest.mark.parametrize("D", [4, 8, 24, 64, 100, 128, 256, 264, 512, 1024])
 def test_ragged_shapes(R, D):
